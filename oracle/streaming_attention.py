@@ -1,0 +1,257 @@
+"""fp64 CPU statement of block-causal chunk attention over a streaming KV cache.
+
+TEST INFRASTRUCTURE (see the package docstring): plain numpy, one obvious step
+per line, no blocking or fusion beyond processing independent query rows in
+chunks to bound memory.
+
+What the pages fix (behaviour only, no formulas are printed):
+
+* "NVIDIA FlashDreams Is the Open-Source Inference Engine Robotics World Models
+  Needed", section Bounded Memory for Infinite Rollouts: each rollout keeps a
+  cache of bounded size and evicts old state, so a 10,000-step rollout does not
+  grow memory.  Section Hot-Path Generation, Background State Updates: the
+  denoising pass (generate) and the cache update (finalize) are separate.
+* "Cosmos3-H-Dreams" model card, Model Architecture: a block-causal, few-step
+  student with a KV cache; the conditioning frame is prefilled into the cache
+  once; each later latent frame consumes the next 4 action vectors.  Section
+  Software Integration: the KV cache has a static shape.
+* AlpaDreams GTC 2026 write-up, section VII: the causal DiT produces the next
+  frame from historical clean frames and the current noisy frame through a KV
+  cache.
+* "Single-GPU inference for DreamZero", Sequential requests: frame positions
+  and KV carry over between requests and are reset explicitly.
+
+Readings taken where the pages are silent:
+
+R1  scores are q.k / sqrt(d); softmax over the whole key set, no bias, no
+    softcap, no mask inside the key set.
+R2  the key set of every query of the current block is all valid cache tokens
+    plus all tokens of the current block (bidirectional inside the block; the
+    whole cache lies in the past of the block).
+R3  the first S frames committed to a rollout are sinks, never evicted; later
+    frames fill a ring of W window slots: slot_of(m) = m for m < S and
+    S + ((m - S) mod W) otherwise.  A commit of F <= W frames therefore evicts
+    the oldest window frames once the ring is full, and the valid slots are
+    always the prefix [0, min(n,S) + min(max(n-S,0), W)).
+R4  3D RoPE: the d/2 rotation pairs split into contiguous sections for t, h, w
+    of p_h = p_w = floor(d/6) pairs and p_t = d/2 - 2 floor(d/6) pairs; pair j
+    of a section of n_s pairs rotates the adjacent elements (2i, 2i+1) by the
+    angle coord * theta^(-j/n_s).
+R5  video token i of a frame sits at (h, w) = (i div Gw, i mod Gw); the action
+    tokens of a frame sit at (0, 0); every token of frame m has t = m.
+R6  t is the absolute frame index since the rollout's start (or last reset);
+    eviction never renumbers frames.
+R7  the cache keeps K/V exactly as committed (before RoPE) plus one int32 frame
+    position per slot (-1 = empty) and the committed-frame counter n; RoPE is
+    applied to cached keys when they are used.
+R8  the block being denoised has frames n .. n+F-1; its K/V are committed after
+    the last denoising step (whatever K/V the caller passes).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+# --------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact value of bfloat16 bit patterns.
+
+    A bfloat16 is the upper 16 bits of an IEEE-754 binary32, so placing the
+    pattern in the high half of a 32-bit word gives the same value exactly.
+    """
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def values_f64(x, dtype: str) -> np.ndarray:
+    """Stored inputs ("bf16" bit patterns or "f32" floats) as exact fp64 values."""
+    if dtype == "bf16":
+        return bf16_bits_to_f64(x)
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    raise ValueError(f"unknown dtype {dtype!r}")
+
+
+# --------------------------------------------------------------------------
+# 3D RoPE (readings R4, R5)
+# --------------------------------------------------------------------------
+def rope_sections(d: int):
+    """(p_t, p_h, p_w): rotation pairs given to the t, h and w axes (R4)."""
+    if d <= 0 or d % 2:
+        raise ValueError("head_dim must be a positive even number")
+    p_hw = d // 6
+    return d // 2 - 2 * p_hw, p_hw, p_hw
+
+
+def rope_inv_freq(n_pairs: int, theta: float) -> np.ndarray:
+    """Angular frequency of each pair of one section: theta^(-j/n_pairs) (R4)."""
+    j = np.arange(n_pairs, dtype=np.float64)
+    return np.power(float(theta), -j / n_pairs)
+
+
+def rope_angles(t, h, w, d: int, theta: float) -> np.ndarray:
+    """Rotation angle of every pair for tokens at coordinates (t, h, w).
+
+    t, h, w broadcast against each other; the result has one more trailing
+    axis of length d/2 ordered [t section | h section | w section].
+    """
+    p_t, p_h, p_w = rope_sections(d)
+    t = np.asarray(t, dtype=np.float64)[..., None]
+    h = np.asarray(h, dtype=np.float64)[..., None]
+    w = np.asarray(w, dtype=np.float64)[..., None]
+    a_t = t * rope_inv_freq(p_t, theta)
+    a_h = h * rope_inv_freq(p_h, theta)
+    a_w = w * rope_inv_freq(p_w, theta)
+    shape =np.broadcast_shapes(a_t.shape[:-1], a_h.shape[:-1], a_w.shape[:-1])
+    return np.concatenate([np.broadcast_to(a_t, shape + (p_t,)),
+                           np.broadcast_to(a_h, shape + (p_h,)),
+                           np.broadcast_to(a_w, shape + (p_w,))], axis=-1)
+
+
+def rope_rotate(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
+    """Rotate adjacent pairs (x[2i], x[2i+1]) of the last axis by angles[..., i]."""
+    x = np.asarray(x, dtype=np.float64)
+    c = np.cos(angles)
+    s = np.sin(angles)
+    x0 = x[..., 0::2]
+    x1 = x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, c.shape[:-1] + (x.shape[-1],)),
+                   dtype=np.float64)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+def token_coords(n_tokens: int, T: int, grid_w: int):
+    """(h, w) of the tokens of one frame (R5): video tokens row-major, actions at 0."""
+    i = np.arange(n_tokens)
+    h = np.where(i < T, i // grid_w, 0)
+    w = np.where(i < T, i % grid_w, 0)
+    return h, w
+
+
+# --------------------------------------------------------------------------
+# bounded streaming cache (readings R3, R6, R7)
+# --------------------------------------------------------------------------
+def slot_of(m: int, S: int, W: int) -> int:
+    """Cache slot of frame m of a rollout (R3)."""
+    if m < S:
+        return m
+    return S + (m - S) % W
+
+
+def valid_slot_count(n: int, S: int, W: int) -> int:
+    """Number of valid slots after n committed frames; they form a prefix (R3)."""
+    return min(n, S) + min(max(n - S, 0), W)
+
+
+class RolloutCache:
+    """Cache of one (rollout, layer): raw K/V per slot, positions and counter."""
+
+    def __init__(self, S: int, W: int, frame_tokens: int, heads: int,
+                 head_dim: int, dtype: str):
+        if W < 1 or S < 0:
+            raise ValueError("need W >= 1 and S >= 0")
+        self.S, self.W, self.dtype = S, W, dtype
+        store = np.uint16 if dtype == "bf16" else np.float32
+        shape = (S + W, frame_tokens, heads, head_dim)
+        self.k = np.zeros(shape, dtype=store)
+        self.v = np.zeros(shape, dtype=store)
+        self.pos = np.full(S + W, -1, dtype=np.int32)
+        self.n = 0
+
+    def reset(self) -> None:
+        """Start a new sequence: no valid frame, positions restart at 0."""
+        self.k[...] = 0
+        self.v[...] = 0
+        self.pos[:] = -1
+        self.n = 0
+
+    def commit(self, k_frames: np.ndarray, v_frames: np.ndarray) -> None:
+        """Write frames n, n+1, ... into their slots (R3, R8); n grows by their count.
+
+        k_frames, v_frames: [frames][Tf][H][d] in storage form, pre-RoPE.
+        """
+        nf = k_frames.shape[0]
+        if nf > self.W:
+            raise ValueError("a commit may not hold more frames than the window")
+        for f in range(nf):
+            s = slot_of(self.n + f, self.S, self.W)
+            self.k[s] = k_frames[f]
+            self.v[s] = v_frames[f]
+            self.pos[s] = self.n + f
+        self.n += nf
+
+    def valid_slots(self) -> int:
+        return valid_slot_count(self.n, self.S, self.W)
+
+
+# --------------------------------------------------------------------------
+# one attention call (readings R1, R2, R4-R8)
+# --------------------------------------------------------------------------
+def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
+                    theta: float, heads=None, row_chunk: int = 512,
+                    return_probs: bool = False):
+    """Attention of the current block's queries of one (rollout, layer).
+
+    q:    [F*T][H][d]  queries of the block, storage form, pre-RoPE
+    k, v: [F*Tf][H][d] keys / values of the block, storage form, pre-RoPE
+    cache: the rollout's cache for this layer (not modified)
+    heads: optional subset of head indices to evaluate (others are left 0)
+
+    Returns (out [F*T][H][d] fp64, lse [H][F*T] fp64 natural-log sum of exp of
+    the scaled scores) and, with return_probs, a dict head -> P [F*T][Nk].
+    """
+    dtype = cache.dtype
+    T = tokens
+    Mq, H, d = q.shape
+    F = Mq // T
+    if F * T != Mq or k.shape[0] % F:
+        raise ValueError("q rows must be F*T and k rows F*Tf")
+    Tf = k.shape[0] // F
+    n = cache.n
+    nv = cache.valid_slots()
+
+    # coordinates of every key: valid cache slots in slot order, then the block
+    h_tok, w_tok = token_coords(Tf, T, grid_w)
+    t_cache = np.repeat(cache.pos[:nv].astype(np.float64), Tf)
+    t_block = np.repeat(np.arange(n, n + F, dtype=np.float64), Tf)
+    t_key = np.concatenate([t_cache, t_block])
+    h_key = np.tile(h_tok, nv + F)
+    w_key = np.tile(w_tok, nv + F)
+    ang_k = rope_angles(t_key, h_key, w_key, d, theta)          # [Nk][d/2]
+
+    # coordinates of every query (video tokens only)
+    rows = np.arange(Mq)
+    tok_q = rows % T
+    ang_q = rope_angles(n + rows // T, tok_q // grid_w, tok_q % grid_w, d, theta)
+
+    scale = 1.0 / math.sqrt(d)
+    out = np.zeros((Mq, H, d), dtype=np.float64)
+    lse = np.zeros((H, Mq), dtype=np.float64)
+    probs = {}
+    for hh in (range(H) if heads is None else heads):
+        qh = rope_rotate(values_f64(q[:, hh, :], dtype), ang_q)
+        kc = values_f64(cache.k[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
+        vc = values_f64(cache.v[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
+        kh = rope_rotate(np.concatenate([kc, values_f64(k[:, hh, :], dtype)]), ang_k)
+        vh = np.concatenate([vc, values_f64(v[:, hh, :], dtype)])
+        if return_probs:
+            probs[hh] = np.zeros((Mq, kh.shape[0]), dtype=np.float64)
+        for r0 in range(0, Mq, row_chunk):
+            r1 = min(Mq, r0 + row_chunk)
+            s = (qh[r0:r1] @ kh.T) * scale
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            out[r0:r1, hh, :] = (e @ vh) / l
+            lse[hh, r0:r1] = (m + np.log(l))[:, 0]
+            if return_probs:
+                probs[hh][r0:r1] = e / l
+    if return_probs:
+        return out, lse, probs
+    return out, lse
