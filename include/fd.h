@@ -1,0 +1,201 @@
+/*
+ * fd.h -- C ABI of the B200 (sm_100a) streaming chunk-attention library.
+ *
+ * One hot path: block-causal chunk attention over a bounded per-rollout KV
+ * cache (sink frames + rolling window ring buffer) with 3D (t,h,w) RoPE on
+ * Q and K, plus the ring-buffer commit that evicts the oldest window frame.
+ *
+ * Sources for the behaviour (the pages describe it in prose; no formula is
+ * printed):
+ *   [FD-BM]  "NVIDIA FlashDreams Is the Open-Source Inference Engine Robotics
+ *            World Models Needed", section Bounded Memory for Infinite
+ *            Rollouts: per-rollout cache of bounded size with eviction.
+ *   [FD-HP]  same page, section Hot-Path Generation, Background State
+ *            Updates: generate() (denoising) vs finalize() (cache update).
+ *   [C3-MA]  "Cosmos3-H-Dreams" model card, Model Architecture: block-causal
+ *            few-step student with a KV cache; conditioning frame prefilled
+ *            once; each latent frame consumes 4 action vectors.
+ *   [C3-SI]  "Cosmos3-H-Dreams" model card, Software Integration: static-shape
+ *            KV cache, CUDA Graphs.
+ *   [AD-VII] AlpaDreams GTC 2026 write-up, section VII: causal DiT attends to
+ *            historical clean frames and the current noisy frame via a KV cache.
+ *   [DZ-SR]  "Single-GPU inference for DreamZero", Sequential requests: KV and
+ *            frame positions carry over between requests; explicit reset.
+ *
+ * Readings where the pages are silent (the same ones the test oracle states):
+ *   - scores q.k/sqrt(d), softmax over the whole key set, no bias or mask
+ *     inside it; key set = valid cache tokens + every token of the block;
+ *   - the first S frames of a rollout are sinks (never evicted); later frames
+ *     go to slot S + ((m - S) mod W) of a W-slot ring; valid slots are always
+ *     a prefix of the slot array;
+ *   - 3D RoPE: pairs (2i, 2i+1) of the head dimension; the d/2 pairs split
+ *     into contiguous t | h | w sections of d/2 - 2*floor(d/6), floor(d/6),
+ *     floor(d/6) pairs; pair j of a section of n pairs turns by
+ *     coord * theta^(-j/n); video token i of a frame is at
+ *     (h, w) = (i / grid_w, i % grid_w), action tokens at (0, 0); t is the
+ *     absolute frame index since the last reset;
+ *   - the cache stores K/V as committed (pre-RoPE) plus an int32 frame
+ *     position per slot; RoPE is applied to cached keys as they are loaded.
+ *
+ * Conventions for every call:
+ *   - all pointers to tensors are DEVICE pointers on the device that owns the
+ *     cache storage; host arrays are marked (host);
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
+ *     every call only enqueues work on it: no host synchronisation, no
+ *     allocation, so a block of calls can be captured in a CUDA graph;
+ *   - argument and shape errors return a status before anything is launched;
+ *   - layouts are dense row-major, token-major then head then dim ("BSHD");
+ *   - bf16 tensors are raw bfloat16 (uint16 bit patterns); f32 are IEEE float.
+ */
+#ifndef FD_H_
+#define FD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FD_OK = 0,
+  FD_ERR_INVALID_ARG = 1,     /* null pointer, index out of range           */
+  FD_ERR_SHAPE = 2,           /* descriptor or call shape not allowed       */
+  FD_ERR_DTYPE = 3,           /* dtype not known                            */
+  FD_ERR_CAPACITY = 4,        /* storage too small / too many frames        */
+  FD_ERR_CUDA = 5,            /* a CUDA runtime or driver call failed       */
+  FD_ERR_DEVICE_TIMEOUT = 6,  /* a device-side wait gave up (see below)     */
+  FD_ERR_UNSUPPORTED = 7,     /* valid request this build does not handle   */
+  FD_ERR_ALIGNMENT = 8        /* a tensor base is not 16-byte aligned       */
+} fd_status;
+
+typedef enum { FD_BF16 = 0, FD_F32 = 1 } fd_dtype;
+
+/* Geometry of one cache.  T = grid_h*grid_w video tokens per latent frame;
+ * Tf = T + action_tokens key/value tokens per frame ([C3-MA]: 4 action
+ * vectors per latent frame).  Requires 1 <= block_frames <= window_frames,
+ * sink_frames >= 0, head_dim even and a multiple of 8. */
+typedef struct {
+  int32_t num_layers;     /* L: one independent cache per layer            */
+  int32_t max_rollouts;   /* R: concurrent rollouts, each with its own cache */
+  int32_t num_heads;      /* H (query heads = key/value heads)             */
+  int32_t head_dim;       /* d                                             */
+  int32_t grid_h;         /* latent grid height                            */
+  int32_t grid_w;         /* latent grid width                             */
+  int32_t action_tokens;  /* A extra K/V tokens per frame (no queries)     */
+  int32_t block_frames;   /* F latent frames denoised together             */
+  int32_t sink_frames;    /* S frames kept for the whole rollout           */
+  int32_t window_frames;  /* W rolling window frames                       */
+  float rope_theta;       /* RoPE base (1e4 in every shipped workload)     */
+  int32_t dtype;          /* fd_dtype of q, k, v, out and the cache        */
+} fd_cache_desc;
+
+/* Byte offsets of the regions inside the caller's storage buffer.
+ *   k, v : [L][R][S+W][Tf][H][d] elements of `dtype`
+ *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
+ *   count: [L][R] int32, frames committed since the last reset (n)
+ *   ttab : [L][R][S+W+F][p_t] float2 (cos, sin) of the t-section angles for
+ *          every slot's frame and for the next block's frames n..n+F-1
+ *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
+ *   err  : int32 device error word (0 = none)                            */
+typedef struct {
+  size_t k, v, pos, count, ttab, htab, wtab, err;
+  size_t total;           /* == fd_cache_bytes(desc)                       */
+  size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
+  int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
+} fd_cache_layout;
+
+typedef struct fd_cache fd_cache;
+
+/* Bytes of device storage a cache with this geometry needs; 0 if the
+ * descriptor is invalid.  Pure host function. */
+size_t fd_cache_bytes(const fd_cache_desc* desc);
+
+/* Region offsets of the storage layout above.  Pure host function. */
+fd_status fd_cache_get_layout(const fd_cache_desc* desc, fd_cache_layout* out);
+
+/* Bind a cache object to caller-owned device storage of at least
+ * fd_cache_bytes(desc) bytes (base 1024-byte aligned).  Clears the storage,
+ * marks every slot empty, sets every counter to 0 and builds the RoPE tables,
+ * then synchronises the device once.  The library allocates no device
+ * memory, here or later: memory stays constant over unbounded rollouts
+ * ([FD-BM], [C3-SI]).  The host object is freed by fd_cache_destroy. */
+fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
+                          size_t bytes, fd_cache** out);
+
+/* Frees the host object only; the storage stays the caller's. */
+fd_status fd_cache_destroy(fd_cache* cache);
+
+/* Copy of the descriptor / layout a cache was created with. */
+fd_status fd_cache_get_desc(const fd_cache* cache, fd_cache_desc* out);
+fd_status fd_cache_layout_of(const fd_cache* cache, fd_cache_layout* out);
+
+/* Start a new sequence for the listed rollouts in every layer ([DZ-SR]):
+ * counter n = 0, every slot empty (pos = -1), K/V of those rollouts zeroed,
+ * t tables rebuilt for frames 0..F-1.  rollout_ids (host) [n_ids], each in
+ * [0, max_rollouts). */
+fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
+                         int32_t n_ids, void* stream);
+
+/* 3D RoPE in place on a block tensor x of rollouts 0..n_rollouts-1:
+ *   x: [n_rollouts][F][tokens_per_frame][H][d] of the cache dtype;
+ *   tokens_per_frame = T (queries) or Tf (keys, action tokens at (t,0,0));
+ * frame f of rollout r is at t = n_r + f with n_r that rollout's counter at
+ * `layer`, i.e. the positions fd_block_attention gives the block.  This is the
+ * same rotation fd_block_attention applies internally; it is exported for
+ * callers that need rotated tensors and for tests. */
+fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
+                    void* x, int32_t tokens_per_frame, void* stream);
+
+/* One denoising-step attention call for `layer` ([C3-MA], [AD-VII]):
+ *   q   : [n_rollouts][F*T][H][d]   queries of the block, pre-RoPE
+ *   k, v: [n_rollouts][F*Tf][H][d]  keys/values of the block, pre-RoPE
+ *   out : [n_rollouts][F*T][H][d]   softmax(q'k'^T/sqrt(d)) v
+ *   lse : [n_rollouts][H][F*T] fp32 natural-log sum of exp of the scaled
+ *         scores, or NULL
+ * For rollout r the key set is its valid cache slots (sinks + window, frame
+ * positions from the slot table) plus all F*Tf block tokens at t = n_r + f.
+ * The cache is read only: call it once per denoising step, then commit.
+ * bf16 runs on tcgen05 tensor cores (fp32 accumulation, P rounded to bf16),
+ * f32 on CUDA cores in fp32 (no TF32).  Tensor bases must be 16-byte aligned.
+ * Device-side waits are bounded: a wait that gives up sets the error word
+ * (fd_get_device_error) instead of hanging. */
+fd_status fd_block_attention(fd_cache* cache, int32_t layer,
+                             int32_t n_rollouts, const void* q, const void* k,
+                             const void* v, void* out, float* lse,
+                             void* stream);
+
+/* Ring-buffer commit for layers [layer_begin, layer_end) -- the finalize()
+ * half of [FD-HP]:  for every rollout r < n_rollouts and f < frames_r,
+ * slot = slot_of(n_r + f) receives frame f of k[l]/v[l] bit for bit,
+ * pos[slot] = n_r + f; then n_r += frames_r and the rollout's t table is
+ * rebuilt.  Once the window is full this evicts the oldest window frames.
+ *   frames (host) [n_rollouts], each in [0, F]; NULL = F for every rollout
+ *   (a ragged prefill commits fewer frames for some rollouts);
+ *   k, v (host arrays of device pointers) [layer_end - layer_begin], each
+ *   [n_rollouts][F*Tf][H][d] pre-RoPE (in practice the last step's k/v). */
+fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,
+                          int32_t layer_end, int32_t n_rollouts,
+                          const int32_t* frames, const void* const* k,
+                          const void* const* v, void* stream);
+
+/* Host mirror of a rollout's counter (updated by commit/reset calls). */
+fd_status fd_cache_frames(const fd_cache* cache, int32_t layer,
+                          int32_t rollout, int64_t* n);
+
+/* Reads (synchronously) and clears the device error word.  *code = 0 when no
+ * device-side check fired; otherwise bits 0-7 give the kind (1 = a bounded
+ * wait gave up) and bits 8-15 the site.  Returns FD_ERR_DEVICE_TIMEOUT when
+ * *code != 0. */
+fd_status fd_get_device_error(fd_cache* cache, int32_t* code);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t fd_launch_count(void);
+
+const char* fd_status_string(fd_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FD_H_ */

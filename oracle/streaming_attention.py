@@ -106,7 +106,7 @@ def rope_angles(t, h, w, d: int, theta: float) -> np.ndarray:
     a_t = t * rope_inv_freq(p_t, theta)
     a_h = h * rope_inv_freq(p_h, theta)
     a_w = w * rope_inv_freq(p_w, theta)
-    shape =np.broadcast_shapes(a_t.shape[:-1], a_h.shape[:-1], a_w.shape[:-1])
+    shape = np.broadcast_shapes(a_t.shape[:-1], a_h.shape[:-1], a_w.shape[:-1])
     return np.concatenate([np.broadcast_to(a_t, shape + (p_t,)),
                            np.broadcast_to(a_h, shape + (p_h,)),
                            np.broadcast_to(a_w, shape + (p_w,))], axis=-1)
@@ -194,7 +194,7 @@ class RolloutCache:
 # one attention call (readings R1, R2, R4-R8)
 # --------------------------------------------------------------------------
 def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
-                    theta: float, heads=None, row_chunk: int = 512,
+                    theta: float, heads=None, rows=None, row_chunk: int = 512,
                     return_probs: bool = False):
     """Attention of the current block's queries of one (rollout, layer).
 
@@ -202,6 +202,8 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     k, v: [F*Tf][H][d] keys / values of the block, storage form, pre-RoPE
     cache: the rollout's cache for this layer (not modified)
     heads: optional subset of head indices to evaluate (others are left 0)
+    rows:  optional subset of query rows to evaluate (others are left 0);
+           every row's softmax still runs over the whole key set
 
     Returns (out [F*T][H][d] fp64, lse [H][F*T] fp64 natural-log sum of exp of
     the scaled scores) and, with return_probs, a dict head -> P [F*T][Nk].
@@ -225,8 +227,8 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     w_key = np.tile(w_tok, nv + F)
     ang_k = rope_angles(t_key, h_key, w_key, d, theta)          # [Nk][d/2]
 
-    # coordinates of every query (video tokens only)
-    rows = np.arange(Mq)
+    # coordinates of the evaluated queries (video tokens only)
+    rows = np.arange(Mq) if rows is None else np.asarray(rows, dtype=np.int64)
     tok_q = rows % T
     ang_q = rope_angles(n + rows // T, tok_q // grid_w, tok_q % grid_w, d, theta)
 
@@ -235,23 +237,23 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     lse = np.zeros((H, Mq), dtype=np.float64)
     probs = {}
     for hh in (range(H) if heads is None else heads):
-        qh = rope_rotate(values_f64(q[:, hh, :], dtype), ang_q)
+        qh = rope_rotate(values_f64(q[rows, hh, :], dtype), ang_q)
         kc = values_f64(cache.k[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
         vc = values_f64(cache.v[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
         kh = rope_rotate(np.concatenate([kc, values_f64(k[:, hh, :], dtype)]), ang_k)
         vh = np.concatenate([vc, values_f64(v[:, hh, :], dtype)])
         if return_probs:
             probs[hh] = np.zeros((Mq, kh.shape[0]), dtype=np.float64)
-        for r0 in range(0, Mq, row_chunk):
-            r1 = min(Mq, r0 + row_chunk)
-            s = (qh[r0:r1] @ kh.T) * scale
+        for c0 in range(0, len(rows), row_chunk):
+            sel = rows[c0:c0 + row_chunk]
+            s = (qh[c0:c0 + row_chunk] @ kh.T) * scale
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             l = e.sum(axis=1, keepdims=True)
-            out[r0:r1, hh, :] = (e @ vh) / l
-            lse[hh, r0:r1] = (m + np.log(l))[:, 0]
+            out[sel, hh, :] = (e @ vh) / l
+            lse[hh, sel] = (m + np.log(l))[:, 0]
             if return_probs:
-                probs[hh][r0:r1] = e / l
+                probs[hh][sel] = e / l
     if return_probs:
         return out, lse, probs
     return out, lse

@@ -1,0 +1,218 @@
+"""ctypes binding of libfd.so: argument marshalling only.
+
+Every function here has the name of a C entry point in include/fd.h, converts
+Python / torch arguments into plain pointers and sizes, calls the library and
+raises FdError on a non-OK status.  No step of the computation runs here; if
+the library cannot be loaded the call fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfd.so")
+
+FD_BF16, FD_F32 = 0, 1
+STATUS = {0: "FD_OK", 1: "FD_ERR_INVALID_ARG", 2: "FD_ERR_SHAPE", 3: "FD_ERR_DTYPE",
+          4: "FD_ERR_CAPACITY", 5: "FD_ERR_CUDA", 6: "FD_ERR_DEVICE_TIMEOUT",
+          7: "FD_ERR_UNSUPPORTED", 8: "FD_ERR_ALIGNMENT"}
+
+# every symbol include/fd.h declares
+EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
+           "fd_cache_destroy", "fd_cache_get_desc", "fd_cache_layout_of",
+           "fd_cache_reset", "fd_rope3d", "fd_block_attention",
+           "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
+           "fd_launch_count", "fd_status_string"]
+
+
+class FdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_int32), ("max_rollouts", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("action_tokens", ctypes.c_int32), ("block_frames", ctypes.c_int32),
+                ("sink_frames", ctypes.c_int32), ("window_frames", ctypes.c_int32),
+                ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class CacheLayout(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_size_t), ("v", ctypes.c_size_t), ("pos", ctypes.c_size_t),
+                ("count", ctypes.c_size_t), ("ttab", ctypes.c_size_t),
+                ("htab", ctypes.c_size_t), ("wtab", ctypes.c_size_t),
+                ("err", ctypes.c_size_t), ("total", ctypes.c_size_t),
+                ("layer_kv_bytes", ctypes.c_size_t), ("rope_pairs_t", ctypes.c_int32),
+                ("rope_pairs_h", ctypes.c_int32), ("rope_pairs_w", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libfd.so (building it in-tree first when it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if build_if_missing and path == LIB_PATH:
+        from . import build as _build
+        if not _build.up_to_date():
+            _build.build()
+    if not os.path.exists(path):
+        raise FdError(-1, f"libfd.so not found at {path}")
+    lib = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.fd_cache_bytes.argtypes = [ctypes.POINTER(CacheDesc)]
+    lib.fd_cache_bytes.restype = sz
+    lib.fd_cache_get_layout.argtypes = [ctypes.POINTER(CacheDesc), ctypes.POINTER(CacheLayout)]
+    lib.fd_cache_create.argtypes = [ctypes.POINTER(CacheDesc), vp, sz, ctypes.POINTER(vp)]
+    lib.fd_cache_destroy.argtypes = [vp]
+    lib.fd_cache_get_desc.argtypes = [vp, ctypes.POINTER(CacheDesc)]
+    lib.fd_cache_layout_of.argtypes = [vp, ctypes.POINTER(CacheLayout)]
+    lib.fd_cache_reset.argtypes = [vp, ctypes.POINTER(i32), i32, vp]
+    lib.fd_rope3d.argtypes = [vp, i32, i32, vp, i32, vp]
+    lib.fd_block_attention.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.fd_cache_commit.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32),
+                                    ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
+    lib.fd_cache_frames.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int64)]
+    lib.fd_get_device_error.argtypes = [vp, ctypes.POINTER(i32)]
+    lib.fd_launch_count.argtypes = []
+    lib.fd_launch_count.restype = ctypes.c_uint64
+    lib.fd_status_string.argtypes = [i32]
+    lib.fd_status_string.restype = ctypes.c_char_p
+    for name in EXPORTS:
+        f = getattr(lib, name)
+        if f.restype is ctypes.c_int:  # default: status-returning functions
+            f.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise FdError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_desc(w, dtype: Optional[str] = None) -> CacheDesc:
+    """CacheDesc of a workload (see workloads.Workload)."""
+    dt = dtype or w.dtype
+    return CacheDesc(w.layers, w.rollouts, w.heads, w.head_dim, w.grid_h, w.grid_w,
+                     w.action_tokens, w.block_frames, w.sink_frames, w.window_frames,
+                     float(w.theta), FD_BF16 if dt == "bf16" else FD_F32)
+
+
+def fd_cache_bytes(desc: CacheDesc) -> int:
+    return load().fd_cache_bytes(ctypes.byref(desc))
+
+
+def fd_cache_get_layout(desc: CacheDesc) -> CacheLayout:
+    lay = CacheLayout()
+    _check(load().fd_cache_get_layout(ctypes.byref(desc), ctypes.byref(lay)),
+           "fd_cache_get_layout")
+    return lay
+
+
+def fd_status_string(status: int) -> str:
+    return load().fd_status_string(status).decode()
+
+
+def fd_launch_count() -> int:
+    return int(load().fd_launch_count())
+
+
+class Cache:
+    """Host handle of a cache bound to caller-owned device storage."""
+
+    def __init__(self, desc: CacheDesc, storage):
+        self.desc = desc
+        self.storage = storage          # keeps the caller's buffer alive
+        self.layout = fd_cache_get_layout(desc)
+        h = ctypes.c_void_p()
+        _check(load().fd_cache_create(ctypes.byref(desc), _ptr(storage),
+                                      storage.numel() * storage.element_size(),
+                                      ctypes.byref(h)), "fd_cache_create")
+        self.handle = h
+
+    def close(self) -> None:
+        if self.handle:
+            _check(load().fd_cache_destroy(self.handle), "fd_cache_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def fd_cache_create(desc: CacheDesc, storage) -> Cache:
+    """Bind a cache to `storage` (a uint8 CUDA tensor of fd_cache_bytes bytes)."""
+    return Cache(desc, storage)
+
+
+def fd_cache_reset(cache: Cache, rollout_ids: Sequence[int], stream=None) -> None:
+    ids = (ctypes.c_int32 * len(rollout_ids))(*rollout_ids)
+    _check(load().fd_cache_reset(cache.handle, ids, len(rollout_ids), _stream(stream)),
+           "fd_cache_reset")
+
+
+def fd_rope3d(cache: Cache, layer: int, n_rollouts: int, x, tokens_per_frame: int,
+              stream=None) -> None:
+    _check(load().fd_rope3d(cache.handle, layer, n_rollouts, _ptr(x), tokens_per_frame,
+                            _stream(stream)), "fd_rope3d")
+
+
+def fd_block_attention(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,
+                       lse=None, stream=None) -> None:
+    _check(load().fd_block_attention(cache.handle, layer, n_rollouts, _ptr(q), _ptr(k),
+                                     _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
+           "fd_block_attention")
+
+
+def fd_cache_commit(cache: Cache, layer_begin: int, layer_end: int, n_rollouts: int,
+                    k_list, v_list, frames: Optional[Sequence[int]] = None,
+                    stream=None) -> None:
+    nl = layer_end - layer_begin
+    kp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in k_list])
+    vp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in v_list])
+    fr = None if frames is None else (ctypes.c_int32 * n_rollouts)(*frames)
+    _check(load().fd_cache_commit(cache.handle, layer_begin, layer_end, n_rollouts, fr,
+                                  kp, vp, _stream(stream)), "fd_cache_commit")
+
+
+def fd_cache_frames(cache: Cache, layer: int, rollout: int) -> int:
+    n = ctypes.c_int64()
+    _check(load().fd_cache_frames(cache.handle, layer, rollout, ctypes.byref(n)),
+           "fd_cache_frames")
+    return n.value
+
+
+def fd_get_device_error(cache: Cache) -> int:
+    code = ctypes.c_int32()
+    st = load().fd_get_device_error(cache.handle, ctypes.byref(code))
+    if st not in (0, 6):
+        raise FdError(st, "fd_get_device_error")
+    return code.value

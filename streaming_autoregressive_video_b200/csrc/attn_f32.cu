@@ -1,0 +1,205 @@
+// fp32 block-causal chunk attention on CUDA cores (no TF32).
+//
+// Same definition as the tensor-core kernel: for every query of the block,
+// softmax(q' k'^T / sqrt(d)) v over the rollout's valid cache tokens (sinks +
+// window, positions from the slot table) and all tokens of the block, with 3D
+// RoPE applied to q and k as they are staged ("Cosmos3-H-Dreams" model card,
+// Model Architecture: block-causal student with a KV cache; AlpaDreams GTC
+// 2026 write-up, section VII: next frame from historical clean frames and the
+// current noisy frame).  Used for fp32 caches, where the tolerance leaves no
+// room for TF32 rounding.
+//
+// One CTA = (query tile of 32 rows, head, rollout); 8 warps x 4 rows.  Keys
+// are staged 64 at a time in shared memory, rotated in fp32; within a warp
+// lane j scores key j, then the warp forms the online softmax and each lane
+// accumulates d/32 output dimensions.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fd_internal.h"
+
+namespace fd {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kRowsPerWarp = 4;
+constexpr int kRows = kWarps * kRowsPerWarp;  // 32 query rows per CTA
+constexpr int kKeys = 64;                     // keys per staged tile
+
+struct KeyCoord {
+  int tidx;  // row of the rollout's t table
+  int h, w;
+};
+
+__device__ __forceinline__ float2 rope_cs(const AttnParams& p,
+                                          const float2* tt, int pair,
+                                          const KeyCoord& kc) {
+  if (pair < p.pt) return tt[kc.tidx * p.pt + pair];
+  if (pair < p.pt + p.ph) return p.htab[kc.h * p.ph + (pair - p.pt)];
+  return p.wtab[kc.w * p.pw + (pair - p.pt - p.ph)];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    attn_f32_kernel(AttnParams p) {
+  constexpr int kPerLane = D / 32;
+  extern __shared__ float sm[];
+  float* Qs = sm;                          // [kRows][D]
+  float* Ks = Qs + kRows * D;              // [kKeys][D + 1]
+  float* Vs = Ks + kKeys * (D + 1);        // [kKeys][D]
+
+  const int r = blockIdx.z, h = blockIdx.y;
+  const int q0 = blockIdx.x * kRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = p.count[r];
+  const int S = p.S, W = p.W;
+  const int nv = min(n, S) + min(max(n - S, 0), W);
+  const int n1 = nv * p.Tf, n2 = p.F * p.Tf;
+  const float2* tt = p.ttab + (size_t)r * (p.slots + p.F) * p.pt;
+  const float* qg = reinterpret_cast<const float*>(p.q);
+  const float* kg = reinterpret_cast<const float*>(p.k);
+  const float* vg = reinterpret_cast<const float*>(p.v);
+  const float* kcg = reinterpret_cast<const float*>(p.kc);
+  const float* vcg = reinterpret_cast<const float*>(p.vc);
+
+  // rotated queries
+  for (int e = threadIdx.x; e < kRows * (D / 2); e += blockDim.x) {
+    const int row = e / (D / 2), pair = e % (D / 2);
+    const int q = q0 + row;
+    float a = 0.f, b = 0.f;
+    if (q < p.Mq) {
+      const int f = q / p.T, tok = q - f * p.T;
+      const KeyCoord kc{p.slots + f, tok / p.gw, tok % p.gw};
+      const float* src = qg + (((size_t)r * p.Mq + q) * p.H + h) * D + 2 * pair;
+      const float2 cs = rope_cs(p, tt, pair, kc);
+      a = src[0] * cs.x - src[1] * cs.y;
+      b = src[0] * cs.y + src[1] * cs.x;
+    }
+    Qs[row * D + 2 * pair] = a;
+    Qs[row * D + 2 * pair + 1] = b;
+  }
+
+  float m[kRowsPerWarp], l[kRowsPerWarp], o[kRowsPerWarp][kPerLane];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) o[i][e] = 0.f;
+  }
+
+  const int nt1 = (n1 + kKeys - 1) / kKeys, nt2 = (n2 + kKeys - 1) / kKeys;
+  for (int j = 0; j < nt1 + nt2; ++j) {
+    const bool seg1 = j < nt1;
+    const int key0 = seg1 ? j * kKeys : (j - nt1) * kKeys;
+    const int nseg = seg1 ? n1 : n2;
+    __syncthreads();
+    for (int e = threadIdx.x; e < kKeys * (D / 2); e += blockDim.x) {
+      const int kr = e / (D / 2), pair = e % (D / 2);
+      const int key = key0 + kr;
+      float a = 0.f, b = 0.f, va = 0.f, vb = 0.f;
+      if (key < nseg) {
+        const int fi = key / p.Tf, tok = key - fi * p.Tf;
+        const KeyCoord kc{seg1 ? fi : p.slots + fi, tok < p.T ? tok / p.gw : 0,
+                          tok < p.T ? tok % p.gw : 0};
+        const size_t off = seg1
+            ? (((size_t)r * p.slots * p.Tf + key) * p.H + h) * D + 2 * pair
+            : (((size_t)r * p.F * p.Tf + key) * p.H + h) * D + 2 * pair;
+        const float* ks = (seg1 ? kcg : kg) + off;
+        const float* vs = (seg1 ? vcg : vg) + off;
+        const float2 cs = rope_cs(p, tt, pair, kc);
+        a = ks[0] * cs.x - ks[1] * cs.y;
+        b = ks[0] * cs.y + ks[1] * cs.x;
+        va = vs[0];
+        vb = vs[1];
+      }
+      Ks[kr * (D + 1) + 2 * pair] = a;
+      Ks[kr * (D + 1) + 2 * pair + 1] = b;
+      Vs[kr * D + 2 * pair] = va;
+      Vs[kr * D + 2 * pair + 1] = vb;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+      const float* qrow = Qs + (warp * kRowsPerWarp + i) * D;
+#pragma unroll
+      for (int sub = 0; sub < kKeys / 32; ++sub) {
+        const int kr = sub * 32 + lane;
+        const bool valid = key0 + kr < nseg;
+        float s = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D; ++e) s = fmaf(qrow[e], Ks[kr * (D + 1) + e], s);
+        s = valid ? s * p.scale : -INFINITY;
+        float mt = s;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        if (mt == -INFINITY) continue;  // whole sub-tile past the segment end
+        const float m_new = fmaxf(m[i], mt);
+        const float alpha = expf(m[i] - m_new);
+        const float pj = valid ? expf(s - m_new) : 0.f;
+        float ps = pj;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        l[i] = l[i] * alpha + ps;
+        m[i] = m_new;
+#pragma unroll
+        for (int e = 0; e < kPerLane; ++e) o[i][e] *= alpha;
+#pragma unroll 4
+        for (int jj = 0; jj < 32; ++jj) {
+          const float pb = __shfl_sync(0xffffffffu, pj, jj);
+          const float* vrow = Vs + (sub * 32 + jj) * D;
+#pragma unroll
+          for (int e = 0; e < kPerLane; ++e)
+            o[i][e] = fmaf(pb, vrow[lane + 32 * e], o[i][e]);
+        }
+      }
+    }
+  }
+
+  float* outg = reinterpret_cast<float*>(p.out);
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp; ++i) {
+    const int q = q0 + warp * kRowsPerWarp + i;
+    if (q >= p.Mq) continue;
+    const float inv = 1.f / l[i];
+    float* dst = outg + (((size_t)r * p.Mq + q) * p.H + h) * D;
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) dst[lane + 32 * e] = o[i][e] * inv;
+    if (p.lse != nullptr && lane == 0)
+      p.lse[((size_t)r * p.H + h) * p.Mq + q] = m[i] + logf(l[i]);
+  }
+}
+
+template <int D>
+cudaError_t launch_d(const AttnParams& p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (kRows * D + kKeys * (D + 1) + kKeys * D);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(
+        attn_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((p.Mq + kRows - 1) / kRows, p.H, p.n_rollouts);
+  attn_f32_kernel<D><<<grid, kWarps * 32, smem, s>>>(p);
+  count_launch(1);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s) {
+  switch (p.d) {
+    case 32: return launch_d<32>(p, s);
+    case 64: return launch_d<64>(p, s);
+    case 96: return launch_d<96>(p, s);
+    case 128: return launch_d<128>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace fd

@@ -1,0 +1,538 @@
+// bf16 block-causal chunk attention on sm_100a tensor cores.
+//
+// What it computes (the behaviour is described on the pages; the formulas are
+// the readings stated in include/fd.h): for every query of the current block
+// of a rollout, softmax(q' k'^T / sqrt(d)) v over the rollout's valid cache
+// tokens (sink frames + rolling window, "NVIDIA FlashDreams ...", Bounded
+// Memory for Infinite Rollouts) and all tokens of the block itself, which
+// attend to each other bidirectionally ("Cosmos3-H-Dreams" model card, Model
+// Architecture: block-causal student with a KV cache; AlpaDreams GTC 2026
+// write-up, section VII).  q' and k' carry 3D (t,h,w) RoPE, applied here as
+// Q and K tiles land in shared memory; the cache holds pre-RoPE keys.
+//
+// Design (one CTA = two 128-row query tiles of one (rollout, head)):
+//   warp 0        TMA producer: Q tiles once, then K and V tiles through
+//                 3-stage (K) and 2-stage (V) shared-memory rings, walking
+//                 the valid slot prefix of the cache and then the block; the
+//                 ring's wraparound needs no gather because attention does
+//                 not depend on key order.  No cluster multicast.
+//   warp 1        MMA issuer (one thread): S = Q K^T and O += P V on tcgen05
+//                 (kind::f16, bf16 operands, fp32 accumulators in TMEM); the
+//                 two query tiles ping-pong so one tile's softmax overlaps the
+//                 other tile's matrix products.
+//   warp 2        TMEM allocator (512 columns: S0, S1, O0, O1).
+//   warps 4-7     RoPE: rotate Q tiles once and every K tile in place in the
+//                 swizzled shared-memory layout, cos/sin from the cache's
+//                 tables (fp64-accurate angles rounded once to fp32).
+//   warps 8-15    softmax, one thread per query row (TMEM lane): row max,
+//                 exp2, row sum, P rounded to bf16 and written back into the
+//                 S columns of TMEM as the A operand of the PV product; the
+//                 O rescale is skipped unless the running max grows by more
+//                 than 2^8, which keeps P <= 256 and the result exact up to
+//                 rounding.  The epilogue divides by the row sum and writes
+//                 bf16 rows (and the optional log-sum-exp).
+// Every mbarrier wait is bounded: a wait that gives up raises a CTA-wide
+// abort flag and the device error word, in-flight copies and MMAs are
+// drained with bounded waits, TMEM is released and the CTA exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fd_internal.h"
+#include "sm100.cuh"
+
+namespace fd {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 512;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kD = 128;   // head dim handled by this kernel
+constexpr uint32_t kTile = kBM * kD * 2;  // 32 KB (bf16)
+constexpr uint32_t kHalf = kTile / 2;     // one 64-column, 128-byte-swizzled half
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = 2 * kTile;
+constexpr uint32_t kOffV = kOffK + kKStages * kTile;
+constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
+
+// TMEM columns
+constexpr uint32_t kColS0 = 0, kColO0 = 256;
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
+
+struct Shared {
+  uint64_t q_full, q_ready;
+  uint64_t k_full[kKStages], k_ready[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full, drain;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+constexpr uint32_t kSmemBytes = kOffShared + sizeof(Shared) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// Site codes for the device error word.
+enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4 };
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
+                                         Shared* sh, int32_t* err, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
+      atomicCAS(err, 0, kDevErrTimeout | (site << 8));
+      return false;
+    }
+  }
+  return true;
+}
+
+// Bounded wait used only while tearing down after an abort.
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+struct TileCounts {
+  int n1, n2, nt1, nt;
+};
+
+__device__ __forceinline__ TileCounts tile_counts(const AttnParams& p, int r) {
+  TileCounts t;
+  const int n = p.count[r];
+  const int nv = min(n, p.S) + min(max(n - p.S, 0), p.W);
+  t.n1 = nv * p.Tf;
+  t.n2 = p.F * p.Tf;
+  t.nt1 = (t.n1 + kBN - 1) / kBN;
+  t.nt = t.nt1 + (t.n2 + kBN - 1) / kBN;
+  return t;
+}
+
+// ---------------------------------------------------------------- RoPE
+// Thread `tid` (0..127) of the RoPE warpgroup owns 16-byte chunk cc = tid%16
+// of every row (8 bf16 = 4 rotation pairs: pairs 4cc..4cc+3) and rows
+// tid/16 + 8m.  A 128-byte-swizzled row keeps each 16-byte chunk intact, so
+// the pairs of a chunk stay together; only the chunk's position moves.
+struct RopeLane {
+  int sec[4];  // 0 = t, 1 = h, 2 = w
+  int j[4];    // pair index within its section
+  int half, chunk, row0;
+};
+
+__device__ __forceinline__ RopeLane rope_lane(const AttnParams& p, int tid) {
+  RopeLane rl;
+  const int cc = tid & 15;
+  rl.half = cc >> 3;
+  rl.chunk = cc & 7;
+  rl.row0 = tid >> 4;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int pair = cc * 4 + e;
+    if (pair < p.pt) { rl.sec[e] = 0; rl.j[e] = pair; }
+    else if (pair < p.pt + p.ph) { rl.sec[e] = 1; rl.j[e] = pair - p.pt; }
+    else { rl.sec[e] = 2; rl.j[e] = pair - p.pt - p.ph; }
+  }
+  return rl;
+}
+
+__device__ __forceinline__ void rotate_chunk(uint8_t* tile, int row,
+                                             const RopeLane& rl,
+                                             const AttnParams& p,
+                                             const float2* tt, int tidx,
+                                             int hh, int ww) {
+  uint4* ptr = reinterpret_cast<uint4*>(tile + rl.half * kHalf + row * 128 +
+                                        ((rl.chunk ^ (row & 7)) << 4));
+  uint4 u = *ptr;
+  uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2* src;
+    if (rl.sec[e] == 0) src = tt + tidx * p.pt + rl.j[e];
+    else if (rl.sec[e] == 1) src = p.htab + hh * p.ph + rl.j[e];
+    else src = p.wtab + ww * p.pw + rl.j[e];
+    const float2 cs = __ldg(src);
+    const float a = __uint_as_float(w4[e] << 16);
+    const float b = __uint_as_float(w4[e] & 0xFFFF0000u);
+    const __nv_bfloat162 r2 =
+        __floats2bfloat162_rn(a * cs.x - b * cs.y, a * cs.y + b * cs.x);
+    w4[e] = *reinterpret_cast<const uint32_t*>(&r2);
+  }
+  *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+}
+
+// Rotate the 128 query rows of tile `qt` (rows past Mq are zero: skipped).
+__device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
+                                            const RopeLane& rl,
+                                            const AttnParams& p,
+                                            const float2* tt) {
+#pragma unroll 4
+  for (int m = 0; m < 16; ++m) {
+    const int row = rl.row0 + 8 * m;
+    const int q = qrow0 + row;
+    if (q >= p.Mq) continue;
+    const int f = (int)fast_div((uint32_t)q, p.div_T);
+    const int tok = q - f * p.T;
+    const int hh = (int)fast_div((uint32_t)tok, p.div_gw);
+    rotate_chunk(tile, row, rl, p, tt, p.slots + f, hh, tok - hh * p.gw);
+  }
+}
+
+// Rotate the valid keys of one K tile (keys key0..key0+127 of a segment).
+__device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
+                                            bool seg1, const RopeLane& rl,
+                                            const AttnParams& p,
+                                            const float2* tt) {
+#pragma unroll 4
+  for (int m = 0; m < 16; ++m) {
+    const int row = rl.row0 + 8 * m;
+    const int key = key0 + row;
+    if (key >= nseg) continue;
+    const int fi = (int)fast_div((uint32_t)key, p.div_Tf);
+    const int tok = key - fi * p.Tf;
+    int hh = 0, ww = 0;
+    if (tok < p.T) {
+      hh = (int)fast_div((uint32_t)tok, p.div_gw);
+      ww = tok - hh * p.gw;
+    }
+    rotate_chunk(tile, row, rl, p, tt, seg1 ? fi : p.slots + fi, hh, ww);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_d128_sm100(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_kc,
+                         const __grid_constant__ CUtensorMap tm_vc,
+                         const __grid_constant__ CUtensorMap tm_kb,
+                         const __grid_constant__ CUtensorMap tm_vb,
+                         const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Shared* sh = reinterpret_cast<Shared*>(smem + kOffShared);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, r = blockIdx.z;
+  const int qrow0 = blockIdx.x * (2 * kBM);
+  const TileCounts tc = tile_counts(p, r);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->q_full, 1);
+    mbar_init(&sh->q_ready, 128);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&sh->k_full[s], 1);
+      mbar_init(&sh->k_ready[s], 128);
+      mbar_init(&sh->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&sh->v_full[s], 1);
+      mbar_init(&sh->v_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sh->s_full[x], 1);
+      mbar_init(&sh->p_full[x], 128);
+    }
+    mbar_init(&sh->o_full, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_kc);
+      prefetch_tmap(&tm_vc);
+      prefetch_tmap(&tm_kb);
+      prefetch_tmap(&tm_vb);
+      mbar_arrive_expect_tx(&sh->q_full, 2 * kTile);
+      for (int t = 0; t < 2; ++t)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(smem + kOffQ + t * kTile + hf * kHalf, &tm_q, &sh->q_full,
+                      hf * 64, h, qrow0 + t * kBM, r);
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < tc.nt; ++j) {
+        const bool seg1 = j < tc.nt1;
+        const int key0 = seg1 ? j * kBN : (j - tc.nt1) * kBN;
+        const CUtensorMap* mk = seg1 ? &tm_kc : &tm_kb;
+        const CUtensorMap* mv = seg1 ? &tm_vc : &tm_vb;
+        const int c3 = seg1 ? p.map_row0 + r : r;
+        const int ks = j % kKStages;
+        if (j >= kKStages &&
+            !wait_bar(&sh->k_empty[ks], ((j / kKStages) - 1) & 1, sh, p.err,
+                      kSiteProducer))
+          break;
+        mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
+                      &sh->k_full[ks], hf * 64, h, key0, c3);
+        issued_k = j + 1;
+        const int vs = j % kVStages;
+        if (j >= kVStages &&
+            !wait_bar(&sh->v_empty[vs], ((j / kVStages) - 1) & 1, sh, p.err,
+                      kSiteProducer))
+          break;
+        mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
+                      &sh->v_full[vs], hf * 64, h, key0, c3);
+        issued_v = j + 1;
+      }
+      if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) {
+        // let every copy still in flight land before the CTA exits
+        drain_bar(&sh->q_full, 0);
+        for (int j = max(0, issued_k - kKStages); j < issued_k; ++j)
+          drain_bar(&sh->k_full[j % kKStages], (j / kKStages) & 1);
+        for (int j = max(0, issued_v - kVStages); j < issued_v; ++j)
+          drain_bar(&sh->v_full[j % kVStages], (j / kVStages) & 1);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t sq = smem_addr(smem + kOffQ);
+      const uint32_t sk = smem_addr(smem + kOffK);
+      const uint32_t sv = smem_addr(smem + kOffV);
+      auto issue_s = [&](int x, int ks) {
+        const uint32_t qa = sq + x * kTile, kb = sk + ks * kTile;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+          mma_ss(tmem + kColS0 + x * 128, sdesc_sw128(qa + off, 16, 1024),
+                 sdesc_sw128(kb + off, 16, 1024), kIdescQK, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int x, int vs, bool acc) {
+        const uint32_t vb = sv + vs * kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_ts(tmem + kColO0 + x * 128, tmem + kColS0 + x * 128 + kk * 8,
+                 sdesc_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
+                 (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = wait_bar(&sh->q_ready, 0, sh, p.err, kSiteMma) &&
+                wait_bar(&sh->k_ready[0], 0, sh, p.err, kSiteMma);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(&sh->s_full[0]);
+        issue_s(1, 0);
+        mma_commit(&sh->s_full[1]);
+        mma_commit(&sh->k_empty[0]);
+        for (int j = 0; j < tc.nt && ok; ++j) {
+          const int vs = j % kVStages;
+          ok = wait_bar(&sh->v_full[vs], (j / kVStages) & 1, sh, p.err, kSiteMma) &&
+               wait_bar(&sh->p_full[0], j & 1, sh, p.err, kSiteMma);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(0, vs, j > 0);
+          const bool more = j + 1 < tc.nt;
+          const int ks = (j + 1) % kKStages;
+          if (more) {
+            ok = wait_bar(&sh->k_ready[ks], ((j + 1) / kKStages) & 1, sh, p.err,
+                          kSiteMma);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(0, ks);
+            mma_commit(&sh->s_full[0]);
+          }
+          ok = wait_bar(&sh->p_full[1], j & 1, sh, p.err, kSiteMma);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(1, vs, j > 0);
+          mma_commit(&sh->v_empty[vs]);
+          if (more) {
+            issue_s(1, ks);
+            mma_commit(&sh->s_full[1]);
+            mma_commit(&sh->k_empty[ks]);
+          }
+        }
+        mma_commit(&sh->o_full);
+      }
+      if (!ok) {
+        // wait for the tensor core to finish what was issued
+        mma_commit(&sh->drain);
+        drain_bar(&sh->drain, 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ RoPE
+    const int tid = threadIdx.x - 128;
+    const RopeLane rl = rope_lane(p, tid);
+    const float2* tt = p.ttab + (size_t)r * (p.slots + p.F) * p.pt;
+    bool ok = __all_sync(0xffffffffu, wait_bar(&sh->q_full, 0, sh, p.err, kSiteRope));
+    if (ok) {
+      rope_q_tile(smem + kOffQ, qrow0, rl, p, tt);
+      rope_q_tile(smem + kOffQ + kTile, qrow0 + kBM, rl, p, tt);
+      fence_proxy_async_smem();
+    }
+    mbar_arrive(&sh->q_ready);
+    for (int j = 0; j < tc.nt && ok; ++j) {
+      const int ks = j % kKStages;
+      ok = __all_sync(0xffffffffu, wait_bar(&sh->k_full[ks], (j / kKStages) & 1,
+                                            sh, p.err, kSiteRope));
+      if (!ok) break;
+      const bool seg1 = j < tc.nt1;
+      rope_k_tile(smem + kOffK + ks * kTile, seg1 ? j * kBN : (j - tc.nt1) * kBN,
+                  seg1 ? tc.n1 : tc.n2, seg1, rl, p, tt);
+      fence_proxy_async_smem();
+      mbar_arrive(&sh->k_ready[ks]);
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ softmax
+    const int x = (warp - 8) >> 2;
+    const int wq = warp & 3;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
+    const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint32_t rr[32];
+    for (int j = 0; j < tc.nt; ++j) {
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
+      if (!ok) break;
+      tc_fence_after();
+      const int valid = j < tc.nt1 ? min(kBN, tc.n1 - j * kBN)
+                                   : min(kBN, tc.n2 - (j - tc.nt1) * kBN);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        tmem_ld32(tS + c4 * 32, rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c4 * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(rr[i]));
+      }
+      const float m_tile = mx * sl2;
+      const bool need = m_tile > m + kRescaleThreshold;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        const float alpha = need ? exp2f(m - m_tile) : 1.f;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          tmem_ld32(tO + c4 * 32, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+          tmem_st32(tO + c4 * 32, rr);
+        }
+        tmem_wait_st();
+      }
+      if (need) {
+        l = (j > 0) ? l * exp2f(m - m_tile) : 0.f;
+        m = m_tile;
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        tmem_ld32(tS + c4 * 32, rr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c0 = c4 * 32 + 2 * i;
+          const float p0 = c0 < valid
+              ? exp2f(fmaf(__uint_as_float(rr[2 * i]), sl2, -m)) : 0.f;
+          const float p1 = c0 + 1 < valid
+              ? exp2f(fmaf(__uint_as_float(rr[2 * i + 1]), sl2, -m)) : 0.f;
+          lsum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + c4 * 16, pk);
+      }
+      l += lsum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sh->p_full[x]);
+    }
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(&sh->o_full, 0, sh, p.err, kSiteSoftmax));
+    if (ok) {
+      tc_fence_after();
+      const int row = qrow0 + x * kBM + wq * 32 + lane;
+      const float inv_l = 1.f / l;
+      uint16_t* out = static_cast<uint16_t*>(p.out) +
+                      (((size_t)r * p.Mq + row) * p.H + h) * kD;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        tmem_ld32(tO + c4 * 32, rr);
+        if (row < p.Mq) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l,
+                              __uint_as_float(rr[2 * i + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(out + c4 * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (p.lse != nullptr && row < p.Mq)
+        p.lse[((size_t)r * p.H + h) * p.Mq + row] =
+            (m + log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
+                                   const CUtensorMap& tm_kc,
+                                   const CUtensorMap& tm_vc,
+                                   const CUtensorMap& tm_kb,
+                                   const CUtensorMap& tm_vb,
+                                   const AttnParams& p, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(
+        attn_bf16_d128_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((p.Mq + 2 * kBM - 1) / (2 * kBM), p.H, p.n_rollouts);
+  attn_bf16_d128_sm100<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_kc, tm_vc,
+                                                          tm_kb, tm_vb, p);
+  count_launch(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fd

@@ -1,0 +1,271 @@
+// Cache maintenance kernels: storage initialisation, ring-buffer commit,
+// rollout reset and the standalone 3D RoPE.
+//
+// The commit is the finalize() half of the generate()/finalize() split in
+// "NVIDIA FlashDreams Is the Open-Source Inference Engine Robotics World
+// Models Needed" (Hot-Path Generation, Background State Updates), and the
+// ring keeps memory bounded as that page's Bounded Memory for Infinite
+// Rollouts section requires.  The slot rule (sinks first, then a W-slot ring)
+// and the RoPE layout are the readings documented in include/fd.h.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fd_internal.h"
+
+namespace fd {
+namespace {
+
+__device__ __forceinline__ int slot_of(int m, int S, int W) {
+  return m < S ? m : S + (m - S) % W;
+}
+
+// t-section (cos, sin) of one rollout/layer: rows 0..slots-1 for the frame
+// held by each slot (identity for empty slots), rows slots..slots+F-1 for the
+// next block's frames n..n+F-1.  Angles in fp64, rounded once to fp32.
+__device__ void fill_ttab(const CacheView& c, int l, int r, int n,
+                          const int32_t* pos_lr) {
+  float2* tab = c.ttab + ((size_t)l * c.R + r) * (c.slots + c.F) * c.pt;
+  const int rows = c.slots + c.F;
+  for (int e = threadIdx.x; e < rows * c.pt; e += blockDim.x) {
+    const int row = e / c.pt, j = e % c.pt;
+    const long long t = row < c.slots ? (long long)pos_lr[row]
+                                      : (long long)n + (row - c.slots);
+    float2 cs = make_float2(1.f, 0.f);
+    if (t >= 0) {
+      const double inv_freq = pow(c.theta, -(double)j / (double)c.pt);
+      double s, co;
+      sincos((double)t * inv_freq, &s, &co);
+      cs = make_float2((float)co, (float)s);
+    }
+    tab[e] = cs;
+  }
+}
+
+// grid: L*R blocks for slot metadata + 1 block for the static h/w tables.
+__global__ void cache_init_kernel(CacheView c) {
+  const int b = blockIdx.x;
+  if (b < c.L * c.R) {
+    const int l = b / c.R, r = b % c.R;
+    int32_t* pos = c.pos + (size_t)b * c.slots;
+    for (int s = threadIdx.x; s < c.slots; s += blockDim.x) pos[s] = -1;
+    if (threadIdx.x == 0) c.count[b] = 0;
+    __syncthreads();
+    fill_ttab(c, l, r, 0, pos);
+    return;
+  }
+  for (int e = threadIdx.x; e < c.gh * c.ph; e += blockDim.x) {
+    const int h = e / c.ph, j = e % c.ph;
+    double s, co;
+    sincos((double)h * pow(c.theta, -(double)j / (double)c.ph), &s, &co);
+    c.htab[e] = make_float2((float)co, (float)s);
+  }
+  for (int e = threadIdx.x; e < c.gw * c.pw; e += blockDim.x) {
+    const int w = e / c.pw, j = e % c.pw;
+    double s, co;
+    sincos((double)w * pow(c.theta, -(double)j / (double)c.pw), &s, &co);
+    c.wtab[e] = make_float2((float)co, (float)s);
+  }
+  if (threadIdx.x == 0) c.err[0] = 0;
+}
+
+// One block copies a 64 KB chunk of one frame of one tensor (K or V) of one
+// (layer, rollout) into the frame's ring slot.  16-byte vectors, 16 per
+// thread in flight.  grid = (chunks per frame, nl * nr * 2 * F).
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVecs = 16;
+
+__global__ void __launch_bounds__(kCopyThreads)
+    commit_copy_kernel(CacheView c, CommitParams p) {
+  const int job = blockIdx.y;
+  const int f = job % c.F;
+  const int kv = (job / c.F) & 1;
+  const int ri = (job / c.F / 2) % p.nr;
+  const int li = job / c.F / 2 / p.nr;
+  if (f >= p.frames[ri]) return;
+  const int l = p.layer0 + li, r = p.rollout0 + ri;
+  const int n = c.count[(size_t)l * c.R + r];
+  const int slot = slot_of(n + f, c.S, c.W);
+  const uint64_t fvecs = c.frame_bytes / 16;
+  const uint8_t* src_base = kv ? p.v[li] : p.k[li];
+  const uint4* src = reinterpret_cast<const uint4*>(
+      src_base + ((uint64_t)r * c.F + f) * c.frame_bytes);
+  uint8_t* dst_base = kv ? c.v : c.k;
+  uint4* dst = reinterpret_cast<uint4*>(
+      dst_base + (((uint64_t)l * c.R + r) * c.slots + slot) * c.frame_bytes);
+  const uint64_t v0 = (uint64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
+  uint4 buf[kCopyVecs];
+#pragma unroll
+  for (int i = 0; i < kCopyVecs; ++i) {
+    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
+    if (vi < fvecs) buf[i] = __ldcs(src + vi);
+  }
+#pragma unroll
+  for (int i = 0; i < kCopyVecs; ++i) {
+    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
+    if (vi < fvecs) dst[vi] = buf[i];
+  }
+}
+
+// After the copy: slot positions, counter and t table of every (layer, rollout).
+__global__ void commit_meta_kernel(CacheView c, CommitParams p) {
+  const int li = blockIdx.x / p.nr, ri = blockIdx.x % p.nr;
+  const int l = p.layer0 + li, r = p.rollout0 + ri;
+  const size_t lr = (size_t)l * c.R + r;
+  int32_t* pos = c.pos + lr * c.slots;
+  const int n = c.count[lr];
+  const int nf = p.frames[ri];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int f = 0; f < nf; ++f) pos[slot_of(n + f, c.S, c.W)] = n + f;
+    c.count[lr] = n + nf;
+  }
+  __syncthreads();
+  fill_ttab(c, l, r, n + nf, pos);
+}
+
+// Zero the K/V of the listed rollouts in every layer.
+// grid = (chunks per (layer, rollout) region, L * n * 2)
+__global__ void __launch_bounds__(kCopyThreads)
+    reset_zero_kernel(CacheView c, ResetParams p) {
+  const int job = blockIdx.y;
+  const int kv = job & 1;
+  const int id = (job >> 1) % p.n;
+  const int l = (job >> 1) / p.n;
+  const int r = p.ids[id];
+  const uint64_t region = (uint64_t)c.slots * c.frame_bytes;
+  uint8_t* base = (kv ? c.v : c.k) + ((uint64_t)l * c.R + r) * region;
+  uint4* dst = reinterpret_cast<uint4*>(base);
+  const uint64_t nvec = region / 16;
+  const uint64_t v0 = (uint64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+  for (int i = 0; i < kCopyVecs; ++i) {
+    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
+    if (vi < nvec) dst[vi] = z;
+  }
+}
+
+__global__ void reset_meta_kernel(CacheView c, ResetParams p) {
+  const int l = blockIdx.x / p.n;
+  const int r = p.ids[blockIdx.x % p.n];
+  const size_t lr = (size_t)l * c.R + r;
+  int32_t* pos = c.pos + lr * c.slots;
+  for (int s = threadIdx.x; s < c.slots; s += blockDim.x) pos[s] = -1;
+  if (threadIdx.x == 0) c.count[lr] = 0;
+  __syncthreads();
+  fill_ttab(c, l, r, 0, pos);
+}
+
+// Rotate one 16-byte chunk of a [R][F][Tx][H][d] tensor in place.
+template <typename Elem>
+__global__ void rope3d_kernel(CacheView c, int layer, int n_rollouts,
+                              Elem* x, int Tx, uint64_t nchunks) {
+  constexpr int kPer = 16 / sizeof(Elem);  // elements per chunk (4 or 8)
+  const int cpr = c.d / kPer;              // chunks per head row
+  for (uint64_t ci = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+       ci < nchunks; ci += (uint64_t)gridDim.x * blockDim.x) {
+    const int cc = (int)(ci % cpr);
+    uint64_t rest = ci / cpr;
+    rest /= c.H;                       // head index does not matter
+    const int tok = (int)(rest % Tx);
+    rest /= Tx;
+    const int f = (int)(rest % c.F);
+    const int r = (int)(rest / c.F);
+    const float2* tt = c.ttab + (((size_t)layer * c.R + r) * (c.slots + c.F) +
+                                 c.slots + f) * c.pt;
+    const int hh = tok < c.T ? tok / c.gw : 0;
+    const int ww = tok < c.T ? tok % c.gw : 0;
+    Elem* px = x + ci * kPer;
+    float vals[kPer];
+    if constexpr (sizeof(Elem) == 2) {
+      const uint4 u = *reinterpret_cast<const uint4*>(px);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        vals[2 * i] = __uint_as_float(w4[i] << 16);
+        vals[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+      }
+    } else {
+      const float4 u = *reinterpret_cast<const float4*>(px);
+      vals[0] = u.x; vals[1] = u.y; vals[2] = u.z; vals[3] = u.w;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer / 2; ++i) {
+      const int pair = cc * (kPer / 2) + i;
+      float2 cs;
+      if (pair < c.pt) cs = tt[pair];
+      else if (pair < c.pt + c.ph) cs = c.htab[hh * c.ph + (pair - c.pt)];
+      else cs = c.wtab[ww * c.pw + (pair - c.pt - c.ph)];
+      const float a = vals[2 * i], b = vals[2 * i + 1];
+      vals[2 * i] = a * cs.x - b * cs.y;
+      vals[2 * i + 1] = a * cs.y + b * cs.x;
+    }
+    if constexpr (sizeof(Elem) == 2) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(vals[2 * i], vals[2 * i + 1]);
+        w4[i] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(px) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    } else {
+      *reinterpret_cast<float4*>(px) = make_float4(vals[0], vals[1], vals[2], vals[3]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s) {
+  cache_init_kernel<<<c.L * c.R + 1, 256, 0, s>>>(c);
+  count_launch(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_commit(const CacheView& c, const CommitParams& p,
+                          cudaStream_t s) {
+  const uint64_t fvecs = c.frame_bytes / 16;
+  const uint64_t chunks = (fvecs + kCopyThreads * kCopyVecs - 1) /
+                          (kCopyThreads * kCopyVecs);
+  dim3 grid((unsigned)chunks, (unsigned)(p.nl * p.nr * 2 * c.F));
+  commit_copy_kernel<<<grid, kCopyThreads, 0, s>>>(c, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  commit_meta_kernel<<<p.nl * p.nr, 128, 0, s>>>(c, p);
+  count_launch(2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
+                         cudaStream_t s) {
+  const uint64_t nvec = (uint64_t)c.slots * c.frame_bytes / 16;
+  const uint64_t chunks = (nvec + kCopyThreads * kCopyVecs - 1) /
+                          (kCopyThreads * kCopyVecs);
+  dim3 grid((unsigned)chunks, (unsigned)(c.L * p.n * 2));
+  reset_zero_kernel<<<grid, kCopyThreads, 0, s>>>(c, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  reset_meta_kernel<<<c.L * p.n, 128, 0, s>>>(c, p);
+  count_launch(2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
+                          void* x, int Tx, cudaStream_t s) {
+  const uint64_t elems = (uint64_t)n_rollouts * c.F * Tx * c.H * c.d;
+  const uint64_t nchunks = elems * c.esz / 16;
+  const unsigned blocks = (unsigned)((nchunks + 255) / 256 < 148ull * 16
+                                         ? (nchunks + 255) / 256
+                                         : 148ull * 16);
+  if (c.esz == 2)
+    rope3d_kernel<uint16_t><<<blocks, 256, 0, s>>>(
+        c, layer, n_rollouts, static_cast<uint16_t*>(x), Tx, nchunks);
+  else
+    rope3d_kernel<float><<<blocks, 256, 0, s>>>(
+        c, layer, n_rollouts, static_cast<float*>(x), Tx, nchunks);
+  count_launch(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fd

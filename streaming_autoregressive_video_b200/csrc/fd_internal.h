@@ -1,0 +1,108 @@
+// Internal definitions shared by the host entry points and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fd.h"
+
+namespace fd {
+
+// Device error word: bits 0-7 kind, bits 8-15 site.
+enum DevErrKind : int32_t { kDevErrTimeout = 1, kDevErrArgument = 2 };
+
+// Exact division by a runtime constant for the index ranges used here
+// (n * d < 2^40): q = (n * m) >> 40 with m = ceil(2^40 / d).
+struct FastDiv {
+  uint64_t m;
+  uint32_t d;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.m = ((1ull << 40) + d - 1) / d;
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
+  return (uint32_t)(((uint64_t)n * f.m) >> 40);
+}
+
+// Device pointers into one cache's storage plus its geometry.
+struct CacheView {
+  uint8_t* k;
+  uint8_t* v;
+  int32_t* pos;
+  int32_t* count;
+  float2* ttab;
+  float2* htab;
+  float2* wtab;
+  int32_t* err;
+  int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz;
+  double theta;
+  uint64_t frame_bytes;  // Tf * H * d * esz
+};
+
+// Limits of one commit launch (host splits larger requests).
+constexpr int kCommitMaxLayers = 32;
+constexpr int kCommitMaxRollouts = 64;
+
+struct CommitParams {
+  const uint8_t* k[kCommitMaxLayers];
+  const uint8_t* v[kCommitMaxLayers];
+  int32_t frames[kCommitMaxRollouts];
+  int layer0;    // first layer of this launch
+  int nl;        // layers in this launch
+  int rollout0;  // first rollout of this launch
+  int nr;        // rollouts in this launch
+  int src_rollouts;  // rollout extent of the k/v buffers (their stride)
+};
+
+struct ResetParams {
+  int32_t ids[kCommitMaxRollouts];
+  int n;
+};
+
+// Parameters of the attention kernels (the tensor maps travel separately).
+struct AttnParams {
+  const void* q;         // block tensors (CUDA-core path reads them directly)
+  const void* k;
+  const void* v;
+  const int32_t* pos;    // [R][slots] of the layer
+  const int32_t* count;  // [R] of the layer
+  const float2* ttab;    // [R][slots+F][pt] of the layer
+  const float2* htab;
+  const float2* wtab;
+  void* out;
+  float* lse;
+  int32_t* err;
+  const uint8_t* kc;     // cache K of the layer, rollout 0 (CUDA-core path)
+  const uint8_t* vc;
+  int H, d, T, Tf, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
+  int map_row0;          // layer * R: row offset of this layer in the cache maps
+  FastDiv div_T, div_Tf, div_gw;
+  float scale_log2;      // log2(e) / sqrt(d)
+  float scale;           // 1 / sqrt(d)
+};
+
+// Launch helpers implemented in the .cu files.
+cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s);
+cudaError_t launch_commit(const CacheView& c, const CommitParams& p,
+                          cudaStream_t s);
+cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
+                         cudaStream_t s);
+cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
+                          void* x, int tokens_per_frame, cudaStream_t s);
+cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
+                                   const CUtensorMap& tm_kc,
+                                   const CUtensorMap& tm_vc,
+                                   const CUtensorMap& tm_kb,
+                                   const CUtensorMap& tm_vb,
+                                   const AttnParams& p, cudaStream_t s);
+
+void count_launch(int n);
+
+}  // namespace fd

@@ -1,0 +1,161 @@
+"""Shared helpers of the GPU tests: cache set-up, host<->device marshalling,
+and lockstep drivers that feed identical seeded bytes to the CUDA path (through
+the C ABI) and to the CPU oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from streaming_autoregressive_video_b200 import binding as fd
+from streaming_autoregressive_video_b200 import synth
+
+TOL_BF16_MAX = 2e-2
+TOL_BF16_MEAN = 2e-3
+TOL_F32_MAX = 1e-4
+
+
+def new_cache(w, device="cuda"):
+    desc = fd.make_desc(w)
+    nbytes = fd.fd_cache_bytes(desc)
+    assert nbytes > 0
+    storage = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
+    off = (-storage.data_ptr()) % 1024
+    storage = storage[off:off + nbytes]
+    return fd.fd_cache_create(desc, storage)
+
+
+def views(cache, w):
+    """torch views of the cache regions inside the caller-owned storage."""
+    lay = cache.layout
+    st = cache.storage
+    L, R, slots = w.layers, w.rollouts, w.slots
+    esz = 2 if w.dtype == "bf16" else 4
+    n_kv = L * R * slots * w.frame_tokens * w.heads * w.head_dim
+    kv_dt = torch.int16 if esz == 2 else torch.float32
+    shape = (L, R, slots, w.frame_tokens, w.heads, w.head_dim)
+    k = st[lay.k:lay.k + n_kv * esz].view(kv_dt).view(shape)
+    v = st[lay.v:lay.v + n_kv * esz].view(kv_dt).view(shape)
+    pos = st[lay.pos:lay.pos + L * R * slots * 4].view(torch.int32).view(L, R, slots)
+    count = st[lay.count:lay.count + L * R * 4].view(torch.int32).view(L, R)
+    return k, v, pos, count
+
+
+def to_device(a: np.ndarray, device="cuda") -> torch.Tensor:
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16).copy()).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def to_host(t: torch.Tensor) -> np.ndarray:
+    a = t.detach().cpu().numpy()
+    return a.view(np.uint16) if a.dtype == np.int16 else a
+
+
+def out_values(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.int16:
+        return oracle.bf16_bits_to_f64(to_host(t))
+    return t.detach().cpu().numpy().astype(np.float64)
+
+
+def empty_like_q(w, n_rollouts, device="cuda"):
+    shape = (n_rollouts, w.queries, w.heads, w.head_dim)
+    dt = torch.int16 if w.dtype == "bf16" else torch.float32
+    return torch.empty(shape, dtype=dt, device=device)
+
+
+def block_inputs(w, seed_parts, n_rollouts):
+    """Seeded q, k, v of one attention call, storage form (numpy)."""
+    qs = (n_rollouts, w.queries, w.heads, w.head_dim)
+    ks = (n_rollouts, w.block_frames * w.frame_tokens, w.heads, w.head_dim)
+    q = synth.normal(synth.seed_of(*seed_parts, 0), qs, w.dtype, w.value_scale)
+    k = synth.normal(synth.seed_of(*seed_parts, 1), ks, w.dtype, w.value_scale)
+    v = synth.normal(synth.seed_of(*seed_parts, 2), ks, w.dtype, w.value_scale)
+    return q, k, v
+
+
+def compare(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):
+    err = np.abs(got - want)
+    mx, mean = float(err.max()), float(err.mean())
+    if dtype == "bf16":
+        assert mx <= TOL_BF16_MAX and mean <= TOL_BF16_MEAN, \
+            f"{what}: max abs {mx:.3g} mean abs {mean:.3g}"
+    else:
+        assert mx <= TOL_F32_MAX, f"{what}: max abs {mx:.3g}"
+    return mx, mean
+
+
+class Lockstep:
+    """Drives the GPU cache and per-(rollout, layer) oracle caches together."""
+
+    def __init__(self, w, device="cuda"):
+        self.w = w
+        self.cache = new_cache(w, device)
+        self.device = device
+        self.orc = [[oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens,
+                                         w.heads, w.head_dim, w.dtype)
+                     for _ in range(w.rollouts)] for _ in range(w.layers)]
+
+    def attention(self, layer, q, k, v, n_rollouts=None, rows=None, with_lse=True,
+                  check=True, what=""):
+        w = self.w
+        nr = n_rollouts or w.rollouts
+        out = empty_like_q(w, nr, self.device)
+        lse = torch.empty((nr, w.heads, w.queries), dtype=torch.float32,
+                          device=self.device) if with_lse else None
+        qd, kd, vd = to_device(q, self.device), to_device(k, self.device), to_device(v, self.device)
+        fd.fd_block_attention(self.cache, layer, nr, qd, kd, vd, out, lse)
+        torch.cuda.synchronize()
+        got = out_values(out)
+        errs = []
+        if check:
+            for r in range(nr):
+                want, want_lse = oracle.block_attention(
+                    self.orc[layer][r], q[r], k[r], v[r], tokens=w.tokens,
+                    grid_w=w.grid_w, theta=w.theta, rows=rows)
+                sel = slice(None) if rows is None else np.asarray(rows)
+                errs.append(compare(got[r][sel], want[sel], w.dtype, f"{what} r={r}"))
+                if with_lse:
+                    lse_got = lse[r].cpu().numpy().astype(np.float64)
+                    d_lse = np.abs(lse_got[:, sel] - want_lse[:, sel]).max()
+                    assert d_lse <= (1e-2 if w.dtype == "bf16" else 1e-4), \
+                        f"{what} r={r}: lse max abs {d_lse:.3g}"
+        return got, errs
+
+    def commit(self, layers, k_list, v_list, n_rollouts=None, frames=None):
+        """k_list[i]: numpy [nr][F*Tf][H][d] for layer layers[0]+i."""
+        w = self.w
+        nr = n_rollouts or w.rollouts
+        kd = [to_device(a, self.device) for a in k_list]
+        vd = [to_device(a, self.device) for a in v_list]
+        fd.fd_cache_commit(self.cache, layers[0], layers[-1] + 1, nr, kd, vd, frames)
+        F, Tf = w.block_frames, w.frame_tokens
+        for i, l in enumerate(layers):
+            for r in range(nr):
+                nf = F if frames is None else int(frames[r])
+                kf = k_list[i][r].reshape(F, Tf, w.heads, w.head_dim)[:nf]
+                vf = v_list[i][r].reshape(F, Tf, w.heads, w.head_dim)[:nf]
+                self.orc[l][r].commit(kf, vf)
+        torch.cuda.synchronize()
+
+    def reset(self, ids):
+        fd.fd_cache_reset(self.cache, ids)
+        for l in range(self.w.layers):
+            for r in ids:
+                self.orc[l][r].reset()
+        torch.cuda.synchronize()
+
+    def check_cache_exact(self):
+        """Slot positions, counters and every valid slot's bytes, bit for bit."""
+        w = self.w
+        k, v, pos, count = views(self.cache, w)
+        k, v, pos, count = to_host(k), to_host(v), to_host(pos), to_host(count)
+        for l in range(w.layers):
+            for r in range(w.rollouts):
+                o = self.orc[l][r]
+                assert count[l, r] == o.n, (l, r, count[l, r], o.n)
+                assert np.array_equal(pos[l, r], o.pos), (l, r, pos[l, r], o.pos)
+                nv = o.valid_slots()
+                assert np.array_equal(k[l, r, :nv], o.k[:nv]), ("K", l, r)
+                assert np.array_equal(v[l, r, :nv], o.v[:nv]), ("V", l, r)
+                assert fd.fd_cache_frames(self.cache, l, r) == o.n

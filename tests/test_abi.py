@@ -1,0 +1,86 @@
+"""The C ABI on the host: the library loads without a GPU, exports every symbol
+include/fd.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from streaming_autoregressive_video_b200 import binding as fd
+from streaming_autoregressive_video_b200.workloads import ALL, SINGLE_480P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "fd.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fd_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fd.load()
+    syms = declared_symbols()
+    assert len(syms) >= 14
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert sorted(fd.EXPORTS) == syms
+
+
+def test_cache_bytes_and_layout():
+    for w in ALL:
+        desc = fd.make_desc(w)
+        n = fd.fd_cache_bytes(desc)
+        lay = fd.fd_cache_get_layout(desc)
+        assert n == lay.total > 0
+        esz = 2 if w.dtype == "bf16" else 4
+        kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.heads * w.head_dim * esz
+        assert lay.layer_kv_bytes * w.layers == kv
+        regions = [lay.k, lay.v, lay.pos, lay.count, lay.ttab, lay.htab, lay.wtab, lay.err]
+        assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
+        assert lay.v - lay.k >= kv and lay.pos - lay.v >= kv
+        assert (lay.rope_pairs_t, lay.rope_pairs_h, lay.rope_pairs_w) == \
+            (w.head_dim // 2 - 2 * (w.head_dim // 6), w.head_dim // 6, w.head_dim // 6)
+
+
+def test_single_480p_cache_is_about_2_gb():
+    n = fd.fd_cache_bytes(fd.make_desc(SINGLE_480P))
+    # 30 layers x 7 slots x 1560 tokens x 12 heads x 128 x 2 B x (K, V)
+    assert abs(n - 30 * 7 * 1560 * 12 * 128 * 2 * 2) < 1 << 20
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("block_frames", 0, 2), ("window_frames", 0, 2), ("head_dim", 12, 2),
+    ("num_heads", 0, 2), ("dtype", 7, 3), ("sink_frames", -1, 2),
+    ("action_tokens", -2, 2), ("rope_theta", float("nan"), 2)])
+def test_bad_descriptors_rejected(field, value, status):
+    desc = fd.make_desc(SINGLE_480P)
+    setattr(desc, field, value)
+    assert fd.fd_cache_bytes(desc) == 0
+    lay = fd.CacheLayout()
+    assert fd.load().fd_cache_get_layout(ctypes.byref(desc), ctypes.byref(lay)) == status
+
+
+def test_block_larger_than_window_rejected():
+    desc = fd.make_desc(SINGLE_480P)
+    desc.block_frames = 7
+    assert fd.fd_cache_bytes(desc) == 0
+
+
+def test_host_errors_before_any_device_call():
+    lib = fd.load()
+    desc = fd.make_desc(SINGLE_480P)
+    h = ctypes.c_void_p()
+    # null storage: rejected after validation, before any CUDA call
+    assert lib.fd_cache_create(ctypes.byref(desc), None, 1 << 40, ctypes.byref(h)) == 1
+    assert lib.fd_cache_create(ctypes.byref(desc), 1024, 16, ctypes.byref(h)) == 4
+    assert lib.fd_cache_create(ctypes.byref(desc), 1000, 1 << 40, ctypes.byref(h)) == 8
+    assert lib.fd_block_attention(None, 0, 1, 16, 16, 16, 16, None, None) == 1
+    assert lib.fd_cache_commit(None, 0, 1, 1, None, None, None, None) == 1
+    assert lib.fd_cache_reset(None, None, 1, None) == 1
+    assert lib.fd_rope3d(None, 0, 1, 16, 4, None) == 1
+    code = ctypes.c_int32()
+    assert lib.fd_get_device_error(None, ctypes.byref(code)) == 1
+    assert lib.fd_cache_destroy(None) == 1
+    assert fd.fd_status_string(6) == "device-side wait gave up"
+    assert fd.fd_launch_count() >= 0
