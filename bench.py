@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming chunk-attention hot path on B200.
+
+One bench step = one block of a rollout through the model's attention layers:
+for every denoising step and every layer, one fd_block_attention call with
+that step's q/k/v, then one batched fd_cache_commit of the last step's k/v
+into every layer's ring buffer.  The cache is full (steady state) before the
+timed region, so every call attends to sinks + the whole window + the block.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference]
+                    [--workload 480p|large|long|ragged]
+
+N > 1 runs one independent replica per GPU (the path has no exchange step):
+value = work of all ranks / max-over-ranks time ("scaling": "weak").
+`--impl reference` times the CPU oracle (the reference arm of this method)
+on a bounded sample of the same workload.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("chunk-attention TFLOP/s & latent-frames/s per layer; "
+          "% of bf16 tensor/HBM roofline")
+PROFILE = os.path.join(ROOT, "profiles", "attn_bf16_d128_sm100.480p.md")
+KERNEL_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
+                          "attn_sm100.cu")
+
+
+def workloads():
+    from streaming_autoregressive_video_b200 import workloads as wl
+    return {"480p": wl.SINGLE_480P, "large": wl.LARGE_ACTIONS,
+            "long": wl.LONG_ROLLOUT, "ragged": wl.BATCHED_RAGGED}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["fd", "reference"], default="fd")
+    ap.add_argument("--workload", default="480p")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small profiling cases only)")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# helpers
+# --------------------------------------------------------------------------
+def attn_flops(w, nkeys_per_rollout):
+    """Algorithmic FLOPs of one call: QK^T + PV over the valid keys only."""
+    return sum(4.0 * w.heads * w.head_dim * w.queries * nk for nk in nkeys_per_rollout)
+
+
+def attn_bytes(w, nkeys_per_rollout, esz=2):
+    """Q + block K/V + valid cache K/V read once + O written once."""
+    per_tok = w.heads * w.head_dim * esz
+    b = 0
+    for nk in nkeys_per_rollout:
+        b += 2 * w.queries * per_tok + 2 * nk * per_tok
+    return float(b)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+            "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profile_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (sha256 recorded in the summary)."""
+    try:
+        text = open(PROFILE).read()
+        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != src:
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd_, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd_)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r[2] > 250.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in load),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timings (baseline / reference arm)
+# --------------------------------------------------------------------------
+def oracle_call_setup(w, heads):
+    import oracle
+    from streaming_autoregressive_video_b200 import synth
+    c = oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens, w.heads,
+                            w.head_dim, "bf16")
+    ks = (w.block_frames, w.frame_tokens, w.heads, w.head_dim)
+    n_commits = -(-w.slots // w.block_frames) + 1
+    for b in range(n_commits):
+        c.commit(synth.normal(synth.seed_of(7, b, 0), ks, "bf16", w.value_scale),
+                 synth.normal(synth.seed_of(7, b, 1), ks, "bf16", w.value_scale))
+    q = synth.normal(synth.seed_of(7, 99, 0), (w.queries, w.heads, w.head_dim), "bf16", w.value_scale)
+    k = synth.normal(synth.seed_of(7, 99, 1), (w.block_frames * w.frame_tokens, w.heads, w.head_dim), "bf16", w.value_scale)
+    v = synth.normal(synth.seed_of(7, 99, 2), (w.block_frames * w.frame_tokens, w.heads, w.head_dim), "bf16", w.value_scale)
+    nk = (c.valid_slots() + w.block_frames) * w.frame_tokens
+
+    def call():
+        oracle.block_attention(c, q, k, v, tokens=w.tokens, grid_w=w.grid_w,
+                               theta=w.theta, heads=heads)
+    return call, 4.0 * len(heads) * w.head_dim * w.queries * nk
+
+
+def oracle_threads():
+    try:
+        import threadpoolctl
+        return max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w):
+    heads = list(range(w.heads))
+    call, flops = oracle_call_setup(w, heads)
+    t0 = time.perf_counter()
+    call()
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"one full attention call ({w.heads} heads x {w.queries} queries, "
+                      f"cache full) in fp64 numpy, {dt:.1f} s"}
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    heads = [0, 1]
+    call, flops = oracle_call_setup(w, heads)
+    for _ in range(args.warmup):
+        call()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        call()
+    dt = (time.perf_counter() - t0) / args.steps
+    val = flops / dt / 1e12
+    sample = (f"per step: {len(heads)} of {w.heads} heads of one attention call "
+              f"({w.queries} queries, cache full), fp64 numpy oracle")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name}, "cpu_baseline": {
+            "value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+# --------------------------------------------------------------------------
+# CUDA path
+# --------------------------------------------------------------------------
+def run_fd(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from streaming_autoregressive_video_b200 import binding as fd
+    from streaming_autoregressive_video_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fd.load(build_if_missing=(rank == 0))
+    L, R, S = w.layers, w.rollouts, w.steps
+    F, Tf, H, d = w.block_frames, w.frame_tokens, w.heads, w.head_dim
+    desc = fd.make_desc(w)
+    nbytes = fd.fd_cache_bytes(desc)
+    raw = torch.empty(nbytes + 1024, dtype=torch.uint8, device=dev)
+    off = (-raw.data_ptr()) % 1024
+    storage = raw[off:off + nbytes]
+    cache = fd.fd_cache_create(desc, storage)
+
+    def gen(seed, shape):
+        return synth.normal_device(seed, shape, "bf16", dev, w.value_scale).view(torch.int16)
+
+    qshape = (R, w.queries, H, d)
+    kshape = (R, F * Tf, H, d)
+    base = 1000 * rank
+    # prefill every layer until the window is full (steady state)
+    pk = [gen(synth.seed_of(base, 1, l), kshape) for l in range(L)]
+    pv = [gen(synth.seed_of(base, 2, l), kshape) for l in range(L)]
+    if w.ragged_window:
+        lo, hi = w.ragged_window
+        fill = synth.ragged_fill(synth.seed_of(base, 3), R, lo, hi)
+        left = fill.copy()
+        while left.max() > 0:
+            fr = [int(min(F, x)) for x in left]
+            fd.fd_cache_commit(cache, 0, L, R, pk, pv, frames=fr)
+            left -= fr
+    else:
+        for _ in range(-(-w.slots // F) + 1):
+            fd.fd_cache_commit(cache, 0, L, R, pk, pv)
+    torch.cuda.synchronize()
+
+    def nkeys():
+        out = []
+        for r in range(R):
+            n = fd.fd_cache_frames(cache, 0, r)
+            nv = min(n, w.sink_frames) + min(max(n - w.sink_frames, 0), w.window_frames)
+            out.append((nv + F) * Tf)
+        return out
+
+    q = [[gen(synth.seed_of(base, 10, s, l), qshape) for l in range(L)] for s in range(S)]
+    k = [[gen(synth.seed_of(base, 11, s, l), kshape) for l in range(L)] for s in range(S)]
+    v = [[gen(synth.seed_of(base, 12, s, l), kshape) for l in range(L)] for s in range(S)]
+    outs = [torch.empty(qshape, dtype=torch.int16, device=dev) for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        for s in range(S):
+            for l in range(L):
+                if evs is not None:
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                fd.fd_block_attention(cache, l, R, q[s][l], k[s][l], v[s][l], outs[l],
+                                      stream=stream)
+                if evs is not None:
+                    b.record(stream)
+                    evs.append((a, b))
+        fd.fd_cache_commit(cache, 0, L, R, k[S - 1], v[S - 1], stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    nk = nkeys()  # steady state: constant over the timed steps when uniform
+    flops_call = attn_flops(w, nk)
+    bytes_call = attn_bytes(w, nk)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = fd.fd_launch_count()
+    evs = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(evs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    launches = fd.fd_launch_count() - launches0
+    ms_step = e0.elapsed_time(e1) / args.steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    t = torch.tensor([ms_step, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step, attn_ms = float(t[0]), float(t[1])
+    err = fd.fd_get_device_error(cache)
+    assert err == 0, f"device error word {err:#x}"
+
+    flops_step = flops_call * S * L
+    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    frames_per_s_layer = R * F * L * world / (ms_step * 1e-3)
+
+    # ---------------- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world)
+
+    if rank != 0:
+        return
+    peaks, src = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = flops_call / (attn_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": profile_traffic(),
+            "kernel": "attn_bf16_d128_sm100", "peak_source": f"{src} bf16_tflops_sustained",
+            "algorithmic_bytes_per_launch": bytes_call,
+            "flops_per_launch": flops_call, "launch_ms": attn_ms}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "rollouts_per_gpu": R, "layers": L, "heads": H,
+                   "head_dim": d, "grid": f"{w.grid_h}x{w.grid_w}",
+                   "action_tokens": w.action_tokens, "block_frames": F,
+                   "sink_frames": w.sink_frames, "window_frames": w.window_frames,
+                   "denoise_steps": S, "keys_per_rollout": nk[0] if len(set(nk)) == 1 else nk,
+                   "l2": "inputs larger than L2: every step reads all layers' caches and "
+                         "fresh q/k/v per (step, layer)",
+                   "parallelism": f"replicas x{world}"},
+        "latent_frames_per_s_per_layer": frames_per_s_layer,
+        "roofline": roof,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
+    """Same steps through the C ABI with the q/k/v of every call copied from
+    pinned host memory and every output copied back, inside the timed region.
+    Copies run on their own streams so they overlap the kernels."""
+    import torch
+    import torch.distributed as dist
+    from streaming_autoregressive_video_b200 import binding as fd
+
+    L, R, S = w.layers, w.rollouts, w.steps
+    hq = [t.cpu().pin_memory() for t in q[0]]
+    hk = [t.cpu().pin_memory() for t in k[0]]
+    hv = [t.cpu().pin_memory() for t in v[0]]
+    hout = [torch.empty(outs[0].shape, dtype=torch.int16).pin_memory() for _ in range(L)]
+    nbuf = 2
+    dq = [torch.empty_like(q[0][0]) for _ in range(nbuf)]
+    dk = [torch.empty_like(k[0][0]) for _ in range(nbuf)]
+    dv = [torch.empty_like(v[0][0]) for _ in range(nbuf)]
+    dout = [torch.empty_like(outs[0]) for _ in range(nbuf)]
+    klast = [torch.empty_like(k[0][0]) for _ in range(L)]
+    vlast = [torch.empty_like(v[0][0]) for _ in range(L)]
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(nbuf)]
+    done = [torch.cuda.Event() for _ in range(nbuf)]
+    freed = [torch.cuda.Event() for _ in range(nbuf)]
+    for e in freed:
+        e.record(d2h)
+    h2d_bytes = d2h_bytes = 0
+
+    def step():
+        nonlocal h2d_bytes, d2h_bytes
+        i = 0
+        for s in range(S):
+            last = s == S - 1
+            for l in range(L):
+                b = i % nbuf
+                kd = klast[l] if last else dk[b]
+                vd = vlast[l] if last else dv[b]
+                h2d.wait_event(freed[b])
+                with torch.cuda.stream(h2d):
+                    dq[b].copy_(hq[l], non_blocking=True)
+                    kd.copy_(hk[l], non_blocking=True)
+                    vd.copy_(hv[l], non_blocking=True)
+                ready[b].record(h2d)
+                stream.wait_event(ready[b])
+                fd.fd_block_attention(cache, l, R, dq[b], kd, vd, dout[b], stream=stream)
+                done[b].record(stream)
+                d2h.wait_event(done[b])
+                with torch.cuda.stream(d2h):
+                    hout[l].copy_(dout[b], non_blocking=True)
+                freed[b].record(d2h)
+                h2d_bytes += 3 * hq[l].numel() * 2
+                d2h_bytes += hout[l].numel() * 2
+                i += 1
+        fd.fd_cache_commit(cache, 0, L, R, klast, vlast, stream=stream)
+
+    for _ in range(max(2, min(3, args.warmup))):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    h2d_bytes = d2h_bytes = 0
+    steps = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    fin = torch.cuda.Event()
+    fin.record(d2h)
+    stream.wait_event(fin)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t[0])
+    return {"value": flops_step * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d_bytes // steps, "d2h_bytes_per_step": d2h_bytes // steps,
+            "ms_per_step": ms}
+
+
+def main():
+    args = parse_args()
+    w = workloads()[args.workload]
+    if args.layers:
+        w = w.scaled(layers=args.layers, name=w.name + f"-L{args.layers}")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_fd(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

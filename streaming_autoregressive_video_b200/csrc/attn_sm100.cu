@@ -90,7 +90,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
                                          Shared* sh, int32_t* err, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
@@ -214,6 +214,15 @@ __device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
   }
 }
 
+// End of every role branch: all 512 threads meet on named barrier 1 (each
+// warp arrives from its own branch), then warp 2 releases the TMEM columns.
+__device__ __forceinline__ void teardown(int warp, uint32_t tmem) {
+  tc_fence_before();
+  asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&r);
@@ -266,7 +275,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
-  if (warp == 0) {
+  // Register split (launch: 512 threads x 128): the producer/MMA warpgroup and
+  // the RoPE warpgroup give registers to the two softmax warpgroups, which
+  // keep a whole 128-column S row in registers.  72 + 72 + 184 + 184 = 4 x 128.
+  // Each warpgroup changes its count exactly once, at the top of its branch,
+  // and never takes registers back: a later increase could claim registers a
+  // softmax warpgroup is still waiting for.  Each branch ends in its own
+  // teardown (block-wide named barrier, then TMEM release) and returns, so no
+  // code runs after the branches join.
+  if (warp < 4) {
+    regs_dec<72>();
+    if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -317,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t sq = smem_addr(smem + kOffQ);
@@ -387,7 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+    }
+    teardown(warp, tmem);
+    return;
+  } else if (warp < 8) {
+    regs_dec<72>();
     // ------------------------------------------------------------ RoPE
     const int tid = threadIdx.x - 128;
     const RopeLane rl = rope_lane(p, tid);
@@ -410,7 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&sh->k_ready[ks]);
     }
-  } else if (warp >= 8) {
+    teardown(warp, tmem);
+    return;
+  } else {
+    regs_inc<184>();
     // ------------------------------------------------------------ softmax
     const int x = (warp - 8) >> 2;
     const int wq = warp & 3;
@@ -421,57 +447,71 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     uint32_t rr[32];
+    uint32_t sa[64], sb[64];
     for (int j = 0; j < tc.nt; ++j) {
       ok = __all_sync(0xffffffffu,
                       wait_bar(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
+      tmem_ld64(tS, sa);
+      tmem_ld64(tS + 64, sb);
       const int valid = j < tc.nt1 ? min(kBN, tc.n1 - j * kBN)
                                    : min(kBN, tc.n2 - (j - tc.nt1) * kBN);
-      float mx = -INFINITY;
+      if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        tmem_ld32(tS + c4 * 32, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c4 * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(rr[i]));
+        for (int i = 0; i < 64; ++i) {
+          if (i >= valid) sa[i] = 0xFF800000u;
+          if (64 + i >= valid) sb[i] = 0xFF800000u;
+        }
       }
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        m8[i] = fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i]));
+#pragma unroll
+      for (int i = 8; i < 64; ++i)
+        m8[i & 7] = fmaxf(m8[i & 7], fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i])));
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_tile = mx * sl2;
       const bool need = m_tile > m + kRescaleThreshold;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? exp2f(m - m_tile) : 1.f;
+        const float alpha = need ? ex2_approx(m - m_tile) : 1.f;
+#pragma unroll 1
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t r16[16];
+          tmem_ld16(tO + c8 * 16, r16);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          tmem_ld32(tO + c4 * 32, rr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-          tmem_st32(tO + c4 * 32, rr);
+          for (int i = 0; i < 16; ++i)
+            r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+          tmem_st16(tO + c8 * 16, r16);
         }
         tmem_wait_st();
       }
       if (need) {
-        l = (j > 0) ? l * exp2f(m - m_tile) : 0.f;
+        l = (j > 0) ? l * ex2_approx(m - m_tile) : 0.f;
         m = m_tile;
       }
-      float lsum = 0.f;
+      const float neg_m = -m;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        tmem_ld32(tS + c4 * 32, rr);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c0 = c4 * 32 + 2 * i;
-          const float p0 = c0 < valid
-              ? exp2f(fmaf(__uint_as_float(rr[2 * i]), sl2, -m)) : 0.f;
-          const float p1 = c0 + 1 < valid
-              ? exp2f(fmaf(__uint_as_float(rr[2 * i + 1]), sl2, -m)) : 0.f;
-          lsum += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tS + c4 * 16, pk);
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sa[2 * i]), sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sa[2 * i + 1]), sl2, neg_m));
+        ls[i & 3] += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
       }
-      l += lsum;
+      tmem_st32(tS, pk);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sb[2 * i]), sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sb[2 * i + 1]), sl2, neg_m));
+        ls[i & 3] += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      tmem_st32(tS + 32, pk);
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sh->p_full[x]);
@@ -504,12 +544,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[((size_t)r * p.H + h) * p.Mq + row] =
             (m + log2f(l)) * 0.69314718055994530942f;
     }
+    teardown(warp, tmem);
+    return;
   }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
@@ -522,9 +559,16 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const AttnParams& p, cudaStream_t s) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(
-        attn_bf16_d128_sm100, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kSmemBytes);
+    // The warpgroup register split (setmaxnreg) assumes the block launches
+    // with exactly 128 registers per thread; refuse to launch otherwise, as
+    // the increase would wait forever for registers that do not exist.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bf16_d128_sm100);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != 128) return cudaErrorNotSupported;
+    e = cudaFuncSetAttribute(attn_bf16_d128_sm100,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
