@@ -12,7 +12,7 @@
 //
 // Design (one CTA = two 128-row query tiles of one (rollout, head)):
 //   warp 0        TMA producer: Q tiles once, then K and V tiles through
-//                 3-stage (K) and 2-stage (V) shared-memory rings, walking
+//                 2-stage K and V shared-memory rings, walking
 //                 the valid slot prefix of the cache and then the block; the
 //                 ring's wraparound needs no gather because attention does
 //                 not depend on key order.  No cluster multicast.
@@ -54,7 +54,7 @@ constexpr int kBN = 128;  // keys per tile
 constexpr int kD = 128;   // head dim handled by this kernel
 constexpr uint32_t kTile = kBM * kD * 2;  // 32 KB (bf16)
 constexpr uint32_t kHalf = kTile / 2;     // one 64-column, 128-byte-swizzled half
-constexpr int kKStages = 3;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = 2 * kTile;
@@ -80,8 +80,11 @@ struct Shared {
   int32_t abort;
 };
 
-constexpr uint32_t kSmemBytes = kOffShared + sizeof(Shared) + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+// RoPE tables follow the barriers; the dynamic size adds them per launch.
+constexpr uint32_t kOffTab = kOffShared + 256;
+static_assert(sizeof(Shared) <= 256, "barrier block");
+constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
+constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
 
 // Site codes for the device error word.
 enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4 };
@@ -129,9 +132,14 @@ __device__ __forceinline__ TileCounts tile_counts(const AttnParams& p, int r) {
 // of every row (8 bf16 = 4 rotation pairs: pairs 4cc..4cc+3) and rows
 // tid/16 + 8m.  A 128-byte-swizzled row keeps each 16-byte chunk intact, so
 // the pairs of a chunk stay together; only the chunk's position moves.
+// cos/sin come from one table in shared memory: [t rows of this rollout |
+// h rows | w rows].  A lane's pair p reads entry off[p] + coord * stride[p],
+// where coord is the key's t-row, h or w; the choice is a select, not a
+// branch, so the lanes of a warp never diverge on the lookup.
 struct RopeLane {
-  int sec[4];  // 0 = t, 1 = h, 2 = w
-  int j[4];    // pair index within its section
+  int sec[4];     // 0 = t, 1 = h, 2 = w
+  int off[4];     // section base + pair index within the section
+  int stride[4];  // pairs of the section
   int half, chunk, row0;
 };
 
@@ -141,46 +149,51 @@ __device__ __forceinline__ RopeLane rope_lane(const AttnParams& p, int tid) {
   rl.half = cc >> 3;
   rl.chunk = cc & 7;
   rl.row0 = tid >> 4;
+  const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int pair = cc * 4 + e;
-    if (pair < p.pt) { rl.sec[e] = 0; rl.j[e] = pair; }
-    else if (pair < p.pt + p.ph) { rl.sec[e] = 1; rl.j[e] = pair - p.pt; }
-    else { rl.sec[e] = 2; rl.j[e] = pair - p.pt - p.ph; }
+    if (pair < p.pt) {
+      rl.sec[e] = 0; rl.off[e] = pair; rl.stride[e] = p.pt;
+    } else if (pair < p.pt + p.ph) {
+      rl.sec[e] = 1; rl.off[e] = n_t + pair - p.pt; rl.stride[e] = p.ph;
+    } else {
+      rl.sec[e] = 2; rl.off[e] = n_t + n_h + pair - p.pt - p.ph; rl.stride[e] = p.pw;
+    }
   }
   return rl;
 }
 
 __device__ __forceinline__ void rotate_chunk(uint8_t* tile, int row,
                                              const RopeLane& rl,
-                                             const AttnParams& p,
-                                             const float2* tt, int tidx,
+                                             const float2* tab, int tidx,
                                              int hh, int ww) {
+  float2 cs[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int coord = rl.sec[e] == 0 ? tidx : (rl.sec[e] == 1 ? hh : ww);
+    cs[e] = tab[rl.off[e] + coord * rl.stride[e]];
+  }
   uint4* ptr = reinterpret_cast<uint4*>(tile + rl.half * kHalf + row * 128 +
                                         ((rl.chunk ^ (row & 7)) << 4));
   uint4 u = *ptr;
   uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const float2* src;
-    if (rl.sec[e] == 0) src = tt + tidx * p.pt + rl.j[e];
-    else if (rl.sec[e] == 1) src = p.htab + hh * p.ph + rl.j[e];
-    else src = p.wtab + ww * p.pw + rl.j[e];
-    const float2 cs = __ldg(src);
     const float a = __uint_as_float(w4[e] << 16);
     const float b = __uint_as_float(w4[e] & 0xFFFF0000u);
-    const __nv_bfloat162 r2 =
-        __floats2bfloat162_rn(a * cs.x - b * cs.y, a * cs.y + b * cs.x);
+    const __nv_bfloat162 r2 = __floats2bfloat162_rn(
+        a * cs[e].x - b * cs[e].y, a * cs[e].y + b * cs[e].x);
     w4[e] = *reinterpret_cast<const uint32_t*>(&r2);
   }
   *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
 }
 
-// Rotate the 128 query rows of tile `qt` (rows past Mq are zero: skipped).
+// Rotate the 128 query rows of a Q tile (rows past Mq are zero: skipped).
 __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
                                             const RopeLane& rl,
-                                            const AttnParams& p,
-                                            const float2* tt) {
+                                            const float2* tab,
+                                            const AttnParams& p) {
 #pragma unroll 4
   for (int m = 0; m < 16; ++m) {
     const int row = rl.row0 + 8 * m;
@@ -189,15 +202,15 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
     const int f = (int)fast_div((uint32_t)q, p.div_T);
     const int tok = q - f * p.T;
     const int hh = (int)fast_div((uint32_t)tok, p.div_gw);
-    rotate_chunk(tile, row, rl, p, tt, p.slots + f, hh, tok - hh * p.gw);
+    rotate_chunk(tile, row, rl, tab, p.slots + f, hh, tok - hh * p.gw);
   }
 }
 
 // Rotate the valid keys of one K tile (keys key0..key0+127 of a segment).
 __device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
                                             bool seg1, const RopeLane& rl,
-                                            const AttnParams& p,
-                                            const float2* tt) {
+                                            const float2* tab,
+                                            const AttnParams& p) {
 #pragma unroll 4
   for (int m = 0; m < 16; ++m) {
     const int row = rl.row0 + 8 * m;
@@ -210,7 +223,7 @@ __device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
       hh = (int)fast_div((uint32_t)tok, p.div_gw);
       ww = tok - hh * p.gw;
     }
-    rotate_chunk(tile, row, rl, p, tt, seg1 ? fi : p.slots + fi, hh, ww);
+    rotate_chunk(tile, row, rl, tab, seg1 ? fi : p.slots + fi, hh, ww);
   }
 }
 
@@ -277,14 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Register split (launch: 512 threads x 128): the producer/MMA warpgroup and
   // the RoPE warpgroup give registers to the two softmax warpgroups, which
-  // keep a whole 128-column S row in registers.  72 + 72 + 184 + 184 = 4 x 128.
+  // keep a whole 128-column S row in registers.  88 + 72 + 176 + 176 = 4 x 128.
   // Each warpgroup changes its count exactly once, at the top of its branch,
   // and never takes registers back: a later increase could claim registers a
   // softmax warpgroup is still waiting for.  Each branch ends in its own
   // teardown (block-wide named barrier, then TMEM release) and returns, so no
   // code runs after the branches join.
   if (warp < 4) {
-    regs_dec<72>();
+    regs_dec<88>();
     if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -414,11 +427,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ RoPE
     const int tid = threadIdx.x - 128;
     const RopeLane rl = rope_lane(p, tid);
-    const float2* tt = p.ttab + (size_t)r * (p.slots + p.F) * p.pt;
+    // stage this rollout's t table and the static h / w tables
+    float2* st = reinterpret_cast<float2*>(smem + kOffTab);
+    const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph, n_w = p.gw * p.pw;
+    const float2* tt = p.ttab + (size_t)r * n_t;
+    for (int i = tid; i < n_t; i += 128) st[i] = tt[i];
+    for (int i = tid; i < n_h; i += 128) st[n_t + i] = p.htab[i];
+    for (int i = tid; i < n_w; i += 128) st[n_t + n_h + i] = p.wtab[i];
+    asm volatile("bar.sync 2, 128;" ::: "memory");
     bool ok = __all_sync(0xffffffffu, wait_bar(&sh->q_full, 0, sh, p.err, kSiteRope));
     if (ok) {
-      rope_q_tile(smem + kOffQ, qrow0, rl, p, tt);
-      rope_q_tile(smem + kOffQ + kTile, qrow0 + kBM, rl, p, tt);
+      rope_q_tile(smem + kOffQ, qrow0, rl, st, p);
+      rope_q_tile(smem + kOffQ + kTile, qrow0 + kBM, rl, st, p);
       fence_proxy_async_smem();
     }
     mbar_arrive(&sh->q_ready);
@@ -429,14 +449,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const bool seg1 = j < tc.nt1;
       rope_k_tile(smem + kOffK + ks * kTile, seg1 ? j * kBN : (j - tc.nt1) * kBN,
-                  seg1 ? tc.n1 : tc.n2, seg1, rl, p, tt);
+                  seg1 ? tc.n1 : tc.n2, seg1, rl, st, p);
       fence_proxy_async_smem();
       mbar_arrive(&sh->k_ready[ks]);
     }
     teardown(warp, tmem);
     return;
   } else {
-    regs_inc<184>();
+    regs_inc<176>();
     // ------------------------------------------------------------ softmax
     const int x = (warp - 8) >> 2;
     const int wq = warp & 3;
@@ -568,12 +588,16 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
     if (fa.numRegs != 128) return cudaErrorNotSupported;
     e = cudaFuncSetAttribute(attn_bf16_d128_sm100,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
+                             (int)kSmemMax);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
+                                        (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
+  const size_t smem = kSmemFixed + tab;
+  if (smem > kSmemMax) return cudaErrorNotSupported;
   dim3 grid((p.Mq + 2 * kBM - 1) / (2 * kBM), p.H, p.n_rollouts);
-  attn_bf16_d128_sm100<<<grid, kThreads, kSmemBytes, s>>>(tm_q, tm_kc, tm_vc,
+  attn_bf16_d128_sm100<<<grid, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc,
                                                           tm_kb, tm_vb, p);
   count_launch(1);
   return cudaGetLastError();

@@ -351,6 +351,7 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   p.d = c.d;
   p.T = c.T;
   p.Tf = c.Tf;
+  p.gh = c.gh;
   p.gw = c.gw;
   p.F = c.F;
   p.S = c.S;

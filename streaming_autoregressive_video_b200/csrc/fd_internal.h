@@ -80,7 +80,7 @@ struct AttnParams {
   int32_t* err;
   const uint8_t* kc;     // cache K of the layer, rollout 0 (CUDA-core path)
   const uint8_t* vc;
-  int H, d, T, Tf, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
+  int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
   int map_row0;          // layer * R: row offset of this layer in the cache maps
   FastDiv div_T, div_Tf, div_gw;
   float scale_log2;      // log2(e) / sqrt(d)
