@@ -35,7 +35,9 @@
  *     (h, w) = (i / grid_w, i % grid_w), action tokens at (0, 0); t is the
  *     absolute frame index since the last reset;
  *   - the cache stores K/V as committed (pre-RoPE) plus an int32 frame
- *     position per slot; RoPE is applied to cached keys as they are loaded.
+ *     position per slot; a cached key's rotation depends only on that
+ *     position, so the commit also stores it rotated (krot) and attention
+ *     applies RoPE in its loads only to the block's own keys and queries.
  *
  * Conventions for every call:
  *   - all pointers to tensors are DEVICE pointers on the device that owns the
@@ -91,7 +93,12 @@ typedef struct {
 } fd_cache_desc;
 
 /* Byte offsets of the regions inside the caller's storage buffer.
- *   k, v : [L][R][S+W][Tf][H][d] elements of `dtype`
+ *   k, v : [L][R][S+W][Tf][H][d] elements of `dtype`, exactly as committed
+ *   krot : [L][R][S+W][Tf][H][d] the same keys rotated by 3D RoPE to their
+ *          frame's position, written by the commit (a committed frame and its
+ *          position never change, so its rotation is computed once instead
+ *          of at every attention call); derived data, not part of the
+ *          cache's observable state
  *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
  *   count: [L][R] int32, frames committed since the last reset (n)
  *   ttab : [L][R][S+W+F][p_t] float2 (cos, sin) of the t-section angles for
@@ -99,7 +106,7 @@ typedef struct {
  *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
  *   err  : int32 device error word (0 = none)                            */
 typedef struct {
-  size_t k, v, pos, count, ttab, htab, wtab, err;
+  size_t k, v, krot, pos, count, ttab, htab, wtab, err;
   size_t total;           /* == fd_cache_bytes(desc)                       */
   size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
   int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
@@ -167,9 +174,10 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
 
 /* Ring-buffer commit for layers [layer_begin, layer_end) -- the finalize()
  * half of [FD-HP]:  for every rollout r < n_rollouts and f < frames_r,
- * slot = slot_of(n_r + f) receives frame f of k[l]/v[l] bit for bit,
- * pos[slot] = n_r + f; then n_r += frames_r and the rollout's t table is
- * rebuilt.  Once the window is full this evicts the oldest window frames.
+ * slot = slot_of(n_r + f) receives frame f of k[l]/v[l] bit for bit (and its
+ * keys rotated to t = n_r + f in the krot region), pos[slot] = n_r + f; then
+ * n_r += frames_r and the rollout's t table is rebuilt.  Once the window is
+ * full this evicts the oldest window frames.
  *   frames (host) [n_rollouts], each in [0, F]; NULL = F for every rollout
  *   (a ragged prefill commits fewer frames for some rollouts);
  *   k, v (host arrays of device pointers) [layer_end - layer_begin], each

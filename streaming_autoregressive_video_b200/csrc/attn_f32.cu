@@ -108,9 +108,14 @@ __global__ void __launch_bounds__(kWarps * 32)
             : (((size_t)r * p.F * p.Tf + key) * p.H + h) * D + 2 * pair;
         const float* ks = (seg1 ? kcg : kg) + off;
         const float* vs = (seg1 ? vcg : vg) + off;
-        const float2 cs = rope_cs(p, tt, pair, kc);
-        a = ks[0] * cs.x - ks[1] * cs.y;
-        b = ks[0] * cs.y + ks[1] * cs.x;
+        if (seg1) {  // cached keys were rotated when their frame was committed
+          a = ks[0];
+          b = ks[1];
+        } else {
+          const float2 cs = rope_cs(p, tt, pair, kc);
+          a = ks[0] * cs.x - ks[1] * cs.y;
+          b = ks[0] * cs.y + ks[1] * cs.x;
+        }
         va = vs[0];
         vb = vs[1];
       }

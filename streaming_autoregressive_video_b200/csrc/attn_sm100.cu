@@ -206,9 +206,10 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
   }
 }
 
-// Rotate the valid keys of one K tile (keys key0..key0+127 of a segment).
+// Rotate the valid keys of one K tile of the block (keys key0..key0+127);
+// block frame f sits at t-row slots + f of the table (t = n + f).
 __device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
-                                            bool seg1, const RopeLane& rl,
+                                            const RopeLane& rl,
                                             const float2* tab,
                                             const AttnParams& p) {
 #pragma unroll 4
@@ -223,7 +224,7 @@ __device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
       hh = (int)fast_div((uint32_t)tok, p.div_gw);
       ww = tok - hh * p.gw;
     }
-    rotate_chunk(tile, row, rl, tab, seg1 ? fi : p.slots + fi, hh, ww);
+    rotate_chunk(tile, row, rl, tab, p.slots + fi, hh, ww);
   }
 }
 
@@ -373,8 +374,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = wait_bar(&sh->q_ready, 0, sh, p.err, kSiteMma) &&
-                wait_bar(&sh->k_ready[0], 0, sh, p.err, kSiteMma);
+      // K tile j is ready once the RoPE warpgroup has passed it: it steps
+      // through every tile in order (rotating only the block's own tiles;
+      // cache tiles hold keys rotated at commit), so the phases of k_full and
+      // k_ready advance together and no waiter can fall two phases behind.
+      auto wait_k = [&](int j) -> bool {
+        return wait_bar(&sh->k_ready[j % kKStages], (j / kKStages) & 1, sh,
+                        p.err, kSiteMma);
+      };
+      bool ok = wait_bar(&sh->q_ready, 0, sh, p.err, kSiteMma) && wait_k(0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -392,8 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool more = j + 1 < tc.nt;
           const int ks = (j + 1) % kKStages;
           if (more) {
-            ok = wait_bar(&sh->k_ready[ks], ((j + 1) / kKStages) & 1, sh, p.err,
-                          kSiteMma);
+            ok = wait_k(j + 1);
             if (!ok) break;
             tc_fence_after();
             issue_s(0, ks);
@@ -442,15 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
     }
     mbar_arrive(&sh->q_ready);
+    // Every K tile passes through here in order; only the block's own tiles
+    // need rotating (cache tiles come from the rotated-key region).
     for (int j = 0; j < tc.nt && ok; ++j) {
       const int ks = j % kKStages;
       ok = __all_sync(0xffffffffu, wait_bar(&sh->k_full[ks], (j / kKStages) & 1,
                                             sh, p.err, kSiteRope));
       if (!ok) break;
-      const bool seg1 = j < tc.nt1;
-      rope_k_tile(smem + kOffK + ks * kTile, seg1 ? j * kBN : (j - tc.nt1) * kBN,
-                  seg1 ? tc.n1 : tc.n2, seg1, rl, st, p);
-      fence_proxy_async_smem();
+      if (j >= tc.nt1) {
+        rope_k_tile(smem + kOffK + ks * kTile, (j - tc.nt1) * kBN, tc.n2, rl, st, p);
+        fence_proxy_async_smem();
+      }
       mbar_arrive(&sh->k_ready[ks]);
     }
     teardown(warp, tmem);

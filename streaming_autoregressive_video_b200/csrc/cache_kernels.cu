@@ -69,14 +69,63 @@ __global__ void cache_init_kernel(CacheView c) {
   if (threadIdx.x == 0) c.err[0] = 0;
 }
 
-// One block copies a 64 KB chunk of one frame of one tensor (K or V) of one
-// (layer, rollout) into the frame's ring slot.  16-byte vectors, 16 per
-// thread in flight.  grid = (chunks per frame, nl * nr * 2 * F).
+// 3D RoPE of the pairs held by one 16-byte vector (4 bf16 pairs or 2 fp32
+// pairs) whose first pair is `pair0`, for a token whose t-section cos/sin row
+// is `tt_row` and whose grid coordinates are (hh, ww).
+template <typename Elem>
+__device__ __forceinline__ uint4 rotate16(uint4 u, int pair0,
+                                          const CacheView& c,
+                                          const float2* tt_row, int hh,
+                                          int ww) {
+  constexpr int kPairs = 8 / sizeof(Elem);
+  float vals[2 * kPairs];
+  const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+  if constexpr (sizeof(Elem) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      vals[2 * i] = __uint_as_float(w4[i] << 16);
+      vals[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vals[i] = __uint_as_float(w4[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {
+    const int pair = pair0 + i;
+    float2 cs;
+    if (pair < c.pt) cs = __ldg(tt_row + pair);
+    else if (pair < c.pt + c.ph) cs = __ldg(c.htab + hh * c.ph + (pair - c.pt));
+    else cs = __ldg(c.wtab + ww * c.pw + (pair - c.pt - c.ph));
+    const float a = vals[2 * i], b = vals[2 * i + 1];
+    vals[2 * i] = a * cs.x - b * cs.y;
+    vals[2 * i + 1] = a * cs.y + b * cs.x;
+  }
+  uint32_t o4[4];
+  if constexpr (sizeof(Elem) == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(vals[2 * i], vals[2 * i + 1]);
+      o4[i] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o4[i] = __float_as_uint(vals[i]);
+  }
+  return make_uint4(o4[0], o4[1], o4[2], o4[3]);
+}
+
+// One block copies a 64 KB chunk of one frame of K or V of one (layer,
+// rollout) into the frame's ring slot; K chunks also go, rotated to the
+// frame's position t = n + f, into the rotated-key region.  16-byte vectors,
+// 16 per thread in flight.  grid = (chunks per frame, nl * nr * 2 * F).
 constexpr int kCopyThreads = 256;
 constexpr int kCopyVecs = 16;
 
+template <typename Elem>
 __global__ void __launch_bounds__(kCopyThreads)
     commit_copy_kernel(CacheView c, CommitParams p) {
+  constexpr int kPer = 16 / sizeof(Elem);
   const int job = blockIdx.y;
   const int f = job % c.F;
   const int kv = (job / c.F) & 1;
@@ -84,15 +133,15 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int li = job / c.F / 2 / p.nr;
   if (f >= p.frames[ri]) return;
   const int l = p.layer0 + li, r = p.rollout0 + ri;
-  const int n = c.count[(size_t)l * c.R + r];
+  const size_t lr = (size_t)l * c.R + r;
+  const int n = c.count[lr];
   const int slot = slot_of(n + f, c.S, c.W);
   const uint64_t fvecs = c.frame_bytes / 16;
   const uint8_t* src_base = kv ? p.v[li] : p.k[li];
   const uint4* src = reinterpret_cast<const uint4*>(
       src_base + ((uint64_t)r * c.F + f) * c.frame_bytes);
-  uint8_t* dst_base = kv ? c.v : c.k;
-  uint4* dst = reinterpret_cast<uint4*>(
-      dst_base + (((uint64_t)l * c.R + r) * c.slots + slot) * c.frame_bytes);
+  const uint64_t dst_off = (lr * c.slots + slot) * c.frame_bytes;
+  uint4* dst = reinterpret_cast<uint4*>((kv ? c.v : c.k) + dst_off);
   const uint64_t v0 = (uint64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
   uint4 buf[kCopyVecs];
 #pragma unroll
@@ -104,6 +153,25 @@ __global__ void __launch_bounds__(kCopyThreads)
   for (int i = 0; i < kCopyVecs; ++i) {
     const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
     if (vi < fvecs) dst[vi] = buf[i];
+  }
+  if (kv) return;
+  // rotated keys: the ttab row slots + f holds frame n + f (the next block)
+  uint4* rdst = reinterpret_cast<uint4*>(c.krot + dst_off);
+  const float2* tt_row = c.ttab + (lr * (c.slots + c.F) + c.slots + f) * c.pt;
+  const uint32_t vec_per_row = c.d / kPer;
+  const uint32_t vec_per_tok = vec_per_row * c.H;
+#pragma unroll
+  for (int i = 0; i < kCopyVecs; ++i) {
+    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
+    if (vi >= fvecs) continue;
+    const uint32_t tok = (uint32_t)(vi / vec_per_tok);
+    const int pair0 = (int)(vi % vec_per_row) * (kPer / 2);
+    int hh = 0, ww = 0;
+    if ((int)tok < c.T) {
+      hh = (int)tok / c.gw;
+      ww = (int)tok - hh * c.gw;
+    }
+    rdst[vi] = rotate16<Elem>(buf[i], pair0, c, tt_row, hh, ww);
   }
 }
 
@@ -124,17 +192,18 @@ __global__ void commit_meta_kernel(CacheView c, CommitParams p) {
   fill_ttab(c, l, r, n + nf, pos);
 }
 
-// Zero the K/V of the listed rollouts in every layer.
-// grid = (chunks per (layer, rollout) region, L * n * 2)
+// Zero the K, V and rotated K of the listed rollouts in every layer.
+// grid = (chunks per (layer, rollout) region, L * n * 3)
 __global__ void __launch_bounds__(kCopyThreads)
     reset_zero_kernel(CacheView c, ResetParams p) {
   const int job = blockIdx.y;
-  const int kv = job & 1;
-  const int id = (job >> 1) % p.n;
-  const int l = (job >> 1) / p.n;
+  const int kv = job % 3;
+  const int id = (job / 3) % p.n;
+  const int l = (job / 3) / p.n;
   const int r = p.ids[id];
   const uint64_t region = (uint64_t)c.slots * c.frame_bytes;
-  uint8_t* base = (kv ? c.v : c.k) + ((uint64_t)l * c.R + r) * region;
+  uint8_t* tensor = kv == 0 ? c.k : (kv == 1 ? c.v : c.krot);
+  uint8_t* base = tensor + ((uint64_t)l * c.R + r) * region;
   uint4* dst = reinterpret_cast<uint4*>(base);
   const uint64_t nvec = region / 16;
   const uint64_t v0 = (uint64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
@@ -177,41 +246,8 @@ __global__ void rope3d_kernel(CacheView c, int layer, int n_rollouts,
     const int hh = tok < c.T ? tok / c.gw : 0;
     const int ww = tok < c.T ? tok % c.gw : 0;
     Elem* px = x + ci * kPer;
-    float vals[kPer];
-    if constexpr (sizeof(Elem) == 2) {
-      const uint4 u = *reinterpret_cast<const uint4*>(px);
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        vals[2 * i] = __uint_as_float(w4[i] << 16);
-        vals[2 * i + 1] = __uint_as_float(w4[i] & 0xFFFF0000u);
-      }
-    } else {
-      const float4 u = *reinterpret_cast<const float4*>(px);
-      vals[0] = u.x; vals[1] = u.y; vals[2] = u.z; vals[3] = u.w;
-    }
-#pragma unroll
-    for (int i = 0; i < kPer / 2; ++i) {
-      const int pair = cc * (kPer / 2) + i;
-      float2 cs;
-      if (pair < c.pt) cs = tt[pair];
-      else if (pair < c.pt + c.ph) cs = c.htab[hh * c.ph + (pair - c.pt)];
-      else cs = c.wtab[ww * c.pw + (pair - c.pt - c.ph)];
-      const float a = vals[2 * i], b = vals[2 * i + 1];
-      vals[2 * i] = a * cs.x - b * cs.y;
-      vals[2 * i + 1] = a * cs.y + b * cs.x;
-    }
-    if constexpr (sizeof(Elem) == 2) {
-      uint32_t w4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(vals[2 * i], vals[2 * i + 1]);
-        w4[i] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      *reinterpret_cast<uint4*>(px) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    } else {
-      *reinterpret_cast<float4*>(px) = make_float4(vals[0], vals[1], vals[2], vals[3]);
-    }
+    const uint4 u = *reinterpret_cast<const uint4*>(px);
+    *reinterpret_cast<uint4*>(px) = rotate16<Elem>(u, cc * (kPer / 2), c, tt, hh, ww);
   }
 }
 
@@ -229,7 +265,10 @@ cudaError_t launch_commit(const CacheView& c, const CommitParams& p,
   const uint64_t chunks = (fvecs + kCopyThreads * kCopyVecs - 1) /
                           (kCopyThreads * kCopyVecs);
   dim3 grid((unsigned)chunks, (unsigned)(p.nl * p.nr * 2 * c.F));
-  commit_copy_kernel<<<grid, kCopyThreads, 0, s>>>(c, p);
+  if (c.esz == 2)
+    commit_copy_kernel<uint16_t><<<grid, kCopyThreads, 0, s>>>(c, p);
+  else
+    commit_copy_kernel<float><<<grid, kCopyThreads, 0, s>>>(c, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   commit_meta_kernel<<<p.nl * p.nr, 128, 0, s>>>(c, p);
@@ -242,7 +281,7 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
   const uint64_t nvec = (uint64_t)c.slots * c.frame_bytes / 16;
   const uint64_t chunks = (nvec + kCopyThreads * kCopyVecs - 1) /
                           (kCopyThreads * kCopyVecs);
-  dim3 grid((unsigned)chunks, (unsigned)(c.L * p.n * 2));
+  dim3 grid((unsigned)chunks, (unsigned)(c.L * p.n * 3));
   reset_zero_kernel<<<grid, kCopyThreads, 0, s>>>(c, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

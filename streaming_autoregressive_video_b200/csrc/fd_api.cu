@@ -81,6 +81,8 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   off = align_up(off + kv);
   lay->v = off;
   off = align_up(off + kv);
+  lay->krot = off;
+  off = align_up(off + kv);
   lay->pos = off;
   off = align_up(off + lr * slots * sizeof(int32_t));
   lay->count = off;
@@ -201,6 +203,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   fd::CacheView& v = c->view;
   v.k = base + lay.k;
   v.v = base + lay.v;
+  v.krot = base + lay.krot;
   v.pos = reinterpret_cast<int32_t*>(base + lay.pos);
   v.count = reinterpret_cast<int32_t*>(base + lay.count);
   v.ttab = reinterpret_cast<float2*>(base + lay.ttab);
@@ -230,7 +233,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   if (desc->dtype == FD_BF16) {
     const uint64_t rows = (uint64_t)v.slots * v.Tf;
     const uint64_t batch = (uint64_t)v.L * v.R;
-    if (!fd::encode_bf16_map(&c->tm_kc, v.k, v.d, v.H, rows, batch) ||
+    if (!fd::encode_bf16_map(&c->tm_kc, v.krot, v.d, v.H, rows, batch) ||
         !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.H, rows, batch)) {
       // only the tensor-core path needs the maps; keep going without them
       c->have_maps = false;
@@ -345,7 +348,7 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   p.out = out;
   p.lse = lse;
   p.err = c.err;
-  p.kc = c.k + (size_t)layer * cache->layout.layer_kv_bytes;
+  p.kc = c.krot + (size_t)layer * cache->layout.layer_kv_bytes;
   p.vc = c.v + (size_t)layer * cache->layout.layer_kv_bytes;
   p.H = c.H;
   p.d = c.d;

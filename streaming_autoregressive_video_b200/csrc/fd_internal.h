@@ -34,6 +34,7 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
 struct CacheView {
   uint8_t* k;
   uint8_t* v;
+  uint8_t* krot;  // committed keys rotated to their frame's position
   int32_t* pos;
   int32_t* count;
   float2* ttab;
@@ -78,7 +79,7 @@ struct AttnParams {
   void* out;
   float* lse;
   int32_t* err;
-  const uint8_t* kc;     // cache K of the layer, rollout 0 (CUDA-core path)
+  const uint8_t* kc;     // rotated cache K of the layer, rollout 0 (CUDA cores)
   const uint8_t* vc;
   int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
   int map_row0;          // layer * R: row offset of this layer in the cache maps

@@ -41,6 +41,32 @@ def views(cache, w):
     return k, v, pos, count
 
 
+def krot_view(cache, w):
+    """The cache's committed keys rotated to their frame positions."""
+    lay = cache.layout
+    esz = 2 if w.dtype == "bf16" else 4
+    n_kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.heads * w.head_dim
+    kv_dt = torch.int16 if esz == 2 else torch.float32
+    shape = (w.layers, w.rollouts, w.slots, w.frame_tokens, w.heads, w.head_dim)
+    return cache.storage[lay.krot:lay.krot + n_kv * esz].view(kv_dt).view(shape)
+
+
+def check_rotated(got_storage: np.ndarray, raw: np.ndarray, t, w, what=""):
+    """got = RoPE(raw) at frame positions t (one entry per frame), within one
+    rounding to the storage dtype of the fp64 rotation."""
+    h, ww = oracle.token_coords(w.frame_tokens, w.tokens, w.grid_w)
+    t = np.asarray(t, dtype=np.float64)[:, None]
+    ang = oracle.rope_angles(t, h[None, :], ww[None, :], w.head_dim, w.theta)[:, :, None, :]
+    want = oracle.rope_rotate(oracle.values_f64(raw, w.dtype), ang)
+    got = oracle.values_f64(got_storage, w.dtype)
+    err = np.abs(got - want)
+    if w.dtype == "bf16":
+        bound = np.abs(want) * 2.0 ** -8 + 1e-30
+    else:
+        bound = np.abs(want) * 1e-6 + 1e-6
+    assert np.all(err <= bound), f"{what}: rotated keys off by {float(err.max()):.3g}"
+
+
 def to_device(a: np.ndarray, device="cuda") -> torch.Tensor:
     if a.dtype == np.uint16:
         return torch.from_numpy(a.view(np.int16).copy()).to(device)
@@ -159,3 +185,14 @@ class Lockstep:
                 assert np.array_equal(k[l, r, :nv], o.k[:nv]), ("K", l, r)
                 assert np.array_equal(v[l, r, :nv], o.v[:nv]), ("V", l, r)
                 assert fd.fd_cache_frames(self.cache, l, r) == o.n
+
+    def check_rotated_keys(self):
+        """The rotated-key region holds every valid slot's keys at its frame position."""
+        w = self.w
+        kr = to_host(krot_view(self.cache, w))
+        for l in range(w.layers):
+            for r in range(w.rollouts):
+                o = self.orc[l][r]
+                nv = o.valid_slots()
+                if nv:
+                    check_rotated(kr[l, r, :nv], o.k[:nv], o.pos[:nv], w, f"krot l={l} r={r}")

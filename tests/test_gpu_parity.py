@@ -40,9 +40,11 @@ def test_commit_and_reset_bit_exact(dtype):
         frames = None if blk % 2 else [int(x) for x in rng.integers(0, w.block_frames + 1, w.rollouts)]
         _commit_block(ls, w, 100 + blk, frames=frames)
         ls.check_cache_exact()
+        ls.check_rotated_keys()
         if blk == 5:
             ls.reset([1])
             ls.check_cache_exact()
+            ls.check_rotated_keys()
     assert fd.fd_get_device_error(ls.cache) == 0
 
 
