@@ -36,8 +36,9 @@
  *     absolute frame index since the last reset;
  *   - the cache stores K/V as committed (pre-RoPE) plus an int32 frame
  *     position per slot; a cached key's rotation depends only on that
- *     position, so the commit also stores it rotated (krot) and attention
- *     applies RoPE in its loads only to the block's own keys and queries.
+ *     position, so the commit also stores it rotated (krot).  Each attention
+ *     call rotates the block's keys once into a work area (kblk) that all
+ *     query tiles read, and rotates each query tile as it is loaded.
  *
  * Conventions for every call:
  *   - all pointers to tensors are DEVICE pointers on the device that owns the
@@ -99,6 +100,10 @@ typedef struct {
  *          position never change, so its rotation is computed once instead
  *          of at every attention call); derived data, not part of the
  *          cache's observable state
+ *   kblk : [L][R][F*Tf][H][d] work area of fd_block_attention: the current
+ *          block's keys rotated once per call, read by every query tile
+ *          (one region per layer, so calls on different layers may run
+ *          concurrently; calls on the same layer must be ordered)
  *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
  *   count: [L][R] int32, frames committed since the last reset (n)
  *   ttab : [L][R][S+W+F][p_t] float2 (cos, sin) of the t-section angles for
@@ -106,7 +111,7 @@ typedef struct {
  *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
  *   err  : int32 device error word (0 = none)                            */
 typedef struct {
-  size_t k, v, krot, pos, count, ttab, htab, wtab, err;
+  size_t k, v, krot, kblk, pos, count, ttab, htab, wtab, err;
   size_t total;           /* == fd_cache_bytes(desc)                       */
   size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
   int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;

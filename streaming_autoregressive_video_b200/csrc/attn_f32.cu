@@ -100,22 +100,15 @@ __global__ void __launch_bounds__(kWarps * 32)
       const int key = key0 + kr;
       float a = 0.f, b = 0.f, va = 0.f, vb = 0.f;
       if (key < nseg) {
-        const int fi = key / p.Tf, tok = key - fi * p.Tf;
-        const KeyCoord kc{seg1 ? fi : p.slots + fi, tok < p.T ? tok / p.gw : 0,
-                          tok < p.T ? tok % p.gw : 0};
         const size_t off = seg1
             ? (((size_t)r * p.slots * p.Tf + key) * p.H + h) * D + 2 * pair
             : (((size_t)r * p.F * p.Tf + key) * p.H + h) * D + 2 * pair;
+        // keys arrive rotated: cached frames were rotated when committed, the
+        // block's keys once per call before this kernel
         const float* ks = (seg1 ? kcg : kg) + off;
         const float* vs = (seg1 ? vcg : vg) + off;
-        if (seg1) {  // cached keys were rotated when their frame was committed
-          a = ks[0];
-          b = ks[1];
-        } else {
-          const float2 cs = rope_cs(p, tt, pair, kc);
-          a = ks[0] * cs.x - ks[1] * cs.y;
-          b = ks[0] * cs.y + ks[1] * cs.x;
-        }
+        a = ks[0];
+        b = ks[1];
         va = vs[0];
         vb = vs[1];
       }

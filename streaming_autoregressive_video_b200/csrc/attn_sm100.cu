@@ -7,8 +7,11 @@
 // Memory for Infinite Rollouts) and all tokens of the block itself, which
 // attend to each other bidirectionally ("Cosmos3-H-Dreams" model card, Model
 // Architecture: block-causal student with a KV cache; AlpaDreams GTC 2026
-// write-up, section VII).  q' and k' carry 3D (t,h,w) RoPE, applied here as
-// Q and K tiles land in shared memory; the cache holds pre-RoPE keys.
+// write-up, section VII).  q' and k' carry 3D (t,h,w) RoPE: each query tile
+// is rotated as it lands in shared memory; keys arrive rotated (cache keys
+// were rotated once when their frame was committed, the block's keys once per
+// call by a pass over the block before this kernel), because every query
+// tile of a head reads the same keys.
 //
 // Design (one CTA = two 128-row query tiles of one (rollout, head)):
 //   warp 0        TMA producer: Q tiles once, then K and V tiles through
@@ -21,9 +24,9 @@
 //                 two query tiles ping-pong so one tile's softmax overlaps the
 //                 other tile's matrix products.
 //   warp 2        TMEM allocator (512 columns: S0, S1, O0, O1).
-//   warps 4-7     RoPE: rotate Q tiles once and every K tile in place in the
-//                 swizzled shared-memory layout, cos/sin from the cache's
-//                 tables (fp64-accurate angles rounded once to fp32).
+//   warps 4-7     RoPE: rotate the two Q tiles in place in the swizzled
+//                 shared-memory layout, cos/sin from the cache's tables
+//                 (fp64-accurate angles rounded once to fp32).
 //   warps 8-15    softmax, one thread per query row (TMEM lane): row max,
 //                 exp2, row sum, P rounded to bf16 and written back into the
 //                 S columns of TMEM as the A operand of the PV product; the
@@ -72,7 +75,7 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct Shared {
   uint64_t q_full, q_ready;
-  uint64_t k_full[kKStages], k_ready[kKStages], k_empty[kKStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, drain;
@@ -89,11 +92,15 @@ constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
 // Site codes for the device error word.
 enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4 };
 
+// Bounded wait.  kSpin (MMA issuer, softmax: the critical path) polls, so
+// the waiter resumes as soon as the phase completes; the other roles sleep
+// between polls and leave issue slots to the working warps.
+template <bool kSpin = false>
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
                                          Shared* sh, int32_t* err, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_sleep(bar, parity)) {
+  while (!(kSpin ? mbar_try_wait(bar, parity) : mbar_try_wait_sleep(bar, parity))) {
     if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
@@ -206,27 +213,6 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
   }
 }
 
-// Rotate the valid keys of one K tile of the block (keys key0..key0+127);
-// block frame f sits at t-row slots + f of the table (t = n + f).
-__device__ __forceinline__ void rope_k_tile(uint8_t* tile, int key0, int nseg,
-                                            const RopeLane& rl,
-                                            const float2* tab,
-                                            const AttnParams& p) {
-#pragma unroll 4
-  for (int m = 0; m < 16; ++m) {
-    const int row = rl.row0 + 8 * m;
-    const int key = key0 + row;
-    if (key >= nseg) continue;
-    const int fi = (int)fast_div((uint32_t)key, p.div_Tf);
-    const int tok = key - fi * p.Tf;
-    int hh = 0, ww = 0;
-    if (tok < p.T) {
-      hh = (int)fast_div((uint32_t)tok, p.div_gw);
-      ww = tok - hh * p.gw;
-    }
-    rotate_chunk(tile, row, rl, tab, p.slots + fi, hh, ww);
-  }
-}
 
 // End of every role branch: all 512 threads meet on named barrier 1 (each
 // warp arrives from its own branch), then warp 2 releases the TMEM columns.
@@ -264,7 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sh->q_ready, 128);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sh->k_full[s], 1);
-      mbar_init(&sh->k_ready[s], 128);
       mbar_init(&sh->k_empty[s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
@@ -316,9 +301,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < tc.nt; ++j) {
         const bool seg1 = j < tc.nt1;
         const int key0 = seg1 ? j * kBN : (j - tc.nt1) * kBN;
+        // keys: rotated cache keys or the block keys rotated for this call,
+        // both batched by (layer, rollout); values: cache (layer, rollout)
+        // or the caller's block values (rollout)
         const CUtensorMap* mk = seg1 ? &tm_kc : &tm_kb;
         const CUtensorMap* mv = seg1 ? &tm_vc : &tm_vb;
-        const int c3 = seg1 ? p.map_row0 + r : r;
+        const int ck3 = p.map_row0 + r;
+        const int cv3 = seg1 ? p.map_row0 + r : r;
         const int ks = j % kKStages;
         if (j >= kKStages &&
             !wait_bar(&sh->k_empty[ks], ((j / kKStages) - 1) & 1, sh, p.err,
@@ -327,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
         for (int hf = 0; hf < 2; ++hf)
           tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
-                      &sh->k_full[ks], hf * 64, h, key0, c3);
+                      &sh->k_full[ks], hf * 64, h, key0, ck3);
         issued_k = j + 1;
         const int vs = j % kVStages;
         if (j >= kVStages &&
@@ -337,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
         for (int hf = 0; hf < 2; ++hf)
           tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
-                      &sh->v_full[vs], hf * 64, h, key0, c3);
+                      &sh->v_full[vs], hf * 64, h, key0, cv3);
         issued_v = j + 1;
       }
       if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) {
@@ -374,15 +363,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
-      // K tile j is ready once the RoPE warpgroup has passed it: it steps
-      // through every tile in order (rotating only the block's own tiles;
-      // cache tiles hold keys rotated at commit), so the phases of k_full and
-      // k_ready advance together and no waiter can fall two phases behind.
+      // K tiles arrive rotated (cache keys at commit, block keys once per
+      // call), so a K tile is ready as soon as its copy has landed.
       auto wait_k = [&](int j) -> bool {
-        return wait_bar(&sh->k_ready[j % kKStages], (j / kKStages) & 1, sh,
-                        p.err, kSiteMma);
+        return wait_bar<true>(&sh->k_full[j % kKStages], (j / kKStages) & 1, sh,
+                              p.err, kSiteMma);
       };
-      bool ok = wait_bar(&sh->q_ready, 0, sh, p.err, kSiteMma) && wait_k(0);
+      bool ok = wait_bar<true>(&sh->q_ready, 0, sh, p.err, kSiteMma) && wait_k(0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -392,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&sh->k_empty[0]);
         for (int j = 0; j < tc.nt && ok; ++j) {
           const int vs = j % kVStages;
-          ok = wait_bar(&sh->v_full[vs], (j / kVStages) & 1, sh, p.err, kSiteMma) &&
-               wait_bar(&sh->p_full[0], j & 1, sh, p.err, kSiteMma);
+          ok = wait_bar<true>(&sh->v_full[vs], (j / kVStages) & 1, sh, p.err, kSiteMma) &&
+               wait_bar<true>(&sh->p_full[0], j & 1, sh, p.err, kSiteMma);
           if (!ok) break;
           tc_fence_after();
           issue_pv(0, vs, j > 0);
@@ -406,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s(0, ks);
             mma_commit(&sh->s_full[0]);
           }
-          ok = wait_bar(&sh->p_full[1], j & 1, sh, p.err, kSiteMma);
+          ok = wait_bar<true>(&sh->p_full[1], j & 1, sh, p.err, kSiteMma);
           if (!ok) break;
           tc_fence_after();
           issue_pv(1, vs, j > 0);
@@ -449,19 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
     }
     mbar_arrive(&sh->q_ready);
-    // Every K tile passes through here in order; only the block's own tiles
-    // need rotating (cache tiles come from the rotated-key region).
-    for (int j = 0; j < tc.nt && ok; ++j) {
-      const int ks = j % kKStages;
-      ok = __all_sync(0xffffffffu, wait_bar(&sh->k_full[ks], (j / kKStages) & 1,
-                                            sh, p.err, kSiteRope));
-      if (!ok) break;
-      if (j >= tc.nt1) {
-        rope_k_tile(smem + kOffK + ks * kTile, (j - tc.nt1) * kBN, tc.n2, rl, st, p);
-        fence_proxy_async_smem();
-      }
-      mbar_arrive(&sh->k_ready[ks]);
-    }
     teardown(warp, tmem);
     return;
   } else {
@@ -479,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t sa[64], sb[64];
     for (int j = 0; j < tc.nt; ++j) {
       ok = __all_sync(0xffffffffu,
-                      wait_bar(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
+                      wait_bar<true>(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
       tmem_ld64(tS, sa);

@@ -226,29 +226,49 @@ __global__ void reset_meta_kernel(CacheView c, ResetParams p) {
   fill_ttab(c, l, r, 0, pos);
 }
 
-// Rotate one 16-byte chunk of a [R][F][Tx][H][d] tensor in place.
+// 3D RoPE of a block tensor [R][F][Tx][H][d]: token row i of rollout r and
+// frame f sits at t = n_r + f (t-row slots + f of the rollout's table).  One
+// warp per token row; out may equal in (in place).
 template <typename Elem>
-__global__ void rope3d_kernel(CacheView c, int layer, int n_rollouts,
-                              Elem* x, int Tx, uint64_t nchunks) {
-  constexpr int kPer = 16 / sizeof(Elem);  // elements per chunk (4 or 8)
-  const int cpr = c.d / kPer;              // chunks per head row
-  for (uint64_t ci = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
-       ci < nchunks; ci += (uint64_t)gridDim.x * blockDim.x) {
-    const int cc = (int)(ci % cpr);
-    uint64_t rest = ci / cpr;
-    rest /= c.H;                       // head index does not matter
-    const int tok = (int)(rest % Tx);
-    rest /= Tx;
-    const int f = (int)(rest % c.F);
-    const int r = (int)(rest / c.F);
+__global__ void __launch_bounds__(256)
+    rope3d_kernel(CacheView c, int layer, int n_rollouts, const Elem* in,
+                  Elem* out, int Tx) {
+  constexpr int kPer = 16 / sizeof(Elem);  // elements per 16-byte chunk
+  const uint32_t cpr = c.d / kPer;         // chunks per head row
+  const uint32_t row_chunks = cpr * c.H;   // chunks per token row
+  const uint32_t rows = (uint32_t)n_rollouts * c.F * Tx;
+  const uint32_t warps = gridDim.x * (blockDim.x >> 5);
+  const int lane = threadIdx.x & 31;
+  for (uint32_t row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row < rows; row += warps) {
+    const uint32_t r = row / (c.F * Tx);
+    const uint32_t rem = row - r * (c.F * Tx);
+    const int f = (int)(rem / Tx);
+    const int tok = (int)(rem - f * Tx);
     const float2* tt = c.ttab + (((size_t)layer * c.R + r) * (c.slots + c.F) +
                                  c.slots + f) * c.pt;
     const int hh = tok < c.T ? tok / c.gw : 0;
-    const int ww = tok < c.T ? tok % c.gw : 0;
-    Elem* px = x + ci * kPer;
-    const uint4 u = *reinterpret_cast<const uint4*>(px);
-    *reinterpret_cast<uint4*>(px) = rotate16<Elem>(u, cc * (kPer / 2), c, tt, hh, ww);
+    const int ww = tok < c.T ? tok - hh * c.gw : 0;
+    const uint4* src = reinterpret_cast<const uint4*>(in) + (size_t)row * row_chunks;
+    uint4* dst = reinterpret_cast<uint4*>(out) + (size_t)row * row_chunks;
+    for (uint32_t ci = lane; ci < row_chunks; ci += 32) {
+      const int pair0 = (int)(ci % cpr) * (kPer / 2);
+      dst[ci] = rotate16<Elem>(src[ci], pair0, c, tt, hh, ww);
+    }
   }
+}
+
+template <typename Elem>
+cudaError_t launch_rope_rows(const CacheView& c, int layer, int n_rollouts,
+                             const void* in, void* out, int Tx, cudaStream_t s) {
+  const uint64_t rows = (uint64_t)n_rollouts * c.F * Tx;
+  const uint64_t blocks_needed = (rows + 7) / 8;  // 8 warps per block
+  const unsigned blocks = (unsigned)(blocks_needed < 148ull * 8 ? blocks_needed : 148ull * 8);
+  rope3d_kernel<Elem><<<blocks, 256, 0, s>>>(c, layer, n_rollouts,
+                                             static_cast<const Elem*>(in),
+                                             static_cast<Elem*>(out), Tx);
+  count_launch(1);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -292,19 +312,17 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
 
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
                           void* x, int Tx, cudaStream_t s) {
-  const uint64_t elems = (uint64_t)n_rollouts * c.F * Tx * c.H * c.d;
-  const uint64_t nchunks = elems * c.esz / 16;
-  const unsigned blocks = (unsigned)((nchunks + 255) / 256 < 148ull * 16
-                                         ? (nchunks + 255) / 256
-                                         : 148ull * 16);
+  if (c.esz == 2) return launch_rope_rows<uint16_t>(c, layer, n_rollouts, x, x, Tx, s);
+  return launch_rope_rows<float>(c, layer, n_rollouts, x, x, Tx, s);
+}
+
+cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
+                                   int n_rollouts, const void* k,
+                                   cudaStream_t s) {
+  void* out = c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes;
   if (c.esz == 2)
-    rope3d_kernel<uint16_t><<<blocks, 256, 0, s>>>(
-        c, layer, n_rollouts, static_cast<uint16_t*>(x), Tx, nchunks);
-  else
-    rope3d_kernel<float><<<blocks, 256, 0, s>>>(
-        c, layer, n_rollouts, static_cast<float*>(x), Tx, nchunks);
-  count_launch(1);
-  return cudaGetLastError();
+    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, k, out, c.Tf, s);
+  return launch_rope_rows<float>(c, layer, n_rollouts, k, out, c.Tf, s);
 }
 
 }  // namespace fd

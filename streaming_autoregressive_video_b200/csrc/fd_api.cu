@@ -23,6 +23,7 @@ struct fd_cache {
   int device;
   std::vector<int64_t> host_n;  // [L][R] mirror of the device counters
   CUtensorMap tm_kc, tm_vc;     // bf16 caches: (d, H, slots*Tf, L*R)
+  CUtensorMap tm_kb;            // rotated block keys: (d, H, F*Tf, L*R)
   bool have_maps;
 };
 
@@ -83,6 +84,10 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   off = align_up(off + kv);
   lay->krot = off;
   off = align_up(off + kv);
+  lay->kblk = off;
+  size_t blk;
+  if (!mul_ok(frame * d->block_frames, lr, &blk)) return FD_ERR_CAPACITY;
+  off = align_up(off + blk);
   lay->pos = off;
   off = align_up(off + lr * slots * sizeof(int32_t));
   lay->count = off;
@@ -204,6 +209,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.k = base + lay.k;
   v.v = base + lay.v;
   v.krot = base + lay.krot;
+  v.kblk = base + lay.kblk;
   v.pos = reinterpret_cast<int32_t*>(base + lay.pos);
   v.count = reinterpret_cast<int32_t*>(base + lay.count);
   v.ttab = reinterpret_cast<float2*>(base + lay.ttab);
@@ -234,7 +240,9 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
     const uint64_t rows = (uint64_t)v.slots * v.Tf;
     const uint64_t batch = (uint64_t)v.L * v.R;
     if (!fd::encode_bf16_map(&c->tm_kc, v.krot, v.d, v.H, rows, batch) ||
-        !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.H, rows, batch)) {
+        !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.H, rows, batch) ||
+        !fd::encode_bf16_map(&c->tm_kb, v.kblk, v.d, v.H, (uint64_t)v.F * v.Tf,
+                             batch)) {
       // only the tensor-core path needs the maps; keep going without them
       c->have_maps = false;
     } else {
@@ -338,7 +346,8 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   fd::AttnParams p;
   memset(&p, 0, sizeof(p));
   p.q = q;
-  p.k = k;
+  // the block's keys, rotated once for all query tiles (see fd.h, kblk)
+  p.k = c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes;
   p.v = v_;
   p.pos = c.pos + (size_t)layer * c.R * c.slots;
   p.count = c.count + (size_t)layer * c.R;
@@ -375,17 +384,19 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
 
   if (cache->desc.dtype == FD_F32) {
     if (c.d % 32 != 0 || c.d > 128) return FD_ERR_UNSUPPORTED;
-    return fd::cuda_status(fd::launch_attn_f32(p, s));
+  } else if (c.d != 128 || !cache->have_maps) {
+    return FD_ERR_UNSUPPORTED;
   }
-  if (c.d != 128 || !cache->have_maps) return FD_ERR_UNSUPPORTED;
-  CUtensorMap tm_q, tm_kb, tm_vb;
+  st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, s));
+  if (st != FD_OK) return st;
+  if (cache->desc.dtype == FD_F32) return fd::cuda_status(fd::launch_attn_f32(p, s));
+  CUtensorMap tm_q, tm_vb;
   const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
   if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
-      !fd::encode_bf16_map(&tm_kb, k, c.d, c.H, kb_rows, n_rollouts) ||
       !fd::encode_bf16_map(&tm_vb, v_, c.d, c.H, kb_rows, n_rollouts))
     return FD_ERR_CUDA;
   return fd::cuda_status(fd::launch_attn_bf16_sm100(
-      tm_q, cache->tm_kc, cache->tm_vc, tm_kb, tm_vb, p, s));
+      tm_q, cache->tm_kc, cache->tm_vc, cache->tm_kb, tm_vb, p, s));
 }
 
 fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,

@@ -35,6 +35,7 @@ struct CacheView {
   uint8_t* k;
   uint8_t* v;
   uint8_t* krot;  // committed keys rotated to their frame's position
+  uint8_t* kblk;  // per-layer work area: the block's keys rotated per call
   int32_t* pos;
   int32_t* count;
   float2* ttab;
@@ -96,6 +97,10 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
                          cudaStream_t s);
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
                           void* x, int tokens_per_frame, cudaStream_t s);
+// block keys k [n_rollouts][F*Tf][H][d] rotated into the layer's kblk region
+cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
+                                   int n_rollouts, const void* k,
+                                   cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kc,
