@@ -202,6 +202,14 @@ fd_status fd_cache_frames(const fd_cache* cache, int32_t layer,
  * *code != 0. */
 fd_status fd_get_device_error(fd_cache* cache, int32_t* code);
 
+/* Verification hook for the base-2 exponential of the bf16 softmax, which
+ * computes part of its weights on the FMA pipe (Cody-Waite reduction and a
+ * cubic, see the attention kernel) and the rest on the hardware unit.  For
+ * each x[i] (device, n floats, each in [-126, 8]) writes (device, 3n floats)
+ * y[3i] = the FMA-pipe value, y[3i+1] = the hardware approximation,
+ * y[3i+2] = CUDA's exp2f(x[i]).  Asynchronous on `stream`. */
+fd_status fd_exp2_selfcheck(const float* x, float* y, int64_t n, void* stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t fd_launch_count(void);
 

@@ -24,7 +24,7 @@ EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
            "fd_cache_destroy", "fd_cache_get_desc", "fd_cache_layout_of",
            "fd_cache_reset", "fd_rope3d", "fd_block_attention",
            "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
-           "fd_launch_count", "fd_status_string"]
+           "fd_exp2_selfcheck", "fd_launch_count", "fd_status_string"]
 
 
 class FdError(RuntimeError):
@@ -83,6 +83,7 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
                                     ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
     lib.fd_cache_frames.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int64)]
     lib.fd_get_device_error.argtypes = [vp, ctypes.POINTER(i32)]
+    lib.fd_exp2_selfcheck.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.fd_launch_count.argtypes = []
     lib.fd_launch_count.restype = ctypes.c_uint64
     lib.fd_status_string.argtypes = [i32]
@@ -209,6 +210,11 @@ def fd_cache_frames(cache: Cache, layer: int, rollout: int) -> int:
     _check(load().fd_cache_frames(cache.handle, layer, rollout, ctypes.byref(n)),
            "fd_cache_frames")
     return n.value
+
+
+def fd_exp2_selfcheck(x, y, stream=None) -> None:
+    _check(load().fd_exp2_selfcheck(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "fd_exp2_selfcheck")
 
 
 def fd_get_device_error(cache: Cache) -> int:

@@ -27,9 +27,11 @@
 //   warps 4-7     RoPE: rotate the two Q tiles in place in the swizzled
 //                 shared-memory layout, cos/sin from the cache's tables
 //                 (fp64-accurate angles rounded once to fp32).
-//   warps 8-15    softmax, one thread per query row (TMEM lane): row max,
-//                 exp2, row sum, P rounded to bf16 and written back into the
-//                 S columns of TMEM as the A operand of the PV product; the
+//   warps 8-15    softmax on one tile at a time, two threads per query row
+//                 (TMEM lane), 64 columns each: row max (halves exchanged
+//                 through shared memory), exp2, row sum, P rounded to bf16
+//                 and written back into the S columns of TMEM as the A
+//                 operand of the PV product; the
 //                 O rescale is skipped unless the running max grows by more
 //                 than 2^8, which keeps P <= 256 and the result exact up to
 //                 rounding.  The epilogue divides by the row sum and writes
@@ -64,6 +66,7 @@ constexpr uint32_t kOffK = 2 * kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
 constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
+constexpr int kPolyEvery = 2;  // every 2nd pair of exponentials on the FMA pipe
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
 
@@ -78,13 +81,15 @@ struct Shared {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
+  uint64_t red_bar[2][4];  // per tile and lane quarter: row halves exchange
   uint64_t o_full, drain;
   uint32_t tmem_base;
   int32_t abort;
 };
 
 // RoPE tables follow the barriers; the dynamic size adds them per launch.
-constexpr uint32_t kOffTab = kOffShared + 256;
+constexpr uint32_t kOffRed = kOffShared + 256;   // [2][2][128] floats
+constexpr uint32_t kOffTab = kOffRed + 2 * 2 * 128 * 4;
 static_assert(sizeof(Shared) <= 256, "barrier block");
 constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
 constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
@@ -258,7 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sh->s_full[x], 1);
-      mbar_init(&sh->p_full[x], 128);
+      mbar_init(&sh->p_full[x], 256);
+      for (int q = 0; q < 4; ++q) mbar_init(&sh->red_bar[x][q], 64);
     }
     mbar_init(&sh->o_full, 1);
     mbar_init(&sh->drain, 1);
@@ -441,111 +447,156 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<176>();
     // ------------------------------------------------------------ softmax
-    const int x = (warp - 8) >> 2;
-    const int wq = warp & 3;
+    // All eight softmax warps work on one query tile at a time, alternating
+    // between the two tiles so that one tile's softmax overlaps the other
+    // tile's matrix products.  Warps 8+q and 12+q share TMEM lanes 32q..32q+31
+    // (query rows): warp 8+q takes S columns 0-63 of each row and warp 12+q
+    // columns 64-127.  The halves of a row exchange partial maxima (and, at
+    // the end, partial sums) through shared memory, synchronised by a bounded
+    // mbarrier of the 64 threads that own those rows.
+    const int hc = (warp - 8) >> 2;    // column half
+    const int wq = warp & 3;           // lane quarter
+    const int row_t = wq * 32 + lane;  // row within a tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
-    const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [tile][half][row]
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     bool ok = true;
-    uint32_t rr[32];
-    uint32_t sa[64], sb[64];
-    for (int j = 0; j < tc.nt; ++j) {
-      ok = __all_sync(0xffffffffu,
-                      wait_bar<true>(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
-      if (!ok) break;
-      tc_fence_after();
-      tmem_ld64(tS, sa);
-      tmem_ld64(tS + 64, sb);
+    uint32_t s[64];
+    // exchange a per-row value with the other column half; bounded wait
+    auto exchange = [&](int x, float mine, uint32_t parity) -> float {
+      red[(x * 2 + hc) * kBM + row_t] = mine;
+      mbar_arrive(&sh->red_bar[x][wq]);
+      ok = __all_sync(0xffffffffu, ok && wait_bar<true>(&sh->red_bar[x][wq], parity, sh,
+                                                        p.err, kSiteSoftmax));
+      return red[(x * 2 + (1 - hc)) * kBM + row_t];
+    };
+    for (int j = 0; j < tc.nt && ok; ++j) {
       const int valid = j < tc.nt1 ? min(kBN, tc.n1 - j * kBN)
                                    : min(kBN, tc.n2 - (j - tc.nt1) * kBN);
-      if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          if (i >= valid) sa[i] = 0xFF800000u;
-          if (64 + i >= valid) sb[i] = 0xFF800000u;
+      for (int x = 0; x < 2; ++x) {
+        if (!ok) break;
+        const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
+        const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+        ok = __all_sync(0xffffffffu,
+                        wait_bar<true>(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld64(tS + hc * 64, s);
+        if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (hc * 64 + i >= valid) s[i] = 0xFF800000u;
         }
-      }
-      float m8[8];
+        float m8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        m8[i] = fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i]));
+        for (int i = 0; i < 8; ++i)
+          m8[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 8]));
 #pragma unroll
-      for (int i = 8; i < 64; ++i)
-        m8[i & 7] = fmaxf(m8[i & 7], fmaxf(__uint_as_float(sa[i]), __uint_as_float(sb[i])));
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      const float m_tile = mx * sl2;
-      const bool need = m_tile > m + kRescaleThreshold;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2_approx(m - m_tile) : 1.f;
+        for (int i = 16; i < 64; i += 2)
+          m8[(i >> 1) & 7] = fmaxf(m8[(i >> 1) & 7],
+                                   fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 1])));
+        const float pmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        // both halves of the row have loaded their S columns once this
+        // returns, so P may now overwrite them
+        const float omax = exchange(x, pmax, j & 1);
+        if (!ok) break;
+        const float m_tile = fmaxf(pmax, omax) * sl2;
+        const bool need = m_tile > m[x] + kRescaleThreshold;
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m[x] - m_tile) : 1.f;
 #pragma unroll 1
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t r16[16];
-          tmem_ld16(tO + c8 * 16, r16);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tO + hc * 64 + c * 16, r16);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
-          tmem_st16(tO + c8 * 16, r16);
+            for (int i = 0; i < 16; ++i)
+              r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+            tmem_st16(tO + hc * 64 + c * 16, r16);
+          }
+          tmem_wait_st();
+        }
+        if (need) {
+          l[x] = (j > 0) ? l[x] * ex2_approx(m[x] - m_tile) : 0.f;
+          m[x] = m_tile;
+        }
+        // P = 2^(s * log2(e)/sqrt(d) - m), two columns per packed
+        // instruction.  In full tiles every kPolyEvery-th pair of
+        // exponentials runs on the FMA pipe (exp2_poly2) to share the load of
+        // the MUFU unit; partial tiles (masked columns at -inf) use MUFU
+        // throughout so masked weights are exactly 0.
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m[x], -m[x]);
+        float ls = 0.f;
+        uint64_t ls2 = 0;  // two packed +0.0f
+        uint32_t pk[32];
+        auto exps = [&](bool full) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint64_t x2 = f2_fma(
+                f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
+            float p0, p1;
+            if (full && (i % kPolyEvery) == kPolyEvery - 1) {
+              const uint64_t e2 = exp2_poly2(x2);
+              ls2 = f2_add(ls2, e2);
+              f2_unpack(e2, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+              ls += p0 + p1;
+            }
+            pk[i] = pack_bf16(p0, p1);
+          }
+        };
+        if (valid == kBN) exps(true); else exps(false);
+        // bf16 P of columns hc*64.. goes to TMEM columns hc*32.. of the tile
+        tmem_st32(tS + hc * 32, pk);
+        {
+          float la, lb;
+          f2_unpack(ls2, la, lb);
+          l[x] += ls + (la + lb);
         }
         tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh->p_full[x]);
       }
-      if (need) {
-        l = (j > 0) ? l * ex2_approx(m - m_tile) : 0.f;
-        m = m_tile;
-      }
-      const float neg_m = -m;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sa[2 * i]), sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sa[2 * i + 1]), sl2, neg_m));
-        ls[i & 3] += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
-      }
-      tmem_st32(tS, pk);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sb[2 * i]), sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sb[2 * i + 1]), sl2, neg_m));
-        ls[i & 3] += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
-      }
-      tmem_st32(tS + 32, pk);
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sh->p_full[x]);
     }
     if (ok)
       ok = __all_sync(0xffffffffu,
                       wait_bar(&sh->o_full, 0, sh, p.err, kSiteSoftmax));
-    if (ok) {
-      tc_fence_after();
-      const int row = qrow0 + x * kBM + wq * 32 + lane;
-      const float inv_l = 1.f / l;
-      uint16_t* out = static_cast<uint16_t*>(p.out) +
-                      (((size_t)r * p.Mq + row) * p.H + h) * kD;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        tmem_ld32(tO + c4 * 32, rr);
+    for (int x = 0; x < 2; ++x) {
+      if (!ok) break;
+      const float l_tot = l[x] + exchange(x, l[x], tc.nt & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+      const int row = qrow0 + x * kBM + row_t;
+      const float inv_l = 1.f / l_tot;
+      uint16_t* out = static_cast<uint16_t*>(p.out) +
+                      (((size_t)r * p.Mq + row) * p.H + h) * kD + hc * 64;
+      uint32_t rr[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(tO + hc * 64 + c * 32, rr);
         if (row < p.Mq) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l,
                               __uint_as_float(rr[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(out + c4 * 32);
+          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
       }
-      if (p.lse != nullptr && row < p.Mq)
+      if (p.lse != nullptr && hc == 0 && row < p.Mq)
         p.lse[((size_t)r * p.H + h) * p.Mq + row] =
-            (m + log2f(l)) * 0.69314718055994530942f;
+            (m[x] + log2f(l_tot)) * 0.69314718055994530942f;
     }
     teardown(warp, tmem);
     return;
@@ -582,6 +633,34 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
   dim3 grid((p.Mq + 2 * kBM - 1) / (2 * kBM), p.H, p.n_rollouts);
   attn_bf16_d128_sm100<<<grid, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc,
                                                           tm_kb, tm_vb, p);
+  count_launch(1);
+  return cudaGetLastError();
+}
+
+}  // namespace fd
+
+namespace fd {
+namespace {
+
+__global__ void exp2_selfcheck_kernel(const float* x, float* y, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = x[i];
+    float a, b;
+    sm100::f2_unpack(sm100::exp2_poly2(sm100::f2_pack(v, v)), a, b);
+    y[3 * i] = a;
+    y[3 * i + 1] = sm100::ex2_approx(v);
+    y[3 * i + 2] = exp2f(v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_exp2_selfcheck(const float* x, float* y, int64_t n,
+                                  cudaStream_t s) {
+  const int64_t blocks = (n + 255) / 256;
+  exp2_selfcheck_kernel<<<(unsigned)(blocks < 1184 ? (blocks > 0 ? blocks : 1) : 1184),
+                          256, 0, s>>>(x, y, n);
   count_launch(1);
   return cudaGetLastError();
 }

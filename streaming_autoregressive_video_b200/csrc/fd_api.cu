@@ -466,3 +466,11 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code) {
 }
 
 }  // extern "C"
+
+extern "C" fd_status fd_exp2_selfcheck(const float* x, float* y, int64_t n,
+                                       void* stream) {
+  if (x == nullptr || y == nullptr || n < 0) return FD_ERR_INVALID_ARG;
+  if (n == 0) return FD_OK;
+  return fd::cuda_status(
+      fd::launch_exp2_selfcheck(x, y, n, static_cast<cudaStream_t>(stream)));
+}

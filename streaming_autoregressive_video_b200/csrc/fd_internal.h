@@ -112,3 +112,8 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
 void count_launch(int n);
 
 }  // namespace fd
+
+namespace fd {
+cudaError_t launch_exp2_selfcheck(const float* x, float* y, int64_t n,
+                                  cudaStream_t s);
+}  // namespace fd

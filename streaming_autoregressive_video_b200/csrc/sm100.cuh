@@ -294,6 +294,71 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x on the FMA/ALU pipes for a pair of x <= 8, written from:
+//  * Cody-Waite style argument reduction (W. J. Cody and W. Waite, "Software
+//    Manual for the Elementary Functions", 1980): x = j + f with j = rint(x)
+//    taken from the low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2];
+//  * 2^f by a cubic fitted here to 2^f on [-1/2, 1/2] (iteratively reweighted
+//    least squares on relative error over Chebyshev nodes, coefficients
+//    rounded to fp32; max relative error 7.5e-5, below the 2^-9 spacing of
+//    the bf16 weights it feeds);
+//  * 2^j applied by adding j to the exponent field.
+// Inputs are clamped to -126, so weights below 2^-126 come out as tiny
+// non-negative numbers instead of 0; callers use it only where every score
+// is finite.  The same split, software exp2 on the FMA units alongside the
+// MUFU unit, is how FlashAttention-4 relieves the exponential unit on
+// Blackwell.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.05517164617776871f;
+constexpr float kExp2Shift = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  x2 = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const uint64_t sh2 = f2_pack(kExp2Shift, kExp2Shift);
+  const uint64_t t2 = f2_add(x2, sh2);           // low bits hold rint(x)
+  const uint64_t fr = f2_sub(x2, f2_sub(t2, sh2));  // x - rint(x), both exact
+  uint64_t p2 = f2_fma(f2_pack(kExp2C3, kExp2C3), fr, f2_pack(kExp2C2, kExp2C2));
+  p2 = f2_fma(p2, fr, f2_pack(kExp2C1, kExp2C1));
+  p2 = f2_fma(p2, fr, f2_pack(kExp2C0, kExp2C0));
+  float pa, pb, ta, tb;
+  f2_unpack(p2, pa, pb);
+  f2_unpack(t2, ta, tb);
+  // bits(t) << 23 == rint(x) << 23 (mod 2^32): the shift constant's own bits
+  // vanish above bit 31
+  const uint32_t ra = __float_as_uint(pa) + (__float_as_uint(ta) << 23);
+  const uint32_t rb = __float_as_uint(pb) + (__float_as_uint(tb) << 23);
+  return f2_pack(__uint_as_float(ra), __uint_as_float(rb));
+}
+
 // Per-warpgroup register reallocation.  Every warpgroup of the block must
 // take part so the block's total never exceeds its launch allocation.
 template <uint32_t N>

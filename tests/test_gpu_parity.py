@@ -130,3 +130,21 @@ def test_attention_bf16_ragged_rollouts():
     ls.attention(0, q, k, v, what="ragged")
     # fewer active rollouts than the cache holds
     ls.attention(0, q[:2], k[:2], v[:2], n_rollouts=2, what="ragged n=2")
+
+
+def test_softmax_exp2_against_exp2f():
+    """The FMA-pipe exponential used for part of the softmax weights agrees
+    with CUDA's exp2f (and the exact 2^x) to the fitted polynomial's bound."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1 << 20),
+                   torch.rand(1 << 18, generator=g) * 134.0 - 126.0]).float()
+    y = torch.empty(3 * x.numel(), dtype=torch.float32, device="cuda")
+    xd = x.cuda()
+    fd.fd_exp2_selfcheck(xd, y)
+    torch.cuda.synchronize()
+    poly, hw, ref = y.view(-1, 3).cpu().double().T
+    exact = torch.exp2(x.double())
+    # the cubic's own bound is 7.5e-5; fp32 evaluation adds a few ulp
+    assert float(((poly - ref).abs() / ref).max()) <= 2.0e-4
+    assert float(((poly - exact).abs() / exact).max()) <= 2.0e-4
+    assert float(((hw - exact).abs() / exact).max()) <= 1.0e-5
