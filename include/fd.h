@@ -177,6 +177,29 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
                              const void* v, void* out, float* lse,
                              void* stream);
 
+/* Allocation-free variant of fd_block_attention.  The pages have no
+ * counterpart: it is an interface for callers that cannot set device memory
+ * aside for the per-layer work area inside the cache storage -- storage
+ * carved from a pool or arena someone else sizes, or a process that may not
+ * call cudaMalloc at all (it can synchronise the device, which a real-time
+ * serving loop cannot afford).  Same arguments, semantics and results as
+ * fd_block_attention; the work area for the block's rotated keys is instead a
+ * static device array of FD_STATIC_WORK_BYTES inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *   - FD_ERR_CAPACITY (before any launch) when n_rollouts*F*Tf*H*d*element
+ *     size exceeds FD_STATIC_WORK_BYTES;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress), so make that first call before any stream
+ *     capture on that device;
+ *   - every call shares the one array: calls that overlap on the GPU race
+ *     and must be ordered (one stream, or events);
+ *   - allocates nothing, neither on the device nor through any library. */
+#define FD_STATIC_WORK_BYTES (32u << 20)
+fd_status fd_block_attention_static(fd_cache* cache, int32_t layer,
+                                    int32_t n_rollouts, const void* q,
+                                    const void* k, const void* v, void* out,
+                                    float* lse, void* stream);
+
 /* Ring-buffer commit for layers [layer_begin, layer_end) -- the finalize()
  * half of [FD-HP]:  for every rollout r < n_rollouts and f < frames_r,
  * slot = slot_of(n_r + f) receives frame f of k[l]/v[l] bit for bit (and its

@@ -23,6 +23,7 @@ STATUS = {0: "FD_OK", 1: "FD_ERR_INVALID_ARG", 2: "FD_ERR_SHAPE", 3: "FD_ERR_DTY
 EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
            "fd_cache_destroy", "fd_cache_get_desc", "fd_cache_layout_of",
            "fd_cache_reset", "fd_rope3d", "fd_block_attention",
+           "fd_block_attention_static",
            "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
            "fd_exp2_selfcheck", "fd_launch_count", "fd_status_string"]
 
@@ -79,6 +80,7 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
     lib.fd_cache_reset.argtypes = [vp, ctypes.POINTER(i32), i32, vp]
     lib.fd_rope3d.argtypes = [vp, i32, i32, vp, i32, vp]
     lib.fd_block_attention.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, vp]
+    lib.fd_block_attention_static.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.fd_cache_commit.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32),
                                     ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
     lib.fd_cache_frames.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int64)]
@@ -192,6 +194,19 @@ def fd_block_attention(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,
     _check(load().fd_block_attention(cache.handle, layer, n_rollouts, _ptr(q), _ptr(k),
                                      _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
            "fd_block_attention")
+
+
+# FD_STATIC_WORK_BYTES of include/fd.h
+STATIC_WORK_BYTES = 32 << 20
+
+
+def fd_block_attention_static(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,
+                              lse=None, stream=None) -> None:
+    """fd_block_attention with its work area in the library's static array."""
+    _check(load().fd_block_attention_static(cache.handle, layer, n_rollouts, _ptr(q),
+                                            _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                            _stream(stream)),
+           "fd_block_attention_static")
 
 
 def fd_cache_commit(cache: Cache, layer_begin: int, layer_end: int, n_rollouts: int,

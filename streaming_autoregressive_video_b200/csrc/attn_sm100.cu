@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // or the caller's block values (rollout)
         const CUtensorMap* mk = seg1 ? &tm_kc : &tm_kb;
         const CUtensorMap* mv = seg1 ? &tm_vc : &tm_vb;
-        const int ck3 = p.map_row0 + r;
+        const int ck3 = seg1 ? p.map_row0 + r : p.kb_row0 + r;
         const int cv3 = seg1 ? p.map_row0 + r : r;
         const int ks = j % kKStages;
         if (j >= kKStages &&

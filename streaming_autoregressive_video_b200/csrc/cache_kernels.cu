@@ -317,9 +317,8 @@ cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
 }
 
 cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
-                                   int n_rollouts, const void* k,
+                                   int n_rollouts, const void* k, void* out,
                                    cudaStream_t s) {
-  void* out = c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes;
   if (c.esz == 2)
     return launch_rope_rows<uint16_t>(c, layer, n_rollouts, k, out, c.Tf, s);
   return launch_rope_rows<float>(c, layer, n_rollouts, k, out, c.Tf, s);

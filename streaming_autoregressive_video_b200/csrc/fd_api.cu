@@ -331,6 +331,20 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
                              int32_t n_rollouts, const void* q, const void* k,
                              const void* v_, void* out, float* lse,
                              void* stream) {
+  return fd::block_attention_impl(cache, layer, n_rollouts, q, k, v_, out, lse,
+                                  stream, nullptr);
+}
+
+}  // extern "C"
+
+size_t fd::block_work_bytes(const fd_cache* cache, int32_t n_rollouts) {
+  return (size_t)n_rollouts * cache->view.F * cache->view.frame_bytes;
+}
+
+fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
+                                   int32_t n_rollouts, const void* q,
+                                   const void* k, const void* v_, void* out,
+                                   float* lse, void* stream, void* work) {
   if (cache == nullptr || q == nullptr || k == nullptr || v_ == nullptr ||
       out == nullptr)
     return FD_ERR_INVALID_ARG;
@@ -346,8 +360,12 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   fd::AttnParams p;
   memset(&p, 0, sizeof(p));
   p.q = q;
-  // the block's keys, rotated once for all query tiles (see fd.h, kblk)
-  p.k = c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes;
+  // the block's keys, rotated once for all query tiles (see fd.h, kblk),
+  // in the layer's work area of the cache or in the caller's `work`
+  void* kblk = work != nullptr
+      ? work
+      : static_cast<void*>(c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes);
+  p.k = kblk;
   p.v = v_;
   p.pos = c.pos + (size_t)layer * c.R * c.slots;
   p.count = c.count + (size_t)layer * c.R;
@@ -375,6 +393,7 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   p.pw = c.pw;
   p.n_rollouts = n_rollouts;
   p.map_row0 = layer * c.R;
+  p.kb_row0 = work != nullptr ? 0 : layer * c.R;
   p.div_T = fd::make_fastdiv((uint32_t)c.T);
   p.div_Tf = fd::make_fastdiv((uint32_t)c.Tf);
   p.div_gw = fd::make_fastdiv((uint32_t)c.gw);
@@ -387,17 +406,23 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
   } else if (c.d != 128 || !cache->have_maps) {
     return FD_ERR_UNSUPPORTED;
   }
-  st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, s));
+  st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
   if (st != FD_OK) return st;
   if (cache->desc.dtype == FD_F32) return fd::cuda_status(fd::launch_attn_f32(p, s));
-  CUtensorMap tm_q, tm_vb;
+  CUtensorMap tm_q, tm_vb, tm_kb_work;
   const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
   if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
       !fd::encode_bf16_map(&tm_vb, v_, c.d, c.H, kb_rows, n_rollouts))
     return FD_ERR_CUDA;
+  if (work != nullptr &&
+      !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.H, kb_rows, n_rollouts))
+    return FD_ERR_CUDA;
   return fd::cuda_status(fd::launch_attn_bf16_sm100(
-      tm_q, cache->tm_kc, cache->tm_vc, cache->tm_kb, tm_vb, p, s));
+      tm_q, cache->tm_kc, cache->tm_vc, work != nullptr ? tm_kb_work : cache->tm_kb,
+      tm_vb, p, s));
 }
+
+extern "C" {
 
 fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,
                           int32_t layer_end, int32_t n_rollouts,

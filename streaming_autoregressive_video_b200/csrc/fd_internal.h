@@ -84,6 +84,7 @@ struct AttnParams {
   const uint8_t* vc;
   int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
   int map_row0;          // layer * R: row offset of this layer in the cache maps
+  int kb_row0;           // batch offset of rollout 0 in the rotated-block-key map
   FastDiv div_T, div_Tf, div_gw;
   float scale_log2;      // log2(e) / sqrt(d)
   float scale;           // 1 / sqrt(d)
@@ -97,9 +98,10 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
                          cudaStream_t s);
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
                           void* x, int tokens_per_frame, cudaStream_t s);
-// block keys k [n_rollouts][F*Tf][H][d] rotated into the layer's kblk region
+// block keys k [n_rollouts][F*Tf][H][d] rotated (positions from `layer`'s
+// counters) into out, same layout
 cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
-                                   int n_rollouts, const void* k,
+                                   int n_rollouts, const void* k, void* out,
                                    cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s);
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
@@ -110,6 +112,15 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const AttnParams& p, cudaStream_t s);
 
 void count_launch(int n);
+
+// Shared body of the attention entry points.  `work` is a device area for the
+// block's rotated keys ([n_rollouts][F*Tf][H][d], block_work_bytes bytes,
+// 16-byte aligned) or nullptr for the layer's work area in the cache storage.
+fd_status block_attention_impl(fd_cache* cache, int32_t layer,
+                               int32_t n_rollouts, const void* q,
+                               const void* k, const void* v, void* out,
+                               float* lse, void* stream, void* work);
+size_t block_work_bytes(const fd_cache* cache, int32_t n_rollouts);
 
 }  // namespace fd
 
