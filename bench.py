@@ -281,18 +281,23 @@ def run_fd(args, w, rank, world, local_rank):
     outs = [torch.empty(qshape, dtype=torch.int16, device=dev) for _ in range(L)]
     stream = torch.cuda.current_stream(dev)
 
-    def step(evs=None):
+    def timed(fn, evs):
+        if evs is None:
+            fn()
+            return
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+
+    def step(evs=None, cevs=None):
         for s in range(S):
             for l in range(L):
-                if evs is not None:
-                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a.record(stream)
-                fd.fd_block_attention(cache, l, R, q[s][l], k[s][l], v[s][l], outs[l],
-                                      stream=stream)
-                if evs is not None:
-                    b.record(stream)
-                    evs.append((a, b))
-        fd.fd_cache_commit(cache, 0, L, R, k[S - 1], v[S - 1], stream=stream)
+                timed(lambda: fd.fd_block_attention(cache, l, R, q[s][l], k[s][l], v[s][l],
+                                                    outs[l], stream=stream), evs)
+        timed(lambda: fd.fd_cache_commit(cache, 0, L, R, k[S - 1], v[S - 1], stream=stream),
+              cevs)
 
     def barrier():
         if world > 1:
@@ -309,11 +314,11 @@ def run_fd(args, w, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     launches0 = fd.fd_launch_count()
-    evs = []
+    evs, cevs = [], []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step(evs)
+        step(evs, cevs)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -321,10 +326,11 @@ def run_fd(args, w, rank, world, local_rank):
     launches = fd.fd_launch_count() - launches0
     ms_step = e0.elapsed_time(e1) / args.steps
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
-    t = torch.tensor([ms_step, attn_ms], dtype=torch.float64, device=dev)
+    commit_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
+    t = torch.tensor([ms_step, attn_ms, commit_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step, attn_ms = float(t[0]), float(t[1])
+    ms_step, attn_ms, commit_ms = float(t[0]), float(t[1]), float(t[2])
     err = fd.fd_get_device_error(cache)
     assert err == 0, f"device error word {err:#x}"
 
@@ -346,7 +352,16 @@ def run_fd(args, w, rank, world, local_rank):
             "frac": achieved / peak, "traffic": profile_traffic(),
             "kernel": "attn_bf16_d128_sm100", "peak_source": f"{src} bf16_tflops_sustained",
             "algorithmic_bytes_per_launch": bytes_call,
-            "flops_per_launch": flops_call, "launch_ms": attn_ms}
+            "flops_per_launch": flops_call, "launch_ms": attn_ms,
+            "launch_covers": "fd_block_attention call: block-key RoPE pass + attention kernel"}
+    # batched commit of all layers: read k, v; write K, V and rotated K
+    commit_bytes = 5.0 * L * R * F * Tf * H * d * 2
+    commit_roof = {"bound": "hbm", "achieved": commit_bytes / (commit_ms * 1e-3) / 1e9,
+                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                   "frac": commit_bytes / (commit_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                   "traffic": None, "kernel": "commit_copy_kernel + commit_meta_kernel",
+                   "peak_source": f"{src} hbm_gbs", "algorithmic_bytes_per_launch": commit_bytes,
+                   "launch_ms": commit_ms, "layers_per_launch": L}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
@@ -362,6 +377,7 @@ def run_fd(args, w, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "latent_frames_per_s_per_layer": frames_per_s_layer,
         "roofline": roof,
+        "commit_roofline": commit_roof,
         "gpu_launches": launches,
         "clocks": clocks,
         "e2e": e2e,

@@ -233,6 +233,16 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code);
  * y[3i+2] = CUDA's exp2f(x[i]).  Asynchronous on `stream`. */
 fd_status fd_exp2_selfcheck(const float* x, float* y, int64_t n, void* stream);
 
+/* Failure-detection self-test (no counterpart on the pages).  Runs one
+ * device-side wait on an mbarrier that nothing ever completes, through the
+ * same bounded wait the attention kernel uses, limited to limit_ms (1..2000)
+ * instead of the kernel's 2 s.  The wait gives up, records kind 1 (timeout)
+ * and site 5 in the cache's error word and the kernel returns: nothing
+ * faults or hangs and the context stays usable.  Read the result with
+ * fd_get_device_error (FD_ERR_DEVICE_TIMEOUT, code 0x501). */
+fd_status fd_selftest_bounded_wait(fd_cache* cache, int32_t limit_ms,
+                                   void* stream);
+
 /* Number of kernels this library has launched in this process. */
 uint64_t fd_launch_count(void);
 

@@ -25,7 +25,8 @@ EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
            "fd_cache_reset", "fd_rope3d", "fd_block_attention",
            "fd_block_attention_static",
            "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
-           "fd_exp2_selfcheck", "fd_launch_count", "fd_status_string"]
+           "fd_exp2_selfcheck", "fd_selftest_bounded_wait", "fd_launch_count",
+           "fd_status_string"]
 
 
 class FdError(RuntimeError):
@@ -86,6 +87,7 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
     lib.fd_cache_frames.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int64)]
     lib.fd_get_device_error.argtypes = [vp, ctypes.POINTER(i32)]
     lib.fd_exp2_selfcheck.argtypes = [vp, vp, ctypes.c_int64, vp]
+    lib.fd_selftest_bounded_wait.argtypes = [vp, i32, vp]
     lib.fd_launch_count.argtypes = []
     lib.fd_launch_count.restype = ctypes.c_uint64
     lib.fd_status_string.argtypes = [i32]
@@ -230,6 +232,11 @@ def fd_cache_frames(cache: Cache, layer: int, rollout: int) -> int:
 def fd_exp2_selfcheck(x, y, stream=None) -> None:
     _check(load().fd_exp2_selfcheck(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
            "fd_exp2_selfcheck")
+
+
+def fd_selftest_bounded_wait(cache: Cache, limit_ms: int, stream=None) -> None:
+    _check(load().fd_selftest_bounded_wait(cache.handle, limit_ms, _stream(stream)),
+           "fd_selftest_bounded_wait")
 
 
 def fd_get_device_error(cache: Cache) -> int:

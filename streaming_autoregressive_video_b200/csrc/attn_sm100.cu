@@ -95,25 +95,33 @@ constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
 constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
 
 // Site codes for the device error word.
-enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4 };
+enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4,
+             kSiteSelftest = 5 };
 
 // Bounded wait.  kSpin (MMA issuer, softmax: the critical path) polls, so
 // the waiter resumes as soon as the phase completes; the other roles sleep
 // between polls and leave issue slots to the working warps.
-template <bool kSpin = false>
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
-                                         Shared* sh, int32_t* err, int site) {
+template <bool kSpin>
+__device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity,
+                                             int32_t* abort, int32_t* err,
+                                             int site, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!(kSpin ? mbar_try_wait(bar, parity) : mbar_try_wait_sleep(bar, parity))) {
-    if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
+    if (*reinterpret_cast<volatile int32_t*>(abort)) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *reinterpret_cast<volatile int32_t*>(abort) = 1;
       atomicCAS(err, 0, kDevErrTimeout | (site << 8));
       return false;
     }
   }
   return true;
+}
+
+template <bool kSpin = false>
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
+                                         Shared* sh, int32_t* err, int site) {
+  return bounded_wait<kSpin>(bar, parity, &sh->abort, err, site, kWaitLimitNs);
 }
 
 // Bounded wait used only while tearing down after an abort.
@@ -655,6 +663,32 @@ __global__ void exp2_selfcheck_kernel(const float* x, float* y, int64_t n) {
 }
 
 }  // namespace
+
+namespace {
+// One thread waits on an mbarrier that nothing ever arrives at, through the
+// same bounded wait the attention kernel uses, with a short limit: the wait
+// gives up, records (timeout, site 5) in the error word and the kernel
+// returns normally, so the context stays usable.
+__global__ void bounded_wait_selftest_kernel(int32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int32_t abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    bounded_wait<false>(&bar, 0, &abort, err, kSiteSelftest, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_bounded_wait_selftest(int32_t* err, uint64_t limit_ns,
+                                         cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  count_launch(1);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_exp2_selfcheck(const float* x, float* y, int64_t n,
                                   cudaStream_t s) {

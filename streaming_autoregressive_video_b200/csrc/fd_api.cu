@@ -490,6 +490,16 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code) {
   return FD_OK;
 }
 
+fd_status fd_selftest_bounded_wait(fd_cache* cache, int32_t limit_ms,
+                                   void* stream) {
+  if (cache == nullptr || limit_ms < 1 || limit_ms > 2000) return FD_ERR_INVALID_ARG;
+  fd_status st = fd::check_device(cache);
+  if (st != FD_OK) return st;
+  return fd::cuda_status(fd::launch_bounded_wait_selftest(
+      cache->view.err, (uint64_t)limit_ms * 1000000ull,
+      static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 extern "C" fd_status fd_exp2_selfcheck(const float* x, float* y, int64_t n,

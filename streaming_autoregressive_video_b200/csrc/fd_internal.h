@@ -112,6 +112,8 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const AttnParams& p, cudaStream_t s);
 
 void count_launch(int n);
+cudaError_t launch_bounded_wait_selftest(int32_t* err, uint64_t limit_ns,
+                                         cudaStream_t s);
 
 // Shared body of the attention entry points.  `work` is a device area for the
 // block's rotated keys ([n_rollouts][F*Tf][H][d], block_work_bytes bytes,

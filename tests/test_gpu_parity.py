@@ -148,3 +148,80 @@ def test_softmax_exp2_against_exp2f():
     assert float(((poly - ref).abs() / ref).max()) <= 2.0e-4
     assert float(((poly - exact).abs() / exact).max()) <= 2.0e-4
     assert float(((hw - exact).abs() / exact).max()) <= 1.0e-5
+
+
+def test_device_wait_gives_up_and_reports():
+    """A device-side wait on a barrier nothing completes gives up after its
+    limit, sets the error word (timeout, site 5) and leaves the context usable."""
+    w = TINY_F32
+    ls = Lockstep(w)
+    assert fd.fd_get_device_error(ls.cache) == 0
+    fd.fd_selftest_bounded_wait(ls.cache, 50)
+    torch.cuda.synchronize()
+    assert fd.fd_get_device_error(ls.cache) == (5 << 8) | 1
+    assert fd.fd_get_device_error(ls.cache) == 0       # read clears it
+    q, k, v = block_inputs(w, (6, 0), 1)               # the context still works
+    ls.attention(0, q, k, v, what="after self-test")
+    assert fd.fd_get_device_error(ls.cache) == 0
+
+
+def test_block_captured_in_cuda_graph_matches_eager():
+    """One block (denoising steps x layers + commit) captured once in a CUDA
+    graph and replayed for three blocks gives bit-identical outputs and cache
+    contents to eager calls (no host synchronisation inside the calls; the
+    device counters drive the positions)."""
+    w = SMALL.scaled(rollouts=2)
+    eager, graphed = Lockstep(w), Lockstep(w)
+    shape_q = (w.rollouts, w.queries, w.heads, w.head_dim)
+    shape_k = (w.rollouts, w.block_frames * w.frame_tokens, w.heads, w.head_dim)
+    sq = [[torch.empty(shape_q, dtype=torch.int16, device="cuda") for _ in range(w.layers)]
+          for _ in range(w.steps)]
+    sk = [[torch.empty(shape_k, dtype=torch.int16, device="cuda") for _ in range(w.layers)]
+          for _ in range(w.steps)]
+    sv = [[torch.empty(shape_k, dtype=torch.int16, device="cuda") for _ in range(w.layers)]
+          for _ in range(w.steps)]
+    outs = [[torch.empty(shape_q, dtype=torch.int16, device="cuda") for _ in range(w.layers)]
+            for _ in range(w.steps)]
+
+    def block(cache):
+        for s in range(w.steps):
+            for l in range(w.layers):
+                fd.fd_block_attention(cache, l, w.rollouts, sq[s][l], sk[s][l], sv[s][l],
+                                      outs[s][l])
+        fd.fd_cache_commit(cache, 0, w.layers, w.rollouts, sk[-1], sv[-1])
+
+    def fill(blk):
+        for s in range(w.steps):
+            for l in range(w.layers):
+                q, k, v = block_inputs(w, (8, blk, s, l), w.rollouts)
+                sq[s][l].copy_(to_device(q))
+                sk[s][l].copy_(to_device(k))
+                sv[s][l].copy_(to_device(v))
+
+    # warm-up launch outside capture (first-call set-up happens here)
+    fill(0)
+    block(eager.cache)
+    want0 = [[o.clone() for o in row] for row in outs]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        block(graphed.cache)
+    for blk in range(3):
+        fill(blk)
+        g.replay()
+        torch.cuda.synchronize()
+        got = [[o.clone() for o in row] for row in outs]
+        if blk > 0:
+            block(eager.cache)
+            torch.cuda.synchronize()
+            want = [[o.clone() for o in row] for row in outs]
+        else:
+            want = want0
+        for s in range(w.steps):
+            for l in range(w.layers):
+                assert torch.equal(got[s][l], want[s][l]), (blk, s, l)
+    ke, ve, pe, ce = views(eager.cache, w)
+    kg, vg, pg, cg = views(graphed.cache, w)
+    assert torch.equal(pe, pg) and torch.equal(ce, cg)
+    assert torch.equal(ke, kg) and torch.equal(ve, vg)
+    assert fd.fd_get_device_error(graphed.cache) == 0
