@@ -104,6 +104,13 @@ typedef struct {
  *          block's keys rotated once per call, read by every query tile
  *          (one region per layer, so calls on different layers may run
  *          concurrently; calls on the same layer must be ordered)
+ *   part : [L][148][2][256*128 + 512] float work area of the bf16 attention
+ *          kernel: a CTA whose share of the work ends or begins inside a
+ *          query tile pair leaves its partial result there (unnormalised
+ *          output rows, running max, row sum); empty (size 0) for fp32
+ *   cnt  : [L][R][H][ceil(F*T/256)] int32 arrival counters of those split
+ *          tile pairs; zero between calls (the last arriving CTA combines
+ *          the partial results and clears its counter)
  *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
  *   count: [L][R] int32, frames committed since the last reset (n)
  *   ttab : [L][R][S+W+F][p_t] float2 (cos, sin) of the t-section angles for
@@ -111,7 +118,7 @@ typedef struct {
  *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
  *   err  : int32 device error word (0 = none)                            */
 typedef struct {
-  size_t k, v, krot, kblk, pos, count, ttab, htab, wtab, err;
+  size_t k, v, krot, kblk, part, cnt, pos, count, ttab, htab, wtab, err;
   size_t total;           /* == fd_cache_bytes(desc)                       */
   size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
   int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
@@ -170,6 +177,11 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * The cache is read only: call it once per denoising step, then commit.
  * bf16 runs on tcgen05 tensor cores (fp32 accumulation, P rounded to bf16),
  * f32 on CUDA cores in fp32 (no TF32).  Tensor bases must be 16-byte aligned.
+ * The bf16 kernel is persistent (one CTA per multiprocessor, at most 148)
+ * and splits the call's KV iterations evenly over its CTAs; it returns
+ * FD_ERR_UNSUPPORTED when n_rollouts x H x ceil(F*T/256) x (ceil((S+W)*Tf
+ * /128) + ceil(F*Tf/128)) x CTAs reaches 2^31.  A query-tile pair split
+ * between CTAs is combined through the layer's `part` / `cnt` regions.
  * Device-side waits are bounded: a wait that gives up sets the error word
  * (fd_get_device_error) instead of hanging. */
 fd_status fd_block_attention(fd_cache* cache, int32_t layer,

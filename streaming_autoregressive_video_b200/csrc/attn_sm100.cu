@@ -13,9 +13,22 @@
 // call by a pass over the block before this kernel), because every query
 // tile of a head reads the same keys.
 //
-// Design (one CTA = two 128-row query tiles of one (rollout, head)):
-//   warp 0        TMA producer: Q tiles once, then K and V tiles through
-//                 2-stage K and V shared-memory rings, walking
+// Schedule (persistent): a work unit is one 256-row query-tile pair of one
+// (rollout, head) against all of the rollout's KV tiles.  The units' KV
+// iterations, laid end to end (rollout, head, pair, KV tile), are cut into G
+// equal ranges, one per CTA and G = one CTA per multiprocessor, so every CTA
+// does the same number of KV tiles (+-1) whatever the number of units: no
+// partly idle last wave.  A unit cut by a range boundary is computed in
+// pieces; every piece but the last to finish leaves its unnormalised rows,
+// row maxima and row sums (fp32) in the layer's partial-result area and
+// counts itself in the unit's arrival counter; the piece that arrives last
+// folds the others into its own rows, writes them and clears the counter.
+// No CTA ever waits for another.
+//
+// Roles (all warps walk the same sequence of pieces):
+//   warp 0        TMA producer: each piece's two Q tiles (once the previous
+//                 piece's last S product has read the old ones), then K and V
+//                 tiles through 2-stage K and V shared-memory rings, walking
 //                 the valid slot prefix of the cache and then the block; the
 //                 ring's wraparound needs no gather because attention does
 //                 not depend on key order.  No cluster multicast.
@@ -24,7 +37,7 @@
 //                 two query tiles ping-pong so one tile's softmax overlaps the
 //                 other tile's matrix products.
 //   warp 2        TMEM allocator (512 columns: S0, S1, O0, O1).
-//   warps 4-7     RoPE: rotate the two Q tiles in place in the swizzled
+//   warps 4-7     RoPE: rotate each piece's Q tiles in place in the swizzled
 //                 shared-memory layout, cos/sin from the cache's tables
 //                 (fp64-accurate angles rounded once to fp32).
 //   warps 8-15    softmax on one tile at a time, two threads per query row
@@ -35,7 +48,8 @@
 //                 O rescale is skipped unless the running max grows by more
 //                 than 2^8, which keeps P <= 256 and the result exact up to
 //                 rounding.  The epilogue divides by the row sum and writes
-//                 bf16 rows (and the optional log-sum-exp).
+//                 bf16 rows (and the optional log-sum-exp), or hands a split
+//                 unit's piece over as described above.
 // Every mbarrier wait is bounded: a wait that gives up raises a CTA-wide
 // abort flag and the device error word, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is released and the CTA exits.
@@ -77,19 +91,24 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct Shared {
-  uint64_t q_full, q_ready;
+  uint64_t q_full, q_ready, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t red_bar[2][4];  // per tile and lane quarter: row halves exchange
-  uint64_t o_full, drain;
+  uint64_t o_full, o_empty, drain;
+  uint64_t tab_bar;   // RoPE warpgroup: tables of the next rollout staged
+  uint64_t part_bar;  // softmax: a piece's partial rows written
+  uint64_t last_bar;  // softmax: the piece's arrival counted
   uint32_t tmem_base;
   int32_t abort;
+  int32_t last;       // this piece arrived last: it writes the unit's rows
 };
 
 // RoPE tables follow the barriers; the dynamic size adds them per launch.
-constexpr uint32_t kOffRed = kOffShared + 256;   // [2][2][128] floats
-constexpr uint32_t kOffTab = kOffRed + 2 * 2 * 128 * 4;
+constexpr uint32_t kOffRed = kOffShared + 256;   // [2 buffers][2][2][128] floats
+constexpr uint32_t kOffMeta = kOffRed + 2 * 2 * 2 * 128 * 4;  // struct Meta
+constexpr uint32_t kOffTab = kOffMeta + 256;
 static_assert(sizeof(Shared) <= 256, "barrier block");
 constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
 constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
@@ -146,6 +165,140 @@ __device__ __forceinline__ TileCounts tile_counts(const AttnParams& p, int r) {
   t.nt = t.nt1 + (t.n2 + kBN - 1) / kBN;
   return t;
 }
+
+// ---------------------------------------------------------------- schedule
+// Work unit u = (rollout, head, pair) in that order; unit u has nt(rollout)
+// KV iterations.  With U units and G CTAs, the first W = floor(U / G) waves
+// run whole units (CTA c takes units c, c + G, ...: the CTAs of one head
+// stream the same K/V tiles at the same time, so most of them come from L2);
+// the iterations of the remaining U - W*G units, laid end to end, are cut
+// into G equal ranges, one per CTA (its range starts at the SK iteration
+// sk0 + c * I2 / G of the call's iteration space).  The host bounds the
+// call's iterations so that iterations x G < 2^31: all of this is 32-bit.
+struct Sched {
+  int W;    // whole-unit waves
+  int sk0;  // first iteration of the split part
+  int I2;   // iterations of the split part
+};
+
+__device__ __forceinline__ Sched make_sched(const AttnParams& p) {
+  const int per_r = p.H * p.nb;
+  Sched s;
+  s.W = p.n_rollouts * per_r / p.G;
+  const int D = s.W * p.G;  // units run whole
+  int total = 0, below = 0;
+  for (int r = 0; r < p.n_rollouts; ++r) {
+    const int nt = tile_counts(p, r).nt;
+    total += per_r * nt;
+    below += min(max(D - r * per_r, 0), per_r) * nt;
+  }
+  s.sk0 = below;
+  s.I2 = total - below;
+  return s;
+}
+
+// First iteration of CTA c's split range.
+__device__ __forceinline__ int cta_begin(int c, const Sched& s, int G) {
+  return s.sk0 + c * s.I2 / G;
+}
+
+// The (non-empty) CTA whose split range holds iteration x.
+__device__ __forceinline__ int cta_of(int x, const Sched& s, int G) {
+  return ((x - s.sk0 + 1) * G - 1) / s.I2;
+}
+
+// One unit's share of a CTA's work: KV tiles [kv0, kv1) of query-tile pair
+// b of (rollout r, head h); the unit's iterations start at U0.
+struct Piece {
+  int r, h, b, kv0, kv1, unit, U0;
+  TileCounts tc;
+};
+
+struct Cursor {
+  int w;        // next whole-unit wave
+  int it, end;  // next iteration, end of this CTA's split range
+  int base;     // first iteration of rollout r
+  int r;
+  TileCounts tc;
+};
+
+__device__ __forceinline__ Cursor cursor_init(const AttnParams& p, const Sched& s) {
+  Cursor c;
+  c.w = 0;
+  c.it = cta_begin(blockIdx.x, s, p.G);
+  c.end = cta_begin(blockIdx.x + 1, s, p.G);
+  c.base = 0;
+  c.r = 0;
+  c.tc = tile_counts(p, 0);
+  return c;
+}
+
+// Next piece of this CTA's work, or false at its end.
+__device__ __forceinline__ bool next_piece(const AttnParams& p, const Sched& s,
+                                           Cursor& c, Piece& pc) {
+  const int per_r = p.H * p.nb;
+  if (c.w < s.W) {  // a whole unit
+    const int unit = c.w * p.G + blockIdx.x;
+    ++c.w;
+    pc.r = unit / per_r;
+    const int u = unit - pc.r * per_r;
+    pc.tc = tile_counts(p, pc.r);
+    pc.h = u / p.nb;
+    pc.b = u - pc.h * p.nb;
+    pc.kv0 = 0;
+    pc.kv1 = pc.tc.nt;
+    pc.unit = unit;
+    pc.U0 = -1;  // not used by whole units
+    return true;
+  }
+  if (c.it >= c.end) return false;
+  int span = per_r * c.tc.nt;
+  while (c.it >= c.base + span && c.r + 1 < p.n_rollouts) {
+    c.base += span;
+    ++c.r;
+    c.tc = tile_counts(p, c.r);
+    span = per_r * c.tc.nt;
+  }
+  const int rel = c.it - c.base;
+  const int u = rel / c.tc.nt;
+  pc.r = c.r;
+  pc.tc = c.tc;
+  pc.h = u / p.nb;
+  pc.b = u - pc.h * p.nb;
+  pc.U0 = c.base + u * c.tc.nt;
+  pc.kv0 = c.it - pc.U0;
+  pc.kv1 = min(c.tc.nt, c.end - pc.U0);
+  pc.unit = c.r * per_r + u;
+  c.it = pc.U0 + pc.kv1;
+  return true;
+}
+
+// Partial-result slot of CTA c's piece of the split unit starting at U0:
+// slot 0 when the piece opens the CTA's split range, slot 1 when it closes it.
+__device__ __forceinline__ const float* part_slot(const AttnParams& p, int c,
+                                                  int U0, const Sched& s) {
+  const int slot = cta_begin(c, s, p.G) >= U0 ? 0 : 1;
+  return p.part + ((size_t)c * 2 + slot) * kPartSlotFloats;
+}
+
+// What every role needs to know about a piece.  The producer walks the
+// schedule and publishes each piece in a 4-entry ring in shared memory
+// (entry k & 3, `seq` = k written last); the other roles read the entry
+// after their first wait for that piece, so only the producer holds the
+// schedule's cursor in registers.  A piece's entry is overwritten four
+// pieces later, long after every role has finished with it.
+struct PieceInfo {
+  int r, h, b, kv0, kv1, unit, U0, nt, nt1, n1, n2;
+  int seq;
+};
+
+struct Meta {
+  PieceInfo ring[4];
+  int n_pieces;   // pieces of this CTA
+  int my_begin;   // first iteration of this CTA's split range
+  Sched sd;
+};
+static_assert(sizeof(Meta) <= 256, "meta block");
 
 // ---------------------------------------------------------------- RoPE
 // Thread `tid` (0..127) of the RoPE warpgroup owns 16-byte chunk cc = tid%16
@@ -241,6 +394,57 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// Reads ring entry k once the producer has published it (bounded wait).
+__device__ __forceinline__ bool read_piece(const Meta* meta, int k, PieceInfo& pi,
+                                           Shared* sh, int32_t* err, int site) {
+  const volatile PieceInfo* e = &meta->ring[k & 3];
+  if (e->seq != k) {
+    const uint64_t t0 = globaltimer_ns();
+    while (e->seq != k) {
+      if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
+        atomicCAS(err, 0, kDevErrTimeout | (site << 8));
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  pi.r = e->r;
+  pi.h = e->h;
+  pi.b = e->b;
+  pi.kv0 = e->kv0;
+  pi.kv1 = e->kv1;
+  pi.unit = e->unit;
+  pi.U0 = e->U0;
+  pi.nt = e->nt;
+  pi.nt1 = e->nt1;
+  pi.n1 = e->n1;
+  pi.n2 = e->n2;
+  pi.seq = k;
+  return true;
+}
+
+// KV iterations of ring entry k (what the MMA issuer needs of a piece).
+__device__ __forceinline__ bool read_piece_len(const Meta* meta, int k, int& n,
+                                               Shared* sh, int32_t* err, int site) {
+  const volatile PieceInfo* e = &meta->ring[k & 3];
+  if (e->seq != k) {
+    const uint64_t t0 = globaltimer_ns();
+    while (e->seq != k) {
+      if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *reinterpret_cast<volatile int32_t*>(&sh->abort) = 1;
+        atomicCAS(err, 0, kDevErrTimeout | (site << 8));
+        return false;
+      }
+    }
+  }
+  __threadfence_block();
+  n = e->kv1 - e->kv0;
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bf16_d128_sm100(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_kc,
@@ -252,15 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Shared* sh = reinterpret_cast<Shared*>(smem + kOffShared);
+  Meta* meta = reinterpret_cast<Meta*>(smem + kOffMeta);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, r = blockIdx.z;
-  const int qrow0 = blockIdx.x * (2 * kBM);
-  const TileCounts tc = tile_counts(p, r);
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
     mbar_init(&sh->q_ready, 128);
+    mbar_init(&sh->q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sh->k_full[s], 1);
       mbar_init(&sh->k_empty[s], 1);
@@ -275,9 +478,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 4; ++q) mbar_init(&sh->red_bar[x][q], 64);
     }
     mbar_init(&sh->o_full, 1);
+    mbar_init(&sh->o_empty, 256);
     mbar_init(&sh->drain, 1);
+    mbar_init(&sh->tab_bar, 128);
+    mbar_init(&sh->part_bar, 256);
+    mbar_init(&sh->last_bar, 1);
     sh->abort = 0;
+    sh->last = 0;
     fence_mbarrier_init();
+    // the CTA's schedule: how many pieces, where its split range starts
+    const Sched sd = make_sched(p);
+    Cursor c = cursor_init(p, sd);
+    meta->sd = sd;
+    meta->my_begin = c.it;
+    int n = 0;
+    Piece pc;
+    while (next_piece(p, sd, c, pc)) ++n;
+    meta->n_pieces = n;
+    for (int i = 0; i < 4; ++i) meta->ring[i].seq = -1;
   }
   if (warp == 2) {
     tmem_alloc(&sh->tmem_base, 512);
@@ -287,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  const int n_pieces = meta->n_pieces;
 
   // Register split (launch: 512 threads x 128): the producer/MMA warpgroup and
   // the RoPE warpgroup give registers to the two softmax warpgroups, which
@@ -295,7 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // and never takes registers back: a later increase could claim registers a
   // softmax warpgroup is still waiting for.  Each branch ends in its own
   // teardown (block-wide named barrier, then TMEM release) and returns, so no
-  // code runs after the branches join.
+  // code runs after the branches join.  Inside a branch, groups of warps
+  // synchronise only through bounded mbarrier waits (a warp that gives up
+  // must not leave the others blocked on a named barrier).
   if (warp < 4) {
     regs_dec<88>();
     if (warp == 0) {
@@ -306,46 +527,77 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_vc);
       prefetch_tmap(&tm_kb);
       prefetch_tmap(&tm_vb);
-      mbar_arrive_expect_tx(&sh->q_full, 2 * kTile);
-      for (int t = 0; t < 2; ++t)
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_4d(smem + kOffQ + t * kTile + hf * kHalf, &tm_q, &sh->q_full,
-                      hf * 64, h, qrow0 + t * kBM, r);
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < tc.nt; ++j) {
-        const bool seg1 = j < tc.nt1;
-        const int key0 = seg1 ? j * kBN : (j - tc.nt1) * kBN;
+      const Sched sd = meta->sd;
+      Cursor cur = cursor_init(p, sd);
+      Piece pc;
+      int g = 0, issued_k = 0, issued_v = 0;  // KV iterations of the CTA
+      int issued_q = 0;                       // pieces of the CTA
+      bool ok = true;
+      for (int k = 0; ok && next_piece(p, sd, cur, pc); ++k) {
+        // the Q tiles are reused once the previous piece's S products are done
+        if (k > 0 && !wait_bar(&sh->q_empty, (k - 1) & 1, sh, p.err, kSiteProducer)) {
+          ok = false;
+          break;
+        }
+        volatile PieceInfo* e = &meta->ring[k & 3];
+        e->r = pc.r;
+        e->h = pc.h;
+        e->b = pc.b;
+        e->kv0 = pc.kv0;
+        e->kv1 = pc.kv1;
+        e->unit = pc.unit;
+        e->U0 = pc.U0;
+        e->nt = pc.tc.nt;
+        e->nt1 = pc.tc.nt1;
+        e->n1 = pc.tc.n1;
+        e->n2 = pc.tc.n2;
+        __threadfence_block();
+        e->seq = k;
+        mbar_arrive_expect_tx(&sh->q_full, 2 * kTile);
+        for (int t = 0; t < 2; ++t)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(smem + kOffQ + t * kTile + hf * kHalf, &tm_q, &sh->q_full,
+                        hf * 64, pc.h, pc.b * 2 * kBM + t * kBM, pc.r);
+        issued_q = k + 1;
         // keys: rotated cache keys or the block keys rotated for this call,
         // both batched by (layer, rollout); values: cache (layer, rollout)
         // or the caller's block values (rollout)
-        const CUtensorMap* mk = seg1 ? &tm_kc : &tm_kb;
-        const CUtensorMap* mv = seg1 ? &tm_vc : &tm_vb;
-        const int ck3 = seg1 ? p.map_row0 + r : p.kb_row0 + r;
-        const int cv3 = seg1 ? p.map_row0 + r : r;
-        const int ks = j % kKStages;
-        if (j >= kKStages &&
-            !wait_bar(&sh->k_empty[ks], ((j / kKStages) - 1) & 1, sh, p.err,
-                      kSiteProducer))
-          break;
-        mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
-                      &sh->k_full[ks], hf * 64, h, key0, ck3);
-        issued_k = j + 1;
-        const int vs = j % kVStages;
-        if (j >= kVStages &&
-            !wait_bar(&sh->v_empty[vs], ((j / kVStages) - 1) & 1, sh, p.err,
-                      kSiteProducer))
-          break;
-        mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
-                      &sh->v_full[vs], hf * 64, h, key0, cv3);
-        issued_v = j + 1;
+        for (int j = pc.kv0; j < pc.kv1; ++j, ++g) {
+          const bool seg1 = j < pc.tc.nt1;
+          const int key0 = seg1 ? j * kBN : (j - pc.tc.nt1) * kBN;
+          const CUtensorMap* mk = seg1 ? &tm_kc : &tm_kb;
+          const CUtensorMap* mv = seg1 ? &tm_vc : &tm_vb;
+          const int ck3 = seg1 ? p.map_row0 + pc.r : p.kb_row0 + pc.r;
+          const int cv3 = seg1 ? p.map_row0 + pc.r : pc.r;
+          const int ks = g % kKStages;
+          if (g >= kKStages &&
+              !wait_bar(&sh->k_empty[ks], ((g / kKStages) - 1) & 1, sh, p.err,
+                        kSiteProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
+                        &sh->k_full[ks], hf * 64, pc.h, key0, ck3);
+          issued_k = g + 1;
+          const int vs = g % kVStages;
+          if (g >= kVStages &&
+              !wait_bar(&sh->v_empty[vs], ((g / kVStages) - 1) & 1, sh, p.err,
+                        kSiteProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
+                        &sh->v_full[vs], hf * 64, pc.h, key0, cv3);
+          issued_v = g + 1;
+        }
       }
       if (*reinterpret_cast<volatile int32_t*>(&sh->abort)) {
         // let every copy still in flight land before the CTA exits
-        drain_bar(&sh->q_full, 0);
+        if (issued_q > 0) drain_bar(&sh->q_full, (issued_q - 1) & 1);
         for (int j = max(0, issued_k - kKStages); j < issued_k; ++j)
           drain_bar(&sh->k_full[j % kKStages], (j / kKStages) & 1);
         for (int j = max(0, issued_v - kVStages); j < issued_v; ++j)
@@ -356,69 +608,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t sq = smem_addr(smem + kOffQ);
-      const uint32_t sk = smem_addr(smem + kOffK);
-      const uint32_t sv = smem_addr(smem + kOffV);
+      // Shared-memory descriptors as (lo, hi) halves: hi (stride 1024 B,
+      // version 1, 128-byte swizzle) is common to all tiles; lo is the tile's
+      // address >> 4 with the leading-byte offset (16 B for the K-major Q and
+      // K tiles, one 64-column half for the MN-major V tile), and a k-step
+      // inside the tile adds its byte offset >> 4.  The bases are made opaque
+      // per call so the compiler adds the step offsets as it issues instead
+      // of keeping every (tile, step) descriptor live across the loop.
+      constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      const uint32_t q_lo = ((smem_addr(smem + kOffQ) & 0x3FFFFu) >> 4) | (1u << 16);
+      const uint32_t k_lo = ((smem_addr(smem + kOffK) & 0x3FFFFu) >> 4) | (1u << 16);
+      const uint32_t v_lo = ((smem_addr(smem + kOffV) & 0x3FFFFu) >> 4) | ((kHalf >> 4) << 16);
+      const uint32_t desc_hi = kDescHi;
       auto issue_s = [&](int x, int ks) {
-        const uint32_t qa = sq + x * kTile, kb = sk + ks * kTile;
+        uint32_t a = q_lo + x * (kTile >> 4), b = k_lo + ks * (kTile >> 4);
+        asm volatile("" : "+r"(a), "+r"(b));
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-          mma_ss(tmem + kColS0 + x * 128, sdesc_sw128(qa + off, 16, 1024),
-                 sdesc_sw128(kb + off, 16, 1024), kIdescQK, kk > 0);
+          const uint32_t step = (kk >> 2) * (kHalf >> 4) + (kk & 3) * 2;  // 32 B per k-step
+          mma_ss_lo(tmem + kColS0 + x * 128, a + step, b + step, desc_hi, kIdescQK, kk > 0);
         }
       };
       auto issue_pv = [&](int x, int vs, bool acc) {
-        const uint32_t vb = sv + vs * kTile;
+        uint32_t b = v_lo + vs * (kTile >> 4);
+        asm volatile("" : "+r"(b));
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts(tmem + kColO0 + x * 128, tmem + kColS0 + x * 128 + kk * 8,
-                 sdesc_sw128(vb + kk * 2048, kHalf, 1024), kIdescPV,
-                 (acc || kk > 0) ? 1u : 0u);
+          mma_ts_lo(tmem + kColO0 + x * 128, tmem + kColS0 + x * 128 + kk * 8,
+                    b + kk * (2048 >> 4), desc_hi, kIdescPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       // K tiles arrive rotated (cache keys at commit, block keys once per
       // call), so a K tile is ready as soon as its copy has landed.
-      auto wait_k = [&](int j) -> bool {
-        return wait_bar<true>(&sh->k_full[j % kKStages], (j / kKStages) & 1, sh,
-                              p.err, kSiteMma);
+      auto wait_k = [&](int g) -> bool {
+        return wait_bar<true>(&sh->k_full[g % kKStages], (g / kKStages) & 1, sh, p.err,
+                              kSiteMma);
       };
-      bool ok = wait_bar<true>(&sh->q_ready, 0, sh, p.err, kSiteMma) && wait_k(0);
-      if (ok) {
+      int g = 0;
+      bool ok = true;
+      for (int k = 0; k < n_pieces && ok; ++k) {
+        int n = 0;
+        ok = wait_bar<true>(&sh->q_ready, k & 1, sh, p.err, kSiteMma) &&
+             read_piece_len(meta, k, n, sh, p.err, kSiteMma) && wait_k(g);
+        if (!ok) break;
         tc_fence_after();
-        issue_s(0, 0);
+        const int ks0 = g % kKStages;
+        issue_s(0, ks0);
         mma_commit(&sh->s_full[0]);
-        issue_s(1, 0);
+        issue_s(1, ks0);
         mma_commit(&sh->s_full[1]);
-        mma_commit(&sh->k_empty[0]);
-        for (int j = 0; j < tc.nt && ok; ++j) {
-          const int vs = j % kVStages;
-          ok = wait_bar<true>(&sh->v_full[vs], (j / kVStages) & 1, sh, p.err, kSiteMma) &&
-               wait_bar<true>(&sh->p_full[0], j & 1, sh, p.err, kSiteMma);
+        mma_commit(&sh->k_empty[ks0]);
+        if (n == 1) mma_commit(&sh->q_empty);
+        for (int jj = 0; jj < n; ++jj) {
+          const int gj = g + jj;
+          const int vs = gj % kVStages;
+          ok = wait_bar<true>(&sh->v_full[vs], (gj / kVStages) & 1, sh, p.err, kSiteMma) &&
+               wait_bar<true>(&sh->p_full[0], gj & 1, sh, p.err, kSiteMma);
+          // the first products of a piece overwrite O: the previous piece's
+          // epilogue must have read it
+          if (ok && jj == 0 && k > 0)
+            ok = wait_bar<true>(&sh->o_empty, (k - 1) & 1, sh, p.err, kSiteMma);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(0, vs, j > 0);
-          const bool more = j + 1 < tc.nt;
-          const int ks = (j + 1) % kKStages;
+          issue_pv(0, vs, jj > 0);
+          const bool more = jj + 1 < n;
+          const int ks = (gj + 1) % kKStages;
           if (more) {
-            ok = wait_k(j + 1);
+            ok = wait_k(gj + 1);
             if (!ok) break;
             tc_fence_after();
             issue_s(0, ks);
             mma_commit(&sh->s_full[0]);
           }
-          ok = wait_bar<true>(&sh->p_full[1], j & 1, sh, p.err, kSiteMma);
+          ok = wait_bar<true>(&sh->p_full[1], gj & 1, sh, p.err, kSiteMma);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(1, vs, j > 0);
+          issue_pv(1, vs, jj > 0);
           mma_commit(&sh->v_empty[vs]);
           if (more) {
             issue_s(1, ks);
             mma_commit(&sh->s_full[1]);
             mma_commit(&sh->k_empty[ks]);
+            if (jj + 2 == n) mma_commit(&sh->q_empty);  // last S products of the piece
           }
         }
+        if (!ok) break;
         mma_commit(&sh->o_full);
+        g += n;
       }
       if (!ok) {
         // wait for the tensor core to finish what was issued
@@ -435,21 +711,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ RoPE
     const int tid = threadIdx.x - 128;
     const RopeLane rl = rope_lane(p, tid);
-    // stage this rollout's t table and the static h / w tables
+    // this rollout's t table and the static h / w tables, in shared memory
     float2* st = reinterpret_cast<float2*>(smem + kOffTab);
     const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph, n_w = p.gw * p.pw;
-    const float2* tt = p.ttab + (size_t)r * n_t;
-    for (int i = tid; i < n_t; i += 128) st[i] = tt[i];
-    for (int i = tid; i < n_h; i += 128) st[n_t + i] = p.htab[i];
-    for (int i = tid; i < n_w; i += 128) st[n_t + n_h + i] = p.wtab[i];
-    asm volatile("bar.sync 2, 128;" ::: "memory");
-    bool ok = __all_sync(0xffffffffu, wait_bar(&sh->q_full, 0, sh, p.err, kSiteRope));
-    if (ok) {
+    int staged = -1;
+    uint32_t n_stage = 0;
+    bool ok = true;
+    for (int k = 0; k < n_pieces && ok; ++k) {
+      PieceInfo pi;
+      ok = __all_sync(0xffffffffu, wait_bar(&sh->q_full, k & 1, sh, p.err, kSiteRope) &&
+                                       read_piece(meta, k, pi, sh, p.err, kSiteRope));
+      if (!ok) break;
+      if (pi.r != staged) {
+        // every RoPE thread has finished the previous Q tiles (arrived on
+        // q_ready) before the tables are overwritten
+        if (k > 0) {
+          ok = __all_sync(0xffffffffu,
+                          wait_bar(&sh->q_ready, (k - 1) & 1, sh, p.err, kSiteRope));
+          if (!ok) break;
+        }
+        const float2* tt = p.ttab + (size_t)pi.r * n_t;
+        for (int i = tid; i < n_t; i += 128) st[i] = tt[i];
+        for (int i = tid; i < n_h; i += 128) st[n_t + i] = p.htab[i];
+        for (int i = tid; i < n_w; i += 128) st[n_t + n_h + i] = p.wtab[i];
+        mbar_arrive(&sh->tab_bar);
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(&sh->tab_bar, n_stage & 1, sh, p.err, kSiteRope));
+        ++n_stage;
+        if (!ok) break;
+        staged = pi.r;
+      }
+      const int qrow0 = pi.b * 2 * kBM;
       rope_q_tile(smem + kOffQ, qrow0, rl, st, p);
       rope_q_tile(smem + kOffQ + kTile, qrow0 + kBM, rl, st, p);
       fence_proxy_async_smem();
+      mbar_arrive(&sh->q_ready);
     }
-    mbar_arrive(&sh->q_ready);
     teardown(warp, tmem);
     return;
   } else {
@@ -466,145 +763,287 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;           // lane quarter
     const int row_t = wq * 32 + lane;  // row within a tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [tile][half][row]
+    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [buf][tile][half][row]
     const float sl2 = p.scale_log2;
-    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    int g = 0;
+    uint32_t ex_n = 0, n_part = 0;
     bool ok = true;
     uint32_t s[64];
-    // exchange a per-row value with the other column half; bounded wait
-    auto exchange = [&](int x, float mine, uint32_t parity) -> float {
-      red[(x * 2 + hc) * kBM + row_t] = mine;
+    // exchange a per-row value with the other column half; bounded wait.
+    // Exchange rounds alternate between two buffers, so a round's write
+    // never meets the partner's read of the round before.
+    auto exchange = [&](int x, float mine) -> float {
+      float* rb = red + (ex_n & 1) * (2 * 2 * kBM);
+      rb[(x * 2 + hc) * kBM + row_t] = mine;
       mbar_arrive(&sh->red_bar[x][wq]);
-      ok = __all_sync(0xffffffffu, ok && wait_bar<true>(&sh->red_bar[x][wq], parity, sh,
-                                                        p.err, kSiteSoftmax));
-      return red[(x * 2 + (1 - hc)) * kBM + row_t];
+      ok = __all_sync(0xffffffffu, ok && wait_bar<true>(&sh->red_bar[x][wq], ex_n & 1,
+                                                        sh, p.err, kSiteSoftmax));
+      return rb[(x * 2 + (1 - hc)) * kBM + row_t];
     };
-    for (int j = 0; j < tc.nt && ok; ++j) {
-      const int valid = j < tc.nt1 ? min(kBN, tc.n1 - j * kBN)
-                                   : min(kBN, tc.n2 - (j - tc.nt1) * kBN);
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (!ok) break;
-        const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
-        const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+    for (int k = 0; k < n_pieces && ok; ++k) {
+      int n, kv0, nt1, n1, n2;
+      {
+        // the piece's first S product is done, so its ring entry is out
+        PieceInfo pi;
         ok = __all_sync(0xffffffffu,
-                        wait_bar<true>(&sh->s_full[x], j & 1, sh, p.err, kSiteSoftmax));
+                        wait_bar<true>(&sh->s_full[0], g & 1, sh, p.err, kSiteSoftmax) &&
+                            read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
         if (!ok) break;
-        tc_fence_after();
-        tmem_ld64(tS + hc * 64, s);
-        if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
+        n = pi.kv1 - pi.kv0;
+        kv0 = pi.kv0;
+        nt1 = pi.nt1;
+        n1 = pi.n1;
+        n2 = pi.n2;
+      }
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      for (int jj = 0; jj < n && ok; ++jj) {
+        const int gj = g + jj;
+        const int j = kv0 + jj;
+        const int valid = j < nt1 ? min(kBN, n1 - j * kBN) : min(kBN, n2 - (j - nt1) * kBN);
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (hc * 64 + i >= valid) s[i] = 0xFF800000u;
-        }
-        float m8[8];
+        for (int x = 0; x < 2; ++x) {
+          if (!ok) break;
+          const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
+          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+          ok = __all_sync(0xffffffffu, wait_bar<true>(&sh->s_full[x], gj & 1, sh,
+                                                      p.err, kSiteSoftmax));
+          if (!ok) break;
+          tc_fence_after();
+          tmem_ld64(tS + hc * 64, s);
+          if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          m8[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 8]));
+            for (int i = 0; i < 64; ++i)
+              if (hc * 64 + i >= valid) s[i] = 0xFF800000u;
+          }
+          float m8[8];
 #pragma unroll
-        for (int i = 16; i < 64; i += 2)
-          m8[(i >> 1) & 7] = fmaxf(m8[(i >> 1) & 7],
-                                   fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 1])));
-        const float pmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        // both halves of the row have loaded their S columns once this
-        // returns, so P may now overwrite them
-        const float omax = exchange(x, pmax, j & 1);
-        if (!ok) break;
-        const float m_tile = fmaxf(pmax, omax) * sl2;
-        const bool need = m_tile > m[x] + kRescaleThreshold;
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m[x] - m_tile) : 1.f;
+          for (int i = 0; i < 8; ++i)
+            m8[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 8]));
+#pragma unroll
+          for (int i = 16; i < 64; i += 2)
+            m8[(i >> 1) & 7] = fmaxf(m8[(i >> 1) & 7],
+                                     fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 1])));
+          const float pmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          // both halves of the row have loaded their S columns once this
+          // returns, so P may now overwrite them
+          const float omax = exchange(x, pmax);
+          if (!ok) break;
+          const float m_tile = fmaxf(pmax, omax) * sl2;
+          const bool need = m_tile > m[x] + kRescaleThreshold;
+          if (jj > 0 && __any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2_approx(m[x] - m_tile) : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r16[16];
-            tmem_ld16(tO + hc * 64 + c * 16, r16);
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r16[16];
+              tmem_ld16(tO + hc * 64 + c * 16, r16);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
-            tmem_st16(tO + hc * 64 + c * 16, r16);
+              for (int i = 0; i < 16; ++i)
+                r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+              tmem_st16(tO + hc * 64 + c * 16, r16);
+            }
+            tmem_wait_st();
+          }
+          if (need) {
+            l[x] = (jj > 0) ? l[x] * ex2_approx(m[x] - m_tile) : 0.f;
+            m[x] = m_tile;
+          }
+          // P = 2^(s * log2(e)/sqrt(d) - m), two columns per packed
+          // instruction.  In full tiles every kPolyEvery-th pair of
+          // exponentials runs on the FMA pipe (exp2_poly2) to share the load of
+          // the MUFU unit; partial tiles (masked columns at -inf) use MUFU
+          // throughout so masked weights are exactly 0.
+          const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m[x], -m[x]);
+          float ls = 0.f;
+          uint64_t ls2 = 0;  // two packed +0.0f
+          uint32_t pk[32];
+          auto exps = [&](bool full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const uint64_t x2 = f2_fma(
+                  f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
+              float p0, p1;
+              if (full && (i % kPolyEvery) == kPolyEvery - 1) {
+                const uint64_t e2 = exp2_poly2(x2);
+                ls2 = f2_add(ls2, e2);
+                f2_unpack(e2, p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+                ls += p0 + p1;
+              }
+              pk[i] = pack_bf16(p0, p1);
+            }
+          };
+          if (valid == kBN) exps(true); else exps(false);
+          // bf16 P of columns hc*64.. goes to TMEM columns hc*32.. of the tile
+          tmem_st32(tS + hc * 32, pk);
+          {
+            float la, lb;
+            f2_unpack(ls2, la, lb);
+            l[x] += ls + (la + lb);
           }
           tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&sh->p_full[x]);
         }
-        if (need) {
-          l[x] = (j > 0) ? l[x] * ex2_approx(m[x] - m_tile) : 0.f;
-          m[x] = m_tile;
-        }
-        // P = 2^(s * log2(e)/sqrt(d) - m), two columns per packed
-        // instruction.  In full tiles every kPolyEvery-th pair of
-        // exponentials runs on the FMA pipe (exp2_poly2) to share the load of
-        // the MUFU unit; partial tiles (masked columns at -inf) use MUFU
-        // throughout so masked weights are exactly 0.
-        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m[x], -m[x]);
-        float ls = 0.f;
-        uint64_t ls2 = 0;  // two packed +0.0f
-        uint32_t pk[32];
-        auto exps = [&](bool full) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const uint64_t x2 = f2_fma(
-                f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
-            float p0, p1;
-            if (full && (i % kPolyEvery) == kPolyEvery - 1) {
-              const uint64_t e2 = exp2_poly2(x2);
-              ls2 = f2_add(ls2, e2);
-              f2_unpack(e2, p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-              ls += p0 + p1;
-            }
-            pk[i] = pack_bf16(p0, p1);
-          }
-        };
-        if (valid == kBN) exps(true); else exps(false);
-        // bf16 P of columns hc*64.. goes to TMEM columns hc*32.. of the tile
-        tmem_st32(tS + hc * 32, pk);
-        {
-          float la, lb;
-          f2_unpack(ls2, la, lb);
-          l[x] += ls + (la + lb);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&sh->p_full[x]);
+        ++ex_n;
       }
-    }
-    if (ok)
-      ok = __all_sync(0xffffffffu,
-                      wait_bar(&sh->o_full, 0, sh, p.err, kSiteSoftmax));
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
       if (!ok) break;
-      const float l_tot = l[x] + exchange(x, l[x], tc.nt & 1);
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(&sh->o_full, k & 1, sh, p.err, kSiteSoftmax));
+      if (!ok) break;
+      float l_tot[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) l_tot[x] = l[x] + exchange(x, l[x]);
+      ++ex_n;
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
-      const int row = qrow0 + x * kBM + row_t;
-      const float inv_l = 1.f / l_tot;
-      uint16_t* out = static_cast<uint16_t*>(p.out) +
-                      (((size_t)r * p.Mq + row) * p.H + h) * kD + hc * 64;
-      uint32_t rr[32];
+      // the piece again, from its ring entry (not kept in registers above)
+      PieceInfo pi;
+      ok = __all_sync(0xffffffffu, read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
+      if (!ok) break;
+      const Sched sd = meta->sd;
+      const bool whole = pi.kv0 == 0 && pi.kv1 == pi.nt;
+      bool write_rows = whole;
+      // CTAs whose pieces make up the unit, folded in this fixed order (so
+      // the rounding does not depend on which piece arrived last)
+      int c_lo = blockIdx.x, c_hi = blockIdx.x;
+      if (!whole) {
+        // hand this piece over: unnormalised rows, running max, row sum
+        float* part = p.part + ((size_t)blockIdx.x * 2 +
+                                (pi.U0 + pi.kv0 == meta->my_begin ? 0 : 1)) * kPartSlotFloats;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(tO + hc * 64 + c * 32, rr);
-        if (row < p.Mq) {
-          uint32_t pk[16];
+        for (int x = 0; x < 2; ++x) {
+          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+          const int row = x * kBM + row_t;
+          uint32_t rr[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l,
-                              __uint_as_float(rr[2 * i + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(tO + hc * 64 + c * 32, rr);
+            float4* dst = reinterpret_cast<float4*>(part + (size_t)row * kD + hc * 64 + c * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
+                                   __uint_as_float(rr[4 * i + 2]),
+                                   __uint_as_float(rr[4 * i + 3]));
+          }
+          if (hc == 0) {
+            part[2 * kBM * kD + row] = m[x];
+            part[2 * kBM * kD + 2 * kBM + row] = l_tot[x];
+          }
+        }
+        __threadfence();
+        mbar_arrive(&sh->part_bar);
+        if (threadIdx.x == 256) {
+          // all 256 threads' rows are out: count this piece's arrival
+          bool got = wait_bar<true>(&sh->part_bar, n_part & 1, sh, p.err, kSiteSoftmax);
+          int last = 0;
+          if (got) {
+            __threadfence();
+            const int lo = cta_of(pi.U0, sd, p.G), hi = cta_of(pi.U0 + pi.nt - 1, sd, p.G);
+            int pieces = 0;
+            for (int c = lo; c <= hi; ++c)
+              pieces += cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G) ? 1 : 0;
+            const int before = atomicAdd(&p.cnt[pi.unit], 1);
+            last = before == pieces - 1;
+            if (last) {
+              atomicExch(&p.cnt[pi.unit], 0);  // ready for the next call
+              __threadfence();
+            }
+          }
+          *reinterpret_cast<volatile int32_t*>(&sh->last) = last;
+          mbar_arrive(&sh->last_bar);
+        }
+        ok = __all_sync(0xffffffffu,
+                        wait_bar<true>(&sh->last_bar, n_part & 1, sh, p.err, kSiteSoftmax));
+        ++n_part;
+        if (!ok) break;
+        write_rows = *reinterpret_cast<volatile int32_t*>(&sh->last) != 0;
+        if (write_rows) {
+          __threadfence();
+          c_lo = cta_of(pi.U0, sd, p.G);
+          c_hi = cta_of(pi.U0 + pi.nt - 1, sd, p.G);
         }
       }
-      if (p.lse != nullptr && hc == 0 && row < p.Mq)
-        p.lse[((size_t)r * p.H + h) * p.Mq + row] =
-            (m[x] + log2f(l_tot)) * 0.69314718055994530942f;
+      if (write_rows) {
+        // rows = sum over pieces i of O_i 2^(m_i - M) / sum of l_i 2^(m_i - M),
+        // M the largest max; this CTA's own piece comes from TMEM
+        constexpr size_t kOffM = 2 * kBM * kD, kOffL = kOffM + 2 * kBM;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+          const int row = x * kBM + row_t;
+          const int qrow = pi.b * 2 * kBM + row;
+          auto skip = [&](int c) {
+            return c != (int)blockIdx.x && cta_begin(c, sd, p.G) == cta_begin(c + 1, sd, p.G);
+          };
+          auto max_of = [&](int c) {
+            return c == (int)blockIdx.x ? m[x] : __ldcg(part_slot(p, c, pi.U0, sd) + kOffM + row);
+          };
+          float M = -INFINITY;
+          for (int c = c_lo; c <= c_hi; ++c)
+            if (!skip(c)) M = fmaxf(M, max_of(c));
+          auto weight = [&](float mc) { return mc == M ? 1.f : ex2_approx(mc - M); };
+          float L = 0.f;
+          for (int c = c_lo; c <= c_hi; ++c) {
+            if (skip(c)) continue;
+            const float lc = c == (int)blockIdx.x ? l_tot[x]
+                                                  : __ldcg(part_slot(p, c, pi.U0, sd) + kOffL + row);
+            L += lc * weight(max_of(c));
+          }
+          const float inv_l = 1.f / L;
+          uint16_t* out = static_cast<uint16_t*>(p.out) +
+                          (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * kD + hc * 64;
+          uint32_t rr[32];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(tO + hc * 64 + c * 32, rr);
+            float acc[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+            for (int c2 = c_lo; c2 <= c_hi; ++c2) {
+              if (skip(c2)) continue;
+              const float w = weight(max_of(c2));
+              if (c2 == (int)blockIdx.x) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] += w * __uint_as_float(rr[i]);
+              } else {
+                const float4* src = reinterpret_cast<const float4*>(
+                    part_slot(p, c2, pi.U0, sd) + (size_t)row * kD + hc * 64 + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 f = __ldcg(src + i);
+                  acc[4 * i] += w * f.x;
+                  acc[4 * i + 1] += w * f.y;
+                  acc[4 * i + 2] += w * f.z;
+                  acc[4 * i + 3] += w * f.w;
+                }
+              }
+            }
+            if (qrow < p.Mq) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16(acc[2 * i] * inv_l, acc[2 * i + 1] * inv_l);
+              uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+          if (p.lse != nullptr && hc == 0 && qrow < p.Mq)
+            p.lse[((size_t)pi.r * p.H + pi.h) * p.Mq + qrow] =
+                (M + log2f(L)) * 0.69314718055994530942f;
+        }
+      }
+      // O may now be overwritten by the next piece
+      tc_fence_before();
+      mbar_arrive(&sh->o_empty);
+      g += n;
     }
     teardown(warp, tmem);
     return;
@@ -638,9 +1077,9 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                         (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
   const size_t smem = kSmemFixed + tab;
   if (smem > kSmemMax) return cudaErrorNotSupported;
-  dim3 grid((p.Mq + 2 * kBM - 1) / (2 * kBM), p.H, p.n_rollouts);
-  attn_bf16_d128_sm100<<<grid, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc,
-                                                          tm_kb, tm_vb, p);
+  if (p.G < 1 || p.G > kAttnMaxCtas) return cudaErrorInvalidValue;
+  attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb,
+                                                   tm_vb, p);
   count_launch(1);
   return cudaGetLastError();
 }

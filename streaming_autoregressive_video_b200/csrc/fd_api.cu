@@ -21,6 +21,7 @@ struct fd_cache {
   fd_cache_layout layout;
   fd::CacheView view;
   int device;
+  int sms;                      // multiprocessors of the device
   std::vector<int64_t> host_n;  // [L][R] mirror of the device counters
   CUtensorMap tm_kc, tm_vc;     // bf16 caches: (d, H, slots*Tf, L*R)
   CUtensorMap tm_kb;            // rotated block keys: (d, H, F*Tf, L*R)
@@ -88,6 +89,18 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   size_t blk;
   if (!mul_ok(frame * d->block_frames, lr, &blk)) return FD_ERR_CAPACITY;
   off = align_up(off + blk);
+  // partial results and arrival counters of the persistent bf16 kernel
+  const bool tensor_path = d->dtype == FD_BF16;
+  const size_t pairs = (T * d->block_frames + 255) / 256;
+  lay->part = off;
+  if (tensor_path)
+    off = align_up(off + (size_t)d->num_layers * kAttnMaxCtas * 2 * kPartSlotFloats *
+                             sizeof(float));
+  lay->cnt = off;
+  if (tensor_path) {
+    if (!mul_ok(lr * d->num_heads, pairs * sizeof(int32_t), &x)) return FD_ERR_CAPACITY;
+    off = align_up(off + x);
+  }
   lay->pos = off;
   off = align_up(off + lr * slots * sizeof(int32_t));
   lay->count = off;
@@ -204,12 +217,20 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   c->desc = *desc;
   c->layout = lay;
   c->device = attr.device;
+  if (cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->device) !=
+          cudaSuccess ||
+      c->sms < 1) {
+    delete c;
+    return FD_ERR_CUDA;
+  }
   uint8_t* base = static_cast<uint8_t*>(dev_storage);
   fd::CacheView& v = c->view;
   v.k = base + lay.k;
   v.v = base + lay.v;
   v.krot = base + lay.krot;
   v.kblk = base + lay.kblk;
+  v.part = reinterpret_cast<float*>(base + lay.part);
+  v.cnt = reinterpret_cast<int32_t*>(base + lay.cnt);
   v.pos = reinterpret_cast<int32_t*>(base + lay.pos);
   v.count = reinterpret_cast<int32_t*>(base + lay.count);
   v.ttab = reinterpret_cast<float2*>(base + lay.ttab);
@@ -228,6 +249,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.S = desc->sink_frames;
   v.W = desc->window_frames;
   v.slots = v.S + v.W;
+  v.nb = (v.F * v.T + 255) / 256;
   v.pt = lay.rope_pairs_t;
   v.ph = lay.rope_pairs_h;
   v.pw = lay.rope_pairs_w;
@@ -377,6 +399,9 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.err = c.err;
   p.kc = c.krot + (size_t)layer * cache->layout.layer_kv_bytes;
   p.vc = c.v + (size_t)layer * cache->layout.layer_kv_bytes;
+  p.part = c.part + (size_t)layer * fd::kAttnMaxCtas * 2 * fd::kPartSlotFloats;
+  p.cnt = c.cnt + (size_t)layer * c.R * c.H * c.nb;
+  p.nb = c.nb;
   p.H = c.H;
   p.d = c.d;
   p.T = c.T;
@@ -417,6 +442,18 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   if (work != nullptr &&
       !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.H, kb_rows, n_rollouts))
     return FD_ERR_CUDA;
+  {
+    // persistent grid: one CTA per multiprocessor, no more CTAs than KV
+    // iterations the call can have (every rollout's cache full)
+    const int64_t nt_max = ((int64_t)c.slots * c.Tf + 127) / 128 +
+                           ((int64_t)c.F * c.Tf + 127) / 128;
+    const int64_t it_max = (int64_t)n_rollouts * c.H * c.nb * nt_max;
+    int64_t g = cache->sms < fd::kAttnMaxCtas ? cache->sms : fd::kAttnMaxCtas;
+    if (it_max < g) g = it_max;
+    // the kernel's schedule arithmetic is 32-bit
+    if (it_max * g >= ((int64_t)1 << 31)) return FD_ERR_UNSUPPORTED;
+    p.G = (int)g;
+  }
   return fd::cuda_status(fd::launch_attn_bf16_sm100(
       tm_q, cache->tm_kc, cache->tm_vc, work != nullptr ? tm_kb_work : cache->tm_kb,
       tm_vb, p, s));
@@ -485,6 +522,10 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code) {
   *code = v;
   if (v != 0) {
     if (cudaMemset(cache->view.err, 0, sizeof(int32_t)) != cudaSuccess) return FD_ERR_CUDA;
+    // a kernel that gave up may have left split-unit arrival counters set
+    const size_t cnt_bytes = cache->layout.pos - cache->layout.cnt;
+    if (cnt_bytes > 0 && cudaMemset(cache->view.cnt, 0, cnt_bytes) != cudaSuccess)
+      return FD_ERR_CUDA;
     return FD_ERR_DEVICE_TIMEOUT;
   }
   return FD_OK;

@@ -41,11 +41,19 @@ struct CacheView {
   float2* ttab;
   float2* htab;
   float2* wtab;
+  float* part;    // [L][kAttnMaxCtas][2][kPartSlotFloats] (bf16 caches)
+  int32_t* cnt;   // [L][R][H][nb] (bf16 caches)
   int32_t* err;
-  int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz;
+  int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz, nb;
   double theta;
   uint64_t frame_bytes;  // Tf * H * d * esz
 };
+
+// Persistent tensor-core attention: at most this many CTAs, each with two
+// partial-result slots of kPartSlotFloats floats (O [256][128], m [256],
+// l [256]) per layer.
+constexpr int kAttnMaxCtas = 148;
+constexpr size_t kPartSlotFloats = 256 * 128 + 2 * 256;
 
 // Limits of one commit launch (host splits larger requests).
 constexpr int kCommitMaxLayers = 32;
@@ -82,7 +90,11 @@ struct AttnParams {
   int32_t* err;
   const uint8_t* kc;     // rotated cache K of the layer, rollout 0 (CUDA cores)
   const uint8_t* vc;
+  float* part;           // per-CTA partial results of split units (tensor path)
+  int32_t* cnt;          // per-unit arrival counters of split units
   int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
+  int nb;                // query-tile pairs per (rollout, head)
+  int G;                 // CTAs of the persistent launch
   int map_row0;          // layer * R: row offset of this layer in the cache maps
   int kb_row0;           // batch offset of rollout 0 in the rotated-block-key map
   FastDiv div_T, div_Tf, div_gw;

@@ -36,10 +36,19 @@ def test_cache_bytes_and_layout():
         esz = 2 if w.dtype == "bf16" else 4
         kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.heads * w.head_dim * esz
         assert lay.layer_kv_bytes * w.layers == kv
-        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.pos, lay.count, lay.ttab, lay.htab, lay.wtab,
-                   lay.err]
+        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.part, lay.cnt, lay.pos, lay.count,
+                   lay.ttab, lay.htab, lay.wtab, lay.err]
         assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
         assert lay.v - lay.k >= kv and lay.krot - lay.v >= kv and lay.kblk - lay.krot >= kv
+        blk = w.layers * w.rollouts * w.block_frames * w.frame_tokens * w.heads * w.head_dim * esz
+        assert lay.part - lay.kblk >= blk
+        # partial results of split query-tile pairs: 148 CTAs x 2 slots per
+        # layer, fp32 O [256][128] + max + sum; none for fp32 caches
+        part = w.layers * 148 * 2 * (256 * 128 + 512) * 4 if w.dtype == "bf16" else 0
+        assert part <= lay.cnt - lay.part < part + 1024
+        pairs = -(-w.block_frames * w.tokens // 256)
+        cnt = w.layers * w.rollouts * w.heads * pairs * 4 if w.dtype == "bf16" else 0
+        assert cnt <= lay.pos - lay.cnt < cnt + 1024
         assert (lay.rope_pairs_t, lay.rope_pairs_h, lay.rope_pairs_w) == \
             (w.head_dim // 2 - 2 * (w.head_dim // 6), w.head_dim // 6, w.head_dim // 6)
 
@@ -48,7 +57,9 @@ def test_single_480p_cache_is_about_3_gb():
     n = fd.fd_cache_bytes(fd.make_desc(SINGLE_480P))
     # 30 layers x 7 slots x 1560 tokens x 12 heads x 128 x 2 B x (K, V, rotated K)
     # + the per-layer work area for the block's rotated keys (3 frames)
-    assert abs(n - 30 * (7 * 3 + 3) * 1560 * 12 * 128 * 2) < 1 << 20
+    # + the per-layer partial-result slots of the attention kernel
+    part = 30 * 148 * 2 * (256 * 128 + 512) * 4
+    assert abs(n - 30 * (7 * 3 + 3) * 1560 * 12 * 128 * 2 - part) < 1 << 20
 
 
 @pytest.mark.parametrize("field,value,status", [
