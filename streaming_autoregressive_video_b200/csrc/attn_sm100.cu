@@ -40,11 +40,10 @@
 //   warps 4-7     RoPE: rotate each piece's Q tiles in place in the swizzled
 //                 shared-memory layout, cos/sin from the cache's tables
 //                 (fp64-accurate angles rounded once to fp32).
-//   warps 8-15    softmax on one tile at a time, two threads per query row
-//                 (TMEM lane), 64 columns each: row max (halves exchanged
-//                 through shared memory), exp2, row sum, P rounded to bf16
-//                 and written back into the S columns of TMEM as the A
-//                 operand of the PV product; the
+//   warps 8-15    softmax: warpgroup x owns query tile x, one thread per
+//                 query row (TMEM lane), all 128 columns: row max, exp2, row
+//                 sum, P rounded to bf16 and written back into the S columns
+//                 of TMEM as the A operand of the PV product; the
 //                 O rescale is skipped unless the running max grows by more
 //                 than 2^8, which keeps P <= 256 and the result exact up to
 //                 rounding.  The epilogue divides by the row sum and writes
@@ -80,7 +79,11 @@ constexpr uint32_t kOffK = 2 * kTile;
 constexpr uint32_t kOffV = kOffK + kKStages * kTile;
 constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
-constexpr int kPolyEvery = 2;  // every 2nd pair of exponentials on the FMA pipe
+// Every kPolyEvery-th pair of exponentials on the FMA pipe (0: all on MUFU).
+// With one warpgroup per query tile the MUFU unit is not the limit and the
+// polynomial's extra instructions cost more than they save (measured: 505 us
+// per 480p call all on MUFU, 521 us with every second pair on the FMA pipe).
+constexpr int kPolyEvery = 0;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
 
@@ -95,7 +98,6 @@ struct Shared {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
-  uint64_t red_bar[2][4];  // per tile and lane quarter: row halves exchange
   uint64_t o_full, o_empty, drain;
   uint64_t tab_bar;   // RoPE warpgroup: tables of the next rollout staged
   uint64_t part_bar;  // softmax: a piece's partial rows written
@@ -106,8 +108,7 @@ struct Shared {
 };
 
 // RoPE tables follow the barriers; the dynamic size adds them per launch.
-constexpr uint32_t kOffRed = kOffShared + 256;   // [2 buffers][2][2][128] floats
-constexpr uint32_t kOffMeta = kOffRed + 2 * 2 * 2 * 128 * 4;  // struct Meta
+constexpr uint32_t kOffMeta = kOffShared + 256;  // struct Meta
 constexpr uint32_t kOffTab = kOffMeta + 256;
 static_assert(sizeof(Shared) <= 256, "barrier block");
 constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
@@ -474,8 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sh->s_full[x], 1);
-      mbar_init(&sh->p_full[x], 256);
-      for (int q = 0; q < 4; ++q) mbar_init(&sh->red_bar[x][q], 64);
+      mbar_init(&sh->p_full[x], 128);
     }
     mbar_init(&sh->o_full, 1);
     mbar_init(&sh->o_empty, 256);
@@ -752,41 +752,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_inc<176>();
     // ------------------------------------------------------------ softmax
-    // All eight softmax warps work on one query tile at a time, alternating
-    // between the two tiles so that one tile's softmax overlaps the other
-    // tile's matrix products.  Warps 8+q and 12+q share TMEM lanes 32q..32q+31
-    // (query rows): warp 8+q takes S columns 0-63 of each row and warp 12+q
-    // columns 64-127.  The halves of a row exchange partial maxima (and, at
-    // the end, partial sums) through shared memory, synchronised by a bounded
-    // mbarrier of the 64 threads that own those rows.
-    const int hc = (warp - 8) >> 2;    // column half
+    // Warpgroup x (warps 8-11: x = 0, warps 12-15: x = 1) owns query tile x:
+    // one thread per query row (TMEM lane), all 128 columns, so no row data
+    // is exchanged.  The MMA ping-pong keeps the two warpgroups half a period
+    // apart: while one waits for its S tile or TMEM traffic, the other
+    // computes on the same SMSPs.
+    const int x = (warp - 8) >> 2;     // tile of this warpgroup
     const int wq = warp & 3;           // lane quarter
-    const int row_t = wq * 32 + lane;  // row within a tile
+    const int row_t = wq * 32 + lane;  // row within the tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [buf][tile][half][row]
+    const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
+    const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
     const float sl2 = p.scale_log2;
     int g = 0;
-    uint32_t ex_n = 0, n_part = 0;
+    uint32_t n_part = 0;
     bool ok = true;
-    uint32_t s[64];
-    // exchange a per-row value with the other column half; bounded wait.
-    // Exchange rounds alternate between two buffers, so a round's write
-    // never meets the partner's read of the round before.
-    auto exchange = [&](int x, float mine) -> float {
-      float* rb = red + (ex_n & 1) * (2 * 2 * kBM);
-      rb[(x * 2 + hc) * kBM + row_t] = mine;
-      mbar_arrive(&sh->red_bar[x][wq]);
-      ok = __all_sync(0xffffffffu, ok && wait_bar<true>(&sh->red_bar[x][wq], ex_n & 1,
-                                                        sh, p.err, kSiteSoftmax));
-      return rb[(x * 2 + (1 - hc)) * kBM + row_t];
-    };
+    uint32_t sa[64], sb[64];
     for (int k = 0; k < n_pieces && ok; ++k) {
       int n, kv0, nt1, n1, n2;
       {
-        // the piece's first S product is done, so its ring entry is out
+        // the piece's first S product of this tile is done, so its ring
+        // entry is out
         PieceInfo pi;
         ok = __all_sync(0xffffffffu,
-                        wait_bar<true>(&sh->s_full[0], g & 1, sh, p.err, kSiteSoftmax) &&
+                        wait_bar<true>(&sh->s_full[x], g & 1, sh, p.err, kSiteSoftmax) &&
                             read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
         if (!ok) break;
         n = pi.kv1 - pi.kv0;
@@ -795,111 +784,112 @@ __global__ void __launch_bounds__(kThreads, 1)
         n1 = pi.n1;
         n2 = pi.n2;
       }
-      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      float m = -INFINITY, l = 0.f;
       for (int jj = 0; jj < n && ok; ++jj) {
         const int gj = g + jj;
         const int j = kv0 + jj;
         const int valid = j < nt1 ? min(kBN, n1 - j * kBN) : min(kBN, n2 - (j - nt1) * kBN);
+        ok = __all_sync(0xffffffffu, wait_bar<true>(&sh->s_full[x], gj & 1, sh, p.err,
+                                                    kSiteSoftmax));
+        if (!ok) break;
+        tc_fence_after();
+        tmem_ld64(tS, sa);
+        tmem_ld64(tS + 64, sb);
+        if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (!ok) break;
-          const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
-          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
-          ok = __all_sync(0xffffffffu, wait_bar<true>(&sh->s_full[x], gj & 1, sh,
-                                                      p.err, kSiteSoftmax));
-          if (!ok) break;
-          tc_fence_after();
-          tmem_ld64(tS + hc * 64, s);
-          if (valid < kBN) {  // last tile of a segment: keys past its end weigh 0
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (hc * 64 + i >= valid) s[i] = 0xFF800000u;
+          for (int i = 0; i < 64; ++i) {
+            if (i >= valid) sa[i] = 0xFF800000u;
+            if (64 + i >= valid) sb[i] = 0xFF800000u;
           }
-          float m8[8];
+        }
+        // row max: three-input max, eight independent chains, two new
+        // columns per step
+        auto col = [&](int c) {
+          return __uint_as_float(c < 64 ? sa[c] : sb[c - 64]);
+        };
+        float m8[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            m8[i] = fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 8]));
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(col(i), col(i + 8), col(i + 16));
 #pragma unroll
-          for (int i = 16; i < 64; i += 2)
-            m8[(i >> 1) & 7] = fmaxf(m8[(i >> 1) & 7],
-                                     fmaxf(__uint_as_float(s[i]), __uint_as_float(s[i + 1])));
-          const float pmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          // both halves of the row have loaded their S columns once this
-          // returns, so P may now overwrite them
-          const float omax = exchange(x, pmax);
-          if (!ok) break;
-          const float m_tile = fmaxf(pmax, omax) * sl2;
-          const bool need = m_tile > m[x] + kRescaleThreshold;
-          if (jj > 0 && __any_sync(0xffffffffu, need)) {
-            const float alpha = need ? ex2_approx(m[x] - m_tile) : 1.f;
+        for (int c = 24; c < 128; c += 2)
+          m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], col(c), col(c + 1));
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
+        const float m_tile = mx * sl2;
+        const bool need = m_tile > m + kRescaleThreshold;
+        if (jj > 0 && __any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m - m_tile) : 1.f;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r16[16];
-              tmem_ld16(tO + hc * 64 + c * 16, r16);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t r16[16];
+            tmem_ld16(tO + c * 16, r16);
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
-              tmem_st16(tO + hc * 64 + c * 16, r16);
-            }
-            tmem_wait_st();
-          }
-          if (need) {
-            l[x] = (jj > 0) ? l[x] * ex2_approx(m[x] - m_tile) : 0.f;
-            m[x] = m_tile;
-          }
-          // P = 2^(s * log2(e)/sqrt(d) - m), two columns per packed
-          // instruction.  In full tiles every kPolyEvery-th pair of
-          // exponentials runs on the FMA pipe (exp2_poly2) to share the load of
-          // the MUFU unit; partial tiles (masked columns at -inf) use MUFU
-          // throughout so masked weights are exactly 0.
-          const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m[x], -m[x]);
-          float ls = 0.f;
-          uint64_t ls2 = 0;  // two packed +0.0f
-          uint32_t pk[32];
-          auto exps = [&](bool full) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const uint64_t x2 = f2_fma(
-                  f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
-              float p0, p1;
-              if (full && (i % kPolyEvery) == kPolyEvery - 1) {
-                const uint64_t e2 = exp2_poly2(x2);
-                ls2 = f2_add(ls2, e2);
-                f2_unpack(e2, p0, p1);
-              } else {
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-                ls += p0 + p1;
-              }
-              pk[i] = pack_bf16(p0, p1);
-            }
-          };
-          if (valid == kBN) exps(true); else exps(false);
-          // bf16 P of columns hc*64.. goes to TMEM columns hc*32.. of the tile
-          tmem_st32(tS + hc * 32, pk);
-          {
-            float la, lb;
-            f2_unpack(ls2, la, lb);
-            l[x] += ls + (la + lb);
+            for (int i = 0; i < 16; ++i)
+              r16[i] = __float_as_uint(__uint_as_float(r16[i]) * alpha);
+            tmem_st16(tO + c * 16, r16);
           }
           tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&sh->p_full[x]);
         }
-        ++ex_n;
+        if (need) {
+          l = (jj > 0) ? l * ex2_approx(m - m_tile) : 0.f;
+          m = m_tile;
+        }
+        // P = 2^(s * log2(e)/sqrt(d) - m), two columns per packed
+        // instruction.  In full tiles every kPolyEvery-th pair of
+        // exponentials runs on the FMA pipe (exp2_poly2) to share the load of
+        // the MUFU unit; partial tiles (masked columns at -inf) use MUFU
+        // throughout so masked weights are exactly 0.  Row sums accumulate
+        // in packed pairs.
+        const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+        uint64_t ls2 = 0;  // two packed +0.0f
+        uint32_t pk[32];
+        auto exps = [&](const uint32_t* sv, bool full) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint64_t x2 = f2_fma(
+                f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
+            uint64_t e2;
+            constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
+            if (kPolyEvery > 0 && full && (i % kEvery) == kEvery - 1) {
+              e2 = exp2_poly2(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              e2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            ls2 = f2_add(ls2, e2);
+            float p0, p1;
+            f2_unpack(e2, p0, p1);
+            pk[i] = pack_bf16(p0, p1);
+          }
+        };
+        // bf16 P of columns 0-63 goes to TMEM columns 0-31, of columns
+        // 64-127 to columns 32-63.  S columns 64-127 are still intact after
+        // the first half is stored: they are loaded again rather than kept
+        // in registers through the first half (which would not fit).
+        if (valid == kBN) exps(sa, true); else exps(sa, false);
+        tmem_st32(tS, pk);
+        tmem_ld64(tS + 64, sb);
+        if (valid < kBN) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (64 + i >= valid) sb[i] = 0xFF800000u;
+        }
+        if (valid == kBN) exps(sb, true); else exps(sb, false);
+        tmem_st32(tS + 32, pk);
+        {
+          float la, lb;
+          f2_unpack(ls2, la, lb);
+          l += la + lb;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh->p_full[x]);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu,
                       wait_bar(&sh->o_full, k & 1, sh, p.err, kSiteSoftmax));
-      if (!ok) break;
-      float l_tot[2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) l_tot[x] = l[x] + exchange(x, l[x]);
-      ++ex_n;
       if (!ok) break;
       tc_fence_after();
       // the piece again, from its ring entry (not kept in registers above)
@@ -907,35 +897,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
       if (!ok) break;
       const Sched sd = meta->sd;
+      const int row = x * kBM + row_t;  // row within the pair
       const bool whole = pi.kv0 == 0 && pi.kv1 == pi.nt;
       bool write_rows = whole;
       // CTAs whose pieces make up the unit, folded in this fixed order (so
       // the rounding does not depend on which piece arrived last)
       int c_lo = blockIdx.x, c_hi = blockIdx.x;
       if (!whole) {
-        // hand this piece over: unnormalised rows, running max, row sum
+        // hand this piece over: unnormalised row, running max, row sum
         float* part = p.part + ((size_t)blockIdx.x * 2 +
                                 (pi.U0 + pi.kv0 == meta->my_begin ? 0 : 1)) * kPartSlotFloats;
+        uint32_t rr[32];
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
-          const int row = x * kBM + row_t;
-          uint32_t rr[32];
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tO + c * 32, rr);
+          float4* dst = reinterpret_cast<float4*>(part + (size_t)row * kD + c * 32);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(tO + hc * 64 + c * 32, rr);
-            float4* dst = reinterpret_cast<float4*>(part + (size_t)row * kD + hc * 64 + c * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
-                                   __uint_as_float(rr[4 * i + 2]),
-                                   __uint_as_float(rr[4 * i + 3]));
-          }
-          if (hc == 0) {
-            part[2 * kBM * kD + row] = m[x];
-            part[2 * kBM * kD + 2 * kBM + row] = l_tot[x];
-          }
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
+                                 __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3]));
         }
+        part[2 * kBM * kD + row] = m;
+        part[2 * kBM * kD + 2 * kBM + row] = l;
         __threadfence();
         mbar_arrive(&sh->part_bar);
         if (threadIdx.x == 256) {
@@ -970,75 +953,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (write_rows) {
-        // rows = sum over pieces i of O_i 2^(m_i - M) / sum of l_i 2^(m_i - M),
+        // row = sum over pieces i of O_i 2^(m_i - M) / sum of l_i 2^(m_i - M),
         // M the largest max; this CTA's own piece comes from TMEM
         constexpr size_t kOffM = 2 * kBM * kD, kOffL = kOffM + 2 * kBM;
+        const int qrow = pi.b * 2 * kBM + row;
+        auto skip = [&](int c) {
+          return c != (int)blockIdx.x && cta_begin(c, sd, p.G) == cta_begin(c + 1, sd, p.G);
+        };
+        auto max_of = [&](int c) {
+          return c == (int)blockIdx.x ? m : __ldcg(part_slot(p, c, pi.U0, sd) + kOffM + row);
+        };
+        float M = -INFINITY;
+        for (int c = c_lo; c <= c_hi; ++c)
+          if (!skip(c)) M = fmaxf(M, max_of(c));
+        auto weight = [&](float mc) { return mc == M ? 1.f : ex2_approx(mc - M); };
+        float L = 0.f;
+        for (int c = c_lo; c <= c_hi; ++c) {
+          if (skip(c)) continue;
+          const float lc = c == (int)blockIdx.x ? l
+                                                : __ldcg(part_slot(p, c, pi.U0, sd) + kOffL + row);
+          L += lc * weight(max_of(c));
+        }
+        const float inv_l = 1.f / L;
+        uint16_t* out = static_cast<uint16_t*>(p.out) +
+                        (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * kD;
+        uint32_t rr[32];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tO + c * 32, rr);
+          float acc[32];
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
-          const int row = x * kBM + row_t;
-          const int qrow = pi.b * 2 * kBM + row;
-          auto skip = [&](int c) {
-            return c != (int)blockIdx.x && cta_begin(c, sd, p.G) == cta_begin(c + 1, sd, p.G);
-          };
-          auto max_of = [&](int c) {
-            return c == (int)blockIdx.x ? m[x] : __ldcg(part_slot(p, c, pi.U0, sd) + kOffM + row);
-          };
-          float M = -INFINITY;
-          for (int c = c_lo; c <= c_hi; ++c)
-            if (!skip(c)) M = fmaxf(M, max_of(c));
-          auto weight = [&](float mc) { return mc == M ? 1.f : ex2_approx(mc - M); };
-          float L = 0.f;
-          for (int c = c_lo; c <= c_hi; ++c) {
-            if (skip(c)) continue;
-            const float lc = c == (int)blockIdx.x ? l_tot[x]
-                                                  : __ldcg(part_slot(p, c, pi.U0, sd) + kOffL + row);
-            L += lc * weight(max_of(c));
-          }
-          const float inv_l = 1.f / L;
-          uint16_t* out = static_cast<uint16_t*>(p.out) +
-                          (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * kD + hc * 64;
-          uint32_t rr[32];
+          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+          for (int c2 = c_lo; c2 <= c_hi; ++c2) {
+            if (skip(c2)) continue;
+            const float w = weight(max_of(c2));
+            if (c2 == (int)blockIdx.x) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(tO + hc * 64 + c * 32, rr);
-            float acc[32];
+              for (int i = 0; i < 32; ++i) acc[i] += w * __uint_as_float(rr[i]);
+            } else {
+              const float4* src = reinterpret_cast<const float4*>(
+                  part_slot(p, c2, pi.U0, sd) + (size_t)row * kD + c * 32);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-            for (int c2 = c_lo; c2 <= c_hi; ++c2) {
-              if (skip(c2)) continue;
-              const float w = weight(max_of(c2));
-              if (c2 == (int)blockIdx.x) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc[i] += w * __uint_as_float(rr[i]);
-              } else {
-                const float4* src = reinterpret_cast<const float4*>(
-                    part_slot(p, c2, pi.U0, sd) + (size_t)row * kD + hc * 64 + c * 32);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 f = __ldcg(src + i);
-                  acc[4 * i] += w * f.x;
-                  acc[4 * i + 1] += w * f.y;
-                  acc[4 * i + 2] += w * f.z;
-                  acc[4 * i + 3] += w * f.w;
-                }
+              for (int i = 0; i < 8; ++i) {
+                const float4 f = __ldcg(src + i);
+                acc[4 * i] += w * f.x;
+                acc[4 * i + 1] += w * f.y;
+                acc[4 * i + 2] += w * f.z;
+                acc[4 * i + 3] += w * f.w;
               }
             }
-            if (qrow < p.Mq) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16(acc[2 * i] * inv_l, acc[2 * i + 1] * inv_l);
-              uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-            }
           }
-          if (p.lse != nullptr && hc == 0 && qrow < p.Mq)
-            p.lse[((size_t)pi.r * p.H + pi.h) * p.Mq + qrow] =
-                (M + log2f(L)) * 0.69314718055994530942f;
+          if (qrow < p.Mq) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16(acc[2 * i] * inv_l, acc[2 * i + 1] * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
         }
+        if (p.lse != nullptr && qrow < p.Mq)
+          p.lse[((size_t)pi.r * p.H + pi.h) * p.Mq + qrow] =
+              (M + log2f(L)) * 0.69314718055994530942f;
       }
       // O may now be overwritten by the next piece
       tc_fence_before();

@@ -290,6 +290,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes).
+// max of three floats in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
