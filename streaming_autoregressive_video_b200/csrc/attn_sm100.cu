@@ -864,17 +864,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         // bf16 P of columns 0-63 goes to TMEM columns 0-31, of columns
-        // 64-127 to columns 32-63.  S columns 64-127 are still intact after
-        // the first half is stored: they are loaded again rather than kept
-        // in registers through the first half (which would not fit).
+        // 64-127 to columns 32-63 (S columns 64-127 are already in registers)
         if (valid == kBN) exps(sa, true); else exps(sa, false);
         tmem_st32(tS, pk);
-        tmem_ld64(tS + 64, sb);
-        if (valid < kBN) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (64 + i >= valid) sb[i] = 0xFF800000u;
-        }
         if (valid == kBN) exps(sb, true); else exps(sb, false);
         tmem_st32(tS + 32, pk);
         {
