@@ -186,6 +186,31 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
+# --------------------------------------------------------------------------
+# Replicas (N > 1): the host-side rank logic, tested with gloo on the CPU
+# --------------------------------------------------------------------------
+def replica_seed_base(rank):
+    """Each replica draws its own inputs (same shapes and distributions)."""
+    return 1000 * rank
+
+
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise max over ranks: the job lasts as long as its slowest rank.
+    Every rank calls this the same number of times, in the same order."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_rate(work_per_rank, world, ms_max):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time
+    (per second)."""
+    return work_per_rank * world / (ms_max * 1e-3)
+
+
 def cpu_baseline(w):
     heads = list(range(w.heads))
     call, flops = oracle_call_setup(w, heads)
@@ -250,7 +275,7 @@ def run_fd(args, w, rank, world, local_rank):
 
     qshape = (R, w.queries, H, d)
     kshape = (R, F * Tf, H, d)
-    base = 1000 * rank
+    base = replica_seed_base(rank)
     # prefill every layer until the window is full (steady state)
     pk = [gen(synth.seed_of(base, 1, l), kshape) for l in range(L)]
     pv = [gen(synth.seed_of(base, 2, l), kshape) for l in range(L)]
@@ -327,16 +352,13 @@ def run_fd(args, w, rank, world, local_rank):
     ms_step = e0.elapsed_time(e1) / args.steps
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
     commit_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
-    t = torch.tensor([ms_step, attn_ms, commit_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step, attn_ms, commit_ms = float(t[0]), float(t[1]), float(t[2])
+    ms_step, attn_ms, commit_ms = max_over_ranks([ms_step, attn_ms, commit_ms], world, dev)
     err = fd.fd_get_device_error(cache)
     assert err == 0, f"device error word {err:#x}"
 
     flops_step = flops_call * S * L
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
-    frames_per_s_layer = R * F * L * world / (ms_step * 1e-3)
+    value = job_rate(flops_step, world, ms_step) / 1e12
+    frames_per_s_layer = job_rate(R * F * L, world, ms_step)
 
     # ---------------- end to end through the C ABI with host buffers
     e2e = None
@@ -459,12 +481,8 @@ def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
     stream.wait_event(fin)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t[0])
-    return {"value": flops_step * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    ms = max_over_ranks([e0.elapsed_time(e1) / steps], world, dev)[0]
+    return {"value": job_rate(flops_step, world, ms) / 1e12, "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d_bytes // steps, "d2h_bytes_per_step": d2h_bytes // steps,
             "ms_per_step": ms}
 

@@ -1,0 +1,81 @@
+"""The N > 1 path of bench.py on the CPU: two ranks over gloo.
+
+The hot path has no exchange step (every (rollout, head) unit lives on one GPU),
+so N GPUs run N independent replicas; what the ranks share is host logic: every
+rank takes the same collective steps in the same order, the job time is the
+maximum over ranks, the job throughput counts the work of all ranks, each
+replica draws its own inputs, and only rank 0 prints (also for the reference
+arm, whose other ranks exit without work)."""
+import contextlib
+import io
+import json
+import os
+import socket
+import sys
+import types
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+WORLD = 2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+
+    import bench
+    from streaming_autoregressive_video_b200.workloads import Workload
+
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        res = {}
+        # rank-dependent local timings: every rank must see the slowest
+        res["max"] = bench.max_over_ranks([1.0 + rank, 5.0 - rank, 3.0], WORLD)
+        # a second reduction in the same order on every rank
+        res["max2"] = bench.max_over_ranks([10.0 * (rank + 1)], WORLD)
+        res["rate"] = bench.job_rate(100.0, WORLD, res["max"][0])
+        res["seed"] = bench.replica_seed_base(rank)
+        # the reference arm: rank 0 alone runs and prints, the others return
+        w = Workload("gloo-tiny", layers=1, rollouts=1, heads=2, head_dim=16, grid_h=3,
+                     grid_w=4, action_tokens=0, block_frames=1, sink_frames=1,
+                     window_frames=2, steps=1, blocks=1, dtype="bf16")
+        args = types.SimpleNamespace(steps=1, warmup=0, gpus=WORLD)
+        buf = io.StringIO()
+        with contextlib.redirect_stdout(buf):
+            bench.run_reference(args, w, rank)
+        res["printed"] = buf.getvalue()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump(res, f)
+
+
+def test_two_replicas_over_gloo(tmp_path):
+    mp.start_processes(_rank_main, args=(_free_port(), str(tmp_path)), nprocs=WORLD,
+                       join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(WORLD)]
+    for r in res:
+        assert r["max"] == [2.0, 5.0, 3.0]
+        assert r["max2"] == [20.0]
+        # 100 units per rank, 2 ranks, slowest rank 2 ms -> 1e5 units/s
+        assert r["rate"] == pytest.approx(100.0 * WORLD / 2e-3)
+    assert res[0]["seed"] != res[1]["seed"]
+    # only rank 0 prints the reference arm's JSON line
+    assert res[1]["printed"] == ""
+    line = json.loads(res[0]["printed"].strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == WORLD
+    assert line["value"] > 0 and line["unit"] == "TFLOP/s"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
