@@ -46,6 +46,12 @@ R7  the cache keeps K/V exactly as committed (before RoPE) plus one int32 frame
     applied to cached keys when they are used.
 R8  the block being denoised has frames n .. n+F-1; its K/V are committed after
     the last denoising step (whatever K/V the caller passes).
+R9  grouped-query attention (a variant of the cache semantics, not on the
+    pages): keys and values carry Hkv heads, queries H = G * Hkv heads, and
+    query head h reads key/value head h div G (consecutive query heads share
+    a key/value head, as in Ainslie et al., "GQA: Training Generalized
+    Multi-Query Transformer Models from Multi-Head Checkpoints", 2023).
+    Hkv = H is plain multi-head attention.
 """
 from __future__ import annotations
 
@@ -198,8 +204,9 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
                     return_probs: bool = False):
     """Attention of the current block's queries of one (rollout, layer).
 
-    q:    [F*T][H][d]  queries of the block, storage form, pre-RoPE
-    k, v: [F*Tf][H][d] keys / values of the block, storage form, pre-RoPE
+    q:    [F*T][H][d]    queries of the block, storage form, pre-RoPE
+    k, v: [F*Tf][Hkv][d] keys / values of the block, storage form, pre-RoPE
+          (Hkv divides H; query head h reads key/value head h div (H/Hkv))
     cache: the rollout's cache for this layer (not modified)
     heads: optional subset of head indices to evaluate (others are left 0)
     rows:  optional subset of query rows to evaluate (others are left 0);
@@ -215,6 +222,10 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     if F * T != Mq or k.shape[0] % F:
         raise ValueError("q rows must be F*T and k rows F*Tf")
     Tf = k.shape[0] // F
+    Hkv = k.shape[1]
+    if H % Hkv or cache.k.shape[2] != Hkv:
+        raise ValueError("key/value heads must divide the query heads and match the cache")
+    group = H // Hkv
     n = cache.n
     nv = cache.valid_slots()
 
@@ -237,11 +248,12 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     lse = np.zeros((H, Mq), dtype=np.float64)
     probs = {}
     for hh in (range(H) if heads is None else heads):
+        g = hh // group  # key/value head of this query head (R9)
         qh = rope_rotate(values_f64(q[rows, hh, :], dtype), ang_q)
-        kc = values_f64(cache.k[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
-        vc = values_f64(cache.v[:nv, :, hh, :], dtype).reshape(nv * Tf, d)
-        kh = rope_rotate(np.concatenate([kc, values_f64(k[:, hh, :], dtype)]), ang_k)
-        vh = np.concatenate([vc, values_f64(v[:, hh, :], dtype)])
+        kc = values_f64(cache.k[:nv, :, g, :], dtype).reshape(nv * Tf, d)
+        vc = values_f64(cache.v[:nv, :, g, :], dtype).reshape(nv * Tf, d)
+        kh = rope_rotate(np.concatenate([kc, values_f64(k[:, g, :], dtype)]), ang_k)
+        vh = np.concatenate([vc, values_f64(v[:, g, :], dtype)])
         if return_probs:
             probs[hh] = np.zeros((Mq, kh.shape[0]), dtype=np.float64)
         for c0 in range(0, len(rows), row_chunk):

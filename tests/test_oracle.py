@@ -366,3 +366,46 @@ def test_uniform_shift_of_all_positions_leaves_attention_unchanged():
     oa, _ = block_attention(a, q, k, v, tokens=T, grid_w=2, theta=1.0e4)
     ob, _ = block_attention(b, q, k, v, tokens=T, grid_w=2, theta=1.0e4)
     np.testing.assert_allclose(ob, oa, rtol=0, atol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# grouped-query attention (reading R9)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 1), (6, 3)])
+def test_grouped_query_attention_equals_repeated_key_value_heads(H, Hkv):
+    # GQA with Hkv key/value heads is multi-head attention on key/value heads
+    # repeated so that query heads h*G .. h*G+G-1 see key/value head h
+    # (np.repeat along the head axis, an independent statement of the map)
+    rng = np.random.default_rng(31)
+    S, W, F, T, d = 1, 3, 2, 6, 12
+    G = H // Hkv
+    gqa = RolloutCache(S, W, T, Hkv, d, "f32")
+    mha = RolloutCache(S, W, T, H, d, "f32")
+    for _ in range(4):
+        kf = rng.standard_normal((F, T, Hkv, d)).astype(np.float32)
+        vf = rng.standard_normal((F, T, Hkv, d)).astype(np.float32)
+        gqa.commit(kf, vf)
+        mha.commit(np.repeat(kf, G, axis=2), np.repeat(vf, G, axis=2))
+    q = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    k = rng.standard_normal((F * T, Hkv, d)).astype(np.float32)
+    v = rng.standard_normal((F * T, Hkv, d)).astype(np.float32)
+    og, lg = block_attention(gqa, q, k, v, tokens=T, grid_w=3, theta=1.0e4)
+    om, lm = block_attention(mha, q, np.repeat(k, G, axis=1), np.repeat(v, G, axis=1),
+                             tokens=T, grid_w=3, theta=1.0e4)
+    np.testing.assert_array_equal(og, om)
+    np.testing.assert_array_equal(lg, lm)
+    # and the map is not interleaved: with G > 1 the first two query heads
+    # share a key/value head (identical queries give identical rows)
+    if G > 1:
+        q2 = q.copy()
+        q2[:, 1] = q2[:, 0]
+        o2, _ = block_attention(gqa, q2, k, v, tokens=T, grid_w=3, theta=1.0e4)
+        np.testing.assert_array_equal(o2[:, 0], o2[:, 1])
+
+
+def test_grouped_query_attention_rejects_non_dividing_heads():
+    c = RolloutCache(0, 2, 4, 2, 12, "f32")
+    q = np.zeros((4, 3, 12), np.float32)
+    kv = np.zeros((4, 2, 12), np.float32)
+    with pytest.raises(ValueError):
+        block_attention(c, q, kv, kv, tokens=4, grid_w=2, theta=1.0e4)
