@@ -52,6 +52,13 @@ R9  grouped-query attention (a variant of the cache semantics, not on the
     a key/value head, as in Ainslie et al., "GQA: Training Generalized
     Multi-Query Transformer Models from Multi-Head Checkpoints", 2023).
     Hkv = H is plain multi-head attention.
+R10 multi-view frames (a shape variant; the pages show four-camera models
+    attending across views without saying how positions are assigned): a
+    frame holds V views of Gh x Gw video tokens, view-major, so T = V*Gh*Gw;
+    video token i sits at (h, w) of its position inside its view, i mod
+    (Gh*Gw), and all views of a frame share t.  Views therefore differ only by
+    content (any learned view embedding belongs to the model, before the
+    attention).  V = 1 is R5.
 """
 from __future__ import annotations
 
@@ -132,11 +139,14 @@ def rope_rotate(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
     return out
 
 
-def token_coords(n_tokens: int, T: int, grid_w: int):
-    """(h, w) of the tokens of one frame (R5): video tokens row-major, actions at 0."""
+def token_coords(n_tokens: int, T: int, grid_w: int, view_tokens: int = 0):
+    """(h, w) of the tokens of one frame (R5, R10): video tokens row-major
+    inside their view (view_tokens = Gh*Gw per view; 0 = a single view of T
+    tokens), actions at 0."""
     i = np.arange(n_tokens)
-    h = np.where(i < T, i // grid_w, 0)
-    w = np.where(i < T, i % grid_w, 0)
+    iv = i % (view_tokens or T)
+    h = np.where(i < T, iv // grid_w, 0)
+    w = np.where(i < T, iv % grid_w, 0)
     return h, w
 
 
@@ -201,7 +211,7 @@ class RolloutCache:
 # --------------------------------------------------------------------------
 def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
                     theta: float, heads=None, rows=None, row_chunk: int = 512,
-                    return_probs: bool = False):
+                    return_probs: bool = False, view_tokens: int = 0):
     """Attention of the current block's queries of one (rollout, layer).
 
     q:    [F*T][H][d]    queries of the block, storage form, pre-RoPE
@@ -211,6 +221,8 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     heads: optional subset of head indices to evaluate (others are left 0)
     rows:  optional subset of query rows to evaluate (others are left 0);
            every row's softmax still runs over the whole key set
+    view_tokens: video tokens per view of a multi-view frame (R10; 0 = one
+           view of all `tokens`)
 
     Returns (out [F*T][H][d] fp64, lse [H][F*T] fp64 natural-log sum of exp of
     the scaled scores) and, with return_probs, a dict head -> P [F*T][Nk].
@@ -230,7 +242,7 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     nv = cache.valid_slots()
 
     # coordinates of every key: valid cache slots in slot order, then the block
-    h_tok, w_tok = token_coords(Tf, T, grid_w)
+    h_tok, w_tok = token_coords(Tf, T, grid_w, view_tokens)
     t_cache = np.repeat(cache.pos[:nv].astype(np.float64), Tf)
     t_block = np.repeat(np.arange(n, n + F, dtype=np.float64), Tf)
     t_key = np.concatenate([t_cache, t_block])
@@ -240,7 +252,7 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
 
     # coordinates of the evaluated queries (video tokens only)
     rows = np.arange(Mq) if rows is None else np.asarray(rows, dtype=np.int64)
-    tok_q = rows % T
+    tok_q = (rows % T) % (view_tokens or T)
     ang_q = rope_angles(n + rows // T, tok_q // grid_w, tok_q % grid_w, d, theta)
 
     scale = 1.0 / math.sqrt(d)

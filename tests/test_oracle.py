@@ -409,3 +409,44 @@ def test_grouped_query_attention_rejects_non_dividing_heads():
     kv = np.zeros((4, 2, 12), np.float32)
     with pytest.raises(ValueError):
         block_attention(c, q, kv, kv, tokens=4, grid_w=2, theta=1.0e4)
+
+
+# --------------------------------------------------------------------------
+# multi-view frames (reading R10)
+# --------------------------------------------------------------------------
+def test_multiview_token_coords_repeat_per_view():
+    # 3 views of a 2 x 4 grid + 2 action tokens, enumerated by hand
+    gh, gw, V, A = 2, 4, 3, 2
+    h, w = token_coords(V * gh * gw + A, V * gh * gw, gw, gh * gw)
+    want_h = [0, 0, 0, 0, 1, 1, 1, 1] * V + [0] * A
+    want_w = [0, 1, 2, 3, 0, 1, 2, 3] * V + [0] * A
+    assert list(h) == want_h and list(w) == want_w
+
+
+def test_multiview_attention_is_equivariant_to_swapping_views():
+    # swapping two views in the cache, the block keys/values and the queries
+    # swaps the corresponding output rows: positions do not depend on the view
+    rng = np.random.default_rng(41)
+    S, W, F, gh, gw, V, A, H, d = 1, 2, 1, 2, 3, 2, 1, 2, 12
+    Tv = gh * gw
+    T, Tf = V * Tv, V * Tv + A
+    perm = np.concatenate([np.arange(Tv, 2 * Tv), np.arange(Tv), np.arange(2 * Tv, Tf)])
+    a = RolloutCache(S, W, Tf, H, d, "f32")
+    b = RolloutCache(S, W, Tf, H, d, "f32")
+    for _ in range(3):
+        kf = rng.standard_normal((F, Tf, H, d)).astype(np.float32)
+        vf = rng.standard_normal((F, Tf, H, d)).astype(np.float32)
+        a.commit(kf, vf)
+        b.commit(kf[:, perm], vf[:, perm])
+    q = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    k = rng.standard_normal((F * Tf, H, d)).astype(np.float32)
+    v = rng.standard_normal((F * Tf, H, d)).astype(np.float32)
+    oa, la = block_attention(a, q, k, v, tokens=T, grid_w=gw, theta=1.0e4, view_tokens=Tv)
+    ob, lb = block_attention(b, q[perm[:T]], k[perm], v[perm], tokens=T, grid_w=gw,
+                             theta=1.0e4, view_tokens=Tv)
+    np.testing.assert_allclose(ob, oa[perm[:T]], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lb, la[:, perm[:T]], rtol=0, atol=1e-12)
+    # with views read as extra grid rows the swap would change the result
+    oc, _ = block_attention(b, q[perm[:T]], k[perm], v[perm], tokens=T, grid_w=gw,
+                            theta=1.0e4)
+    assert np.abs(oc - oa[perm[:T]]).max() > 1e-3
