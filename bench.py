@@ -8,7 +8,7 @@ into every layer's ring buffer.  The cache is full (steady state) before the
 timed region, so every call attends to sinks + the whole window + the block.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference]
-                    [--workload 480p|large|long|ragged]
+                    [--workload 480p|large|long|ragged|multiview|gqa]
 
 N > 1 runs one independent replica per GPU (the path has no exchange step):
 value = work of all ranks / max-over-ranks time ("scaling": "weak").
@@ -41,7 +41,8 @@ KERNEL_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
 def workloads():
     from streaming_autoregressive_video_b200 import workloads as wl
     return {"480p": wl.SINGLE_480P, "large": wl.LARGE_ACTIONS,
-            "long": wl.LONG_ROLLOUT, "ragged": wl.BATCHED_RAGGED}
+            "long": wl.LONG_ROLLOUT, "ragged": wl.BATCHED_RAGGED,
+            "multiview": wl.MULTIVIEW_4, "gqa": wl.GQA_480P}
 
 
 def parse_args():
@@ -67,11 +68,13 @@ def attn_flops(w, nkeys_per_rollout):
 
 
 def attn_bytes(w, nkeys_per_rollout, esz=2):
-    """Q + block K/V + valid cache K/V read once + O written once."""
-    per_tok = w.heads * w.head_dim * esz
+    """Q + block K/V + valid cache K/V read once + O written once (queries and
+    outputs carry H heads, keys and values Hkv)."""
+    per_q = w.heads * w.head_dim * esz
+    per_kv = w.hkv * w.head_dim * esz
     b = 0
     for nk in nkeys_per_rollout:
-        b += 2 * w.queries * per_tok + 2 * nk * per_tok
+        b += 2 * w.queries * per_q + 2 * nk * per_kv
     return float(b)
 
 
@@ -160,21 +163,21 @@ class ClockSampler:
 def oracle_call_setup(w, heads):
     import oracle
     from streaming_autoregressive_video_b200 import synth
-    c = oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens, w.heads,
+    c = oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens, w.hkv,
                             w.head_dim, "bf16")
-    ks = (w.block_frames, w.frame_tokens, w.heads, w.head_dim)
+    ks = (w.block_frames, w.frame_tokens, w.hkv, w.head_dim)
     n_commits = -(-w.slots // w.block_frames) + 1
     for b in range(n_commits):
         c.commit(synth.normal(synth.seed_of(7, b, 0), ks, "bf16", w.value_scale),
                  synth.normal(synth.seed_of(7, b, 1), ks, "bf16", w.value_scale))
     q = synth.normal(synth.seed_of(7, 99, 0), (w.queries, w.heads, w.head_dim), "bf16", w.value_scale)
-    k = synth.normal(synth.seed_of(7, 99, 1), (w.block_frames * w.frame_tokens, w.heads, w.head_dim), "bf16", w.value_scale)
-    v = synth.normal(synth.seed_of(7, 99, 2), (w.block_frames * w.frame_tokens, w.heads, w.head_dim), "bf16", w.value_scale)
+    k = synth.normal(synth.seed_of(7, 99, 1), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), "bf16", w.value_scale)
+    v = synth.normal(synth.seed_of(7, 99, 2), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), "bf16", w.value_scale)
     nk = (c.valid_slots() + w.block_frames) * w.frame_tokens
 
     def call():
         oracle.block_attention(c, q, k, v, tokens=w.tokens, grid_w=w.grid_w,
-                               theta=w.theta, heads=heads)
+                               theta=w.theta, heads=heads, view_tokens=w.view_tokens)
     return call, 4.0 * len(heads) * w.head_dim * w.queries * nk
 
 
@@ -274,7 +277,7 @@ def run_fd(args, w, rank, world, local_rank):
         return synth.normal_device(seed, shape, "bf16", dev, w.value_scale).view(torch.int16)
 
     qshape = (R, w.queries, H, d)
-    kshape = (R, F * Tf, H, d)
+    kshape = (R, F * Tf, w.hkv, d)
     base = replica_seed_base(rank)
     # prefill every layer until the window is full (steady state)
     pk = [gen(synth.seed_of(base, 1, l), kshape) for l in range(L)]

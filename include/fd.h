@@ -74,14 +74,20 @@ typedef enum {
 
 typedef enum { FD_BF16 = 0, FD_F32 = 1 } fd_dtype;
 
-/* Geometry of one cache.  T = grid_h*grid_w video tokens per latent frame;
+/* Geometry of one cache.  T = views*grid_h*grid_w video tokens per latent
+ * frame (views of one frame side by side, view-major; a single view when
+ * num_views is 0 or 1);
  * Tf = T + action_tokens key/value tokens per frame ([C3-MA]: 4 action
  * vectors per latent frame).  Requires 1 <= block_frames <= window_frames,
- * sink_frames >= 0, head_dim even and a multiple of 8. */
+ * sink_frames >= 0, head_dim even and a multiple of 8.
+ * Grouped-query attention (no counterpart on the pages; a variant of the
+ * cache semantics): keys and values carry Hkv = num_kv_heads heads, queries
+ * and outputs H = num_heads; Hkv divides H and query head h reads key/value
+ * head h / (H / Hkv).  num_kv_heads = 0 means Hkv = H (multi-head). */
 typedef struct {
   int32_t num_layers;     /* L: one independent cache per layer            */
   int32_t max_rollouts;   /* R: concurrent rollouts, each with its own cache */
-  int32_t num_heads;      /* H (query heads = key/value heads)             */
+  int32_t num_heads;      /* H query heads                                 */
   int32_t head_dim;       /* d                                             */
   int32_t grid_h;         /* latent grid height                            */
   int32_t grid_w;         /* latent grid width                             */
@@ -91,16 +97,21 @@ typedef struct {
   int32_t window_frames;  /* W rolling window frames                       */
   float rope_theta;       /* RoPE base (1e4 in every shipped workload)     */
   int32_t dtype;          /* fd_dtype of q, k, v, out and the cache        */
+  int32_t num_kv_heads;   /* Hkv key/value heads (0: = num_heads)          */
+  int32_t num_views;      /* V camera views per frame (0: = 1); video
+                           * token i sits at (h, w) of i mod (grid_h*grid_w)
+                           * and all views share t (no counterpart on the
+                           * pages beyond their four-view models)           */
 } fd_cache_desc;
 
 /* Byte offsets of the regions inside the caller's storage buffer.
- *   k, v : [L][R][S+W][Tf][H][d] elements of `dtype`, exactly as committed
- *   krot : [L][R][S+W][Tf][H][d] the same keys rotated by 3D RoPE to their
+ *   k, v : [L][R][S+W][Tf][Hkv][d] elements of `dtype`, exactly as committed
+ *   krot : [L][R][S+W][Tf][Hkv][d] the same keys rotated by 3D RoPE to their
  *          frame's position, written by the commit (a committed frame and its
  *          position never change, so its rotation is computed once instead
  *          of at every attention call); derived data, not part of the
  *          cache's observable state
- *   kblk : [L][R][F*Tf][H][d] work area of fd_block_attention: the current
+ *   kblk : [L][R][F*Tf][Hkv][d] work area of fd_block_attention: the current
  *          block's keys rotated once per call, read by every query tile
  *          (one region per layer, so calls on different layers may run
  *          concurrently; calls on the same layer must be ordered)
@@ -157,18 +168,20 @@ fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
                          int32_t n_ids, void* stream);
 
 /* 3D RoPE in place on a block tensor x of rollouts 0..n_rollouts-1:
- *   x: [n_rollouts][F][tokens_per_frame][H][d] of the cache dtype;
+ *   x: [n_rollouts][F][tokens_per_frame][heads][d] of the cache dtype;
  *   tokens_per_frame = T (queries) or Tf (keys, action tokens at (t,0,0));
+ *   heads = num_heads (queries) or Hkv (keys); anything else FD_ERR_SHAPE;
  * frame f of rollout r is at t = n_r + f with n_r that rollout's counter at
  * `layer`, i.e. the positions fd_block_attention gives the block.  This is the
  * same rotation fd_block_attention applies internally; it is exported for
  * callers that need rotated tensors and for tests. */
 fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
-                    void* x, int32_t tokens_per_frame, void* stream);
+                    void* x, int32_t tokens_per_frame, int32_t heads,
+                    void* stream);
 
 /* One denoising-step attention call for `layer` ([C3-MA], [AD-VII]):
  *   q   : [n_rollouts][F*T][H][d]   queries of the block, pre-RoPE
- *   k, v: [n_rollouts][F*Tf][H][d]  keys/values of the block, pre-RoPE
+ *   k, v: [n_rollouts][F*Tf][Hkv][d] keys/values of the block, pre-RoPE
  *   out : [n_rollouts][F*T][H][d]   softmax(q'k'^T/sqrt(d)) v
  *   lse : [n_rollouts][H][F*T] fp32 natural-log sum of exp of the scaled
  *         scores, or NULL
@@ -221,7 +234,7 @@ fd_status fd_block_attention_static(fd_cache* cache, int32_t layer,
  *   frames (host) [n_rollouts], each in [0, F]; NULL = F for every rollout
  *   (a ragged prefill commits fewer frames for some rollouts);
  *   k, v (host arrays of device pointers) [layer_end - layer_begin], each
- *   [n_rollouts][F*Tf][H][d] pre-RoPE (in practice the last step's k/v). */
+ *   [n_rollouts][F*Tf][Hkv][d] pre-RoPE (in practice the last step's k/v). */
 fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,
                           int32_t layer_end, int32_t n_rollouts,
                           const int32_t* frames, const void* const* k,

@@ -41,7 +41,8 @@ class CacheDesc(ctypes.Structure):
                 ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
                 ("action_tokens", ctypes.c_int32), ("block_frames", ctypes.c_int32),
                 ("sink_frames", ctypes.c_int32), ("window_frames", ctypes.c_int32),
-                ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32)]
+                ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("num_views", ctypes.c_int32)]
 
 
 class CacheLayout(ctypes.Structure):
@@ -80,7 +81,7 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
     lib.fd_cache_get_desc.argtypes = [vp, ctypes.POINTER(CacheDesc)]
     lib.fd_cache_layout_of.argtypes = [vp, ctypes.POINTER(CacheLayout)]
     lib.fd_cache_reset.argtypes = [vp, ctypes.POINTER(i32), i32, vp]
-    lib.fd_rope3d.argtypes = [vp, i32, i32, vp, i32, vp]
+    lib.fd_rope3d.argtypes = [vp, i32, i32, vp, i32, i32, vp]
     lib.fd_block_attention.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.fd_block_attention_static.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.fd_cache_commit.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32),
@@ -128,7 +129,8 @@ def make_desc(w, dtype: Optional[str] = None) -> CacheDesc:
     dt = dtype or w.dtype
     return CacheDesc(w.layers, w.rollouts, w.heads, w.head_dim, w.grid_h, w.grid_w,
                      w.action_tokens, w.block_frames, w.sink_frames, w.window_frames,
-                     float(w.theta), FD_BF16 if dt == "bf16" else FD_F32)
+                     float(w.theta), FD_BF16 if dt == "bf16" else FD_F32,
+                     getattr(w, "kv_heads", 0), getattr(w, "views", 1))
 
 
 def fd_cache_bytes(desc: CacheDesc) -> int:
@@ -187,9 +189,9 @@ def fd_cache_reset(cache: Cache, rollout_ids: Sequence[int], stream=None) -> Non
 
 
 def fd_rope3d(cache: Cache, layer: int, n_rollouts: int, x, tokens_per_frame: int,
-              stream=None) -> None:
+              heads: int, stream=None) -> None:
     _check(load().fd_rope3d(cache.handle, layer, n_rollouts, _ptr(x), tokens_per_frame,
-                            _stream(stream)), "fd_rope3d")
+                            heads, _stream(stream)), "fd_rope3d")
 
 
 def fd_block_attention(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int q = q0 + row;
     float a = 0.f, b = 0.f;
     if (q < p.Mq) {
-      const int f = q / p.T, tok = q - f * p.T;
+      const int f = q / p.T, tok = (q - f * p.T) % p.Tv;  // inside its view
       const KeyCoord kc{p.slots + f, tok / p.gw, tok % p.gw};
       const float* src = qg + (((size_t)r * p.Mq + q) * p.H + h) * D + 2 * pair;
       const float2 cs = rope_cs(p, tt, pair, kc);
@@ -100,9 +100,11 @@ __global__ void __launch_bounds__(kWarps * 32)
       const int key = key0 + kr;
       float a = 0.f, b = 0.f, va = 0.f, vb = 0.f;
       if (key < nseg) {
+        // key/value head of this query head (grouped-query attention)
+        const int hk = h / p.kv_group;
         const size_t off = seg1
-            ? (((size_t)r * p.slots * p.Tf + key) * p.H + h) * D + 2 * pair
-            : (((size_t)r * p.F * p.Tf + key) * p.H + h) * D + 2 * pair;
+            ? (((size_t)r * p.slots * p.Tf + key) * p.Hkv + hk) * D + 2 * pair
+            : (((size_t)r * p.F * p.Tf + key) * p.Hkv + hk) * D + 2 * pair;
         // keys arrive rotated: cached frames were rotated when committed, the
         // block's keys once per call before this kernel
         const float* ks = (seg1 ? kcg : kg) + off;

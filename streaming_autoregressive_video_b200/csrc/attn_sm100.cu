@@ -374,7 +374,8 @@ __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
     const int q = qrow0 + row;
     if (q >= p.Mq) continue;
     const int f = (int)fast_div((uint32_t)q, p.div_T);
-    const int tok = q - f * p.T;
+    const int tq = q - f * p.T;
+    const int tok = tq - (int)fast_div((uint32_t)tq, p.div_Tv) * p.Tv;  // inside its view
     const int hh = (int)fast_div((uint32_t)tok, p.div_gw);
     rotate_chunk(tile, row, rl, tab, p.slots + f, hh, tok - hh * p.gw);
   }
@@ -561,7 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued_q = k + 1;
         // keys: rotated cache keys or the block keys rotated for this call,
         // both batched by (layer, rollout); values: cache (layer, rollout)
-        // or the caller's block values (rollout)
+        // or the caller's block values (rollout); head: the query head's
+        // key/value head (grouped-query attention)
+        const int hkv = pc.h / p.kv_group;
         for (int j = pc.kv0; j < pc.kv1; ++j, ++g) {
           const bool seg1 = j < pc.tc.nt1;
           const int key0 = seg1 ? j * kBN : (j - pc.tc.nt1) * kBN;
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
-                        &sh->k_full[ks], hf * 64, pc.h, key0, ck3);
+                        &sh->k_full[ks], hf * 64, hkv, key0, ck3);
           issued_k = g + 1;
           const int vs = g % kVStages;
           if (g >= kVStages &&
@@ -591,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
-                        &sh->v_full[vs], hf * 64, pc.h, key0, cv3);
+                        &sh->v_full[vs], hf * 64, hkv, key0, cv3);
           issued_v = g + 1;
         }
       }

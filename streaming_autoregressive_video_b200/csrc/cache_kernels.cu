@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kCopyThreads)
   uint4* rdst = reinterpret_cast<uint4*>(c.krot + dst_off);
   const float2* tt_row = c.ttab + (lr * (c.slots + c.F) + c.slots + f) * c.pt;
   const uint32_t vec_per_row = c.d / kPer;
-  const uint32_t vec_per_tok = vec_per_row * c.H;
+  const uint32_t vec_per_tok = vec_per_row * c.Hkv;
 #pragma unroll
   for (int i = 0; i < kCopyVecs; ++i) {
     const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
@@ -168,8 +168,9 @@ __global__ void __launch_bounds__(kCopyThreads)
     const int pair0 = (int)(vi % vec_per_row) * (kPer / 2);
     int hh = 0, ww = 0;
     if ((int)tok < c.T) {
-      hh = (int)tok / c.gw;
-      ww = (int)tok - hh * c.gw;
+      const int tv = (int)tok % c.Tv;  // position inside the token's view
+      hh = tv / c.gw;
+      ww = tv - hh * c.gw;
     }
     rdst[vi] = rotate16<Elem>(buf[i], pair0, c, tt_row, hh, ww);
   }
@@ -226,16 +227,16 @@ __global__ void reset_meta_kernel(CacheView c, ResetParams p) {
   fill_ttab(c, l, r, 0, pos);
 }
 
-// 3D RoPE of a block tensor [R][F][Tx][H][d]: token row i of rollout r and
+// 3D RoPE of a block tensor [R][F][Tx][heads][d]: token row i of rollout r and
 // frame f sits at t = n_r + f (t-row slots + f of the rollout's table).  One
 // warp per token row; out may equal in (in place).
 template <typename Elem>
 __global__ void __launch_bounds__(256)
     rope3d_kernel(CacheView c, int layer, int n_rollouts, const Elem* in,
-                  Elem* out, int Tx) {
+                  Elem* out, int Tx, int heads) {
   constexpr int kPer = 16 / sizeof(Elem);  // elements per 16-byte chunk
   const uint32_t cpr = c.d / kPer;         // chunks per head row
-  const uint32_t row_chunks = cpr * c.H;   // chunks per token row
+  const uint32_t row_chunks = cpr * heads;  // chunks per token row
   const uint32_t rows = (uint32_t)n_rollouts * c.F * Tx;
   const uint32_t warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -247,8 +248,9 @@ __global__ void __launch_bounds__(256)
     const int tok = (int)(rem - f * Tx);
     const float2* tt = c.ttab + (((size_t)layer * c.R + r) * (c.slots + c.F) +
                                  c.slots + f) * c.pt;
-    const int hh = tok < c.T ? tok / c.gw : 0;
-    const int ww = tok < c.T ? tok - hh * c.gw : 0;
+    const int tv = tok % c.Tv;  // position inside the token's view
+    const int hh = tok < c.T ? tv / c.gw : 0;
+    const int ww = tok < c.T ? tv - hh * c.gw : 0;
     const uint4* src = reinterpret_cast<const uint4*>(in) + (size_t)row * row_chunks;
     uint4* dst = reinterpret_cast<uint4*>(out) + (size_t)row * row_chunks;
     for (uint32_t ci = lane; ci < row_chunks; ci += 32) {
@@ -260,13 +262,14 @@ __global__ void __launch_bounds__(256)
 
 template <typename Elem>
 cudaError_t launch_rope_rows(const CacheView& c, int layer, int n_rollouts,
-                             const void* in, void* out, int Tx, cudaStream_t s) {
+                             const void* in, void* out, int Tx, int heads,
+                             cudaStream_t s) {
   const uint64_t rows = (uint64_t)n_rollouts * c.F * Tx;
   const uint64_t blocks_needed = (rows + 7) / 8;  // 8 warps per block
   const unsigned blocks = (unsigned)(blocks_needed < 148ull * 8 ? blocks_needed : 148ull * 8);
   rope3d_kernel<Elem><<<blocks, 256, 0, s>>>(c, layer, n_rollouts,
                                              static_cast<const Elem*>(in),
-                                             static_cast<Elem*>(out), Tx);
+                                             static_cast<Elem*>(out), Tx, heads);
   count_launch(1);
   return cudaGetLastError();
 }
@@ -311,17 +314,18 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
 }
 
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
-                          void* x, int Tx, cudaStream_t s) {
-  if (c.esz == 2) return launch_rope_rows<uint16_t>(c, layer, n_rollouts, x, x, Tx, s);
-  return launch_rope_rows<float>(c, layer, n_rollouts, x, x, Tx, s);
+                          void* x, int Tx, int heads, cudaStream_t s) {
+  if (c.esz == 2)
+    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, x, x, Tx, heads, s);
+  return launch_rope_rows<float>(c, layer, n_rollouts, x, x, Tx, heads, s);
 }
 
 cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
                                    int n_rollouts, const void* k, void* out,
                                    cudaStream_t s) {
   if (c.esz == 2)
-    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, k, out, c.Tf, s);
-  return launch_rope_rows<float>(c, layer, n_rollouts, k, out, c.Tf, s);
+    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, k, out, c.Tf, c.Hkv, s);
+  return launch_rope_rows<float>(c, layer, n_rollouts, k, out, c.Tf, c.Hkv, s);
 }
 
 }  // namespace fd

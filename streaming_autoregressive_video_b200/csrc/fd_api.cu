@@ -56,10 +56,14 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   if (d->num_layers > 256 || d->max_rollouts > 65535 || d->num_heads > 65535 ||
       d->block_frames > 64)
     return FD_ERR_SHAPE;
+  const int32_t hkv = d->num_kv_heads == 0 ? d->num_heads : d->num_kv_heads;
+  if (hkv < 1 || hkv > d->num_heads || d->num_heads % hkv != 0) return FD_ERR_SHAPE;
   if (d->head_dim < 8 || d->head_dim % 8 != 0 || d->head_dim > 256)
     return FD_ERR_SHAPE;
   if (!(d->rope_theta > 1.0f) || !isfinite(d->rope_theta)) return FD_ERR_SHAPE;
-  const size_t T = (size_t)d->grid_h * d->grid_w;
+  const int32_t views = d->num_views == 0 ? 1 : d->num_views;
+  if (views < 1 || views > 64) return FD_ERR_SHAPE;
+  const size_t T = (size_t)views * d->grid_h * d->grid_w;
   const size_t Tf = T + (size_t)d->action_tokens;
   if (Tf > (1u << 24) || T * d->block_frames > (1u << 30)) return FD_ERR_SHAPE;
   const size_t slots = (size_t)d->sink_frames + d->window_frames;
@@ -73,7 +77,7 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   if (p_hw < 1) return FD_ERR_SHAPE;
 
   size_t frame, layer_kv, kv, lr, x;
-  if (!mul_ok(Tf * d->num_heads, (size_t)d->head_dim * esz, &frame) ||
+  if (!mul_ok(Tf * hkv, (size_t)d->head_dim * esz, &frame) ||
       !mul_ok(frame, slots * d->max_rollouts, &layer_kv) ||
       !mul_ok(layer_kv, (size_t)d->num_layers, &kv))
     return FD_ERR_CAPACITY;
@@ -240,10 +244,12 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.L = desc->num_layers;
   v.R = desc->max_rollouts;
   v.H = desc->num_heads;
+  v.Hkv = desc->num_kv_heads == 0 ? desc->num_heads : desc->num_kv_heads;
   v.d = desc->head_dim;
   v.gh = desc->grid_h;
   v.gw = desc->grid_w;
-  v.T = desc->grid_h * desc->grid_w;
+  v.Tv = desc->grid_h * desc->grid_w;
+  v.T = (desc->num_views == 0 ? 1 : desc->num_views) * v.Tv;
   v.Tf = v.T + desc->action_tokens;
   v.F = desc->block_frames;
   v.S = desc->sink_frames;
@@ -255,15 +261,15 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.pw = lay.rope_pairs_w;
   v.esz = desc->dtype == FD_BF16 ? 2 : 4;
   v.theta = (double)desc->rope_theta;
-  v.frame_bytes = (uint64_t)v.Tf * v.H * v.d * v.esz;
+  v.frame_bytes = (uint64_t)v.Tf * v.Hkv * v.d * v.esz;
   c->host_n.assign((size_t)v.L * v.R, 0);
   c->have_maps = false;
   if (desc->dtype == FD_BF16) {
     const uint64_t rows = (uint64_t)v.slots * v.Tf;
     const uint64_t batch = (uint64_t)v.L * v.R;
-    if (!fd::encode_bf16_map(&c->tm_kc, v.krot, v.d, v.H, rows, batch) ||
-        !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.H, rows, batch) ||
-        !fd::encode_bf16_map(&c->tm_kb, v.kblk, v.d, v.H, (uint64_t)v.F * v.Tf,
+    if (!fd::encode_bf16_map(&c->tm_kc, v.krot, v.d, v.Hkv, rows, batch) ||
+        !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.Hkv, rows, batch) ||
+        !fd::encode_bf16_map(&c->tm_kb, v.kblk, v.d, v.Hkv, (uint64_t)v.F * v.Tf,
                              batch)) {
       // only the tensor-core path needs the maps; keep going without them
       c->have_maps = false;
@@ -335,17 +341,19 @@ fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
 }
 
 fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
-                    void* x, int32_t tokens_per_frame, void* stream) {
+                    void* x, int32_t tokens_per_frame, int32_t heads,
+                    void* stream) {
   if (cache == nullptr || x == nullptr) return FD_ERR_INVALID_ARG;
   const fd::CacheView& v = cache->view;
   if (layer < 0 || layer >= v.L || n_rollouts < 1 || n_rollouts > v.R)
     return FD_ERR_INVALID_ARG;
   if (tokens_per_frame != v.T && tokens_per_frame != v.Tf) return FD_ERR_SHAPE;
+  if (heads != v.H && heads != v.Hkv) return FD_ERR_SHAPE;
   if (!fd::aligned16(x)) return FD_ERR_ALIGNMENT;
   fd_status st = fd::check_device(cache);
   if (st != FD_OK) return st;
   return fd::cuda_status(fd::launch_rope3d(v, layer, n_rollouts, x,
-                                           tokens_per_frame,
+                                           tokens_per_frame, heads,
                                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -403,6 +411,8 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.cnt = c.cnt + (size_t)layer * c.R * c.H * c.nb;
   p.nb = c.nb;
   p.H = c.H;
+  p.Hkv = c.Hkv;
+  p.kv_group = c.H / c.Hkv;
   p.d = c.d;
   p.T = c.T;
   p.Tf = c.Tf;
@@ -422,6 +432,8 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.div_T = fd::make_fastdiv((uint32_t)c.T);
   p.div_Tf = fd::make_fastdiv((uint32_t)c.Tf);
   p.div_gw = fd::make_fastdiv((uint32_t)c.gw);
+  p.div_Tv = fd::make_fastdiv((uint32_t)c.Tv);
+  p.Tv = c.Tv;
   p.scale = (float)(1.0 / sqrt((double)c.d));
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -437,10 +449,10 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   CUtensorMap tm_q, tm_vb, tm_kb_work;
   const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
   if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
-      !fd::encode_bf16_map(&tm_vb, v_, c.d, c.H, kb_rows, n_rollouts))
+      !fd::encode_bf16_map(&tm_vb, v_, c.d, c.Hkv, kb_rows, n_rollouts))
     return FD_ERR_CUDA;
   if (work != nullptr &&
-      !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.H, kb_rows, n_rollouts))
+      !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.Hkv, kb_rows, n_rollouts))
     return FD_ERR_CUDA;
   {
     // persistent grid: one CTA per multiprocessor, no more CTAs than KV

@@ -45,8 +45,10 @@ struct CacheView {
   int32_t* cnt;   // [L][R][H][nb] (bf16 caches)
   int32_t* err;
   int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz, nb;
+  int Hkv;               // key/value heads (divides H)
+  int Tv;                // video tokens per view (gh * gw); T = views * Tv
   double theta;
-  uint64_t frame_bytes;  // Tf * H * d * esz
+  uint64_t frame_bytes;  // Tf * Hkv * d * esz (one frame of K or V)
 };
 
 // Persistent tensor-core attention: at most this many CTAs, each with two
@@ -94,6 +96,10 @@ struct AttnParams {
   int32_t* cnt;          // per-unit arrival counters of split units
   int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
   int nb;                // query-tile pairs per (rollout, head)
+  int Hkv;               // key/value heads
+  int kv_group;          // H / Hkv: query head h reads key/value head h / kv_group
+  int Tv;                // video tokens per view
+  FastDiv div_Tv;
   int G;                 // CTAs of the persistent launch
   int map_row0;          // layer * R: row offset of this layer in the cache maps
   int kb_row0;           // batch offset of rollout 0 in the rotated-block-key map
@@ -109,8 +115,9 @@ cudaError_t launch_commit(const CacheView& c, const CommitParams& p,
 cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
                          cudaStream_t s);
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
-                          void* x, int tokens_per_frame, cudaStream_t s);
-// block keys k [n_rollouts][F*Tf][H][d] rotated (positions from `layer`'s
+                          void* x, int tokens_per_frame, int heads,
+                          cudaStream_t s);
+// block keys k [n_rollouts][F*Tf][Hkv][d] rotated (positions from `layer`'s
 // counters) into out, same layout
 cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
                                    int n_rollouts, const void* k, void* out,

@@ -42,9 +42,21 @@ class Workload:
     # ragged cache fill: window frames committed per rollout drawn uniformly
     # from [lo, hi] before the measured block (None = uniform fill)
     ragged_window: Optional[Tuple[int, int]] = None
+    # key/value heads (grouped-query attention); 0 = heads
+    kv_heads: int = 0
+    # camera views per frame (multi-view models); tokens = views * Gh * Gw
+    views: int = 1
+
+    @property
+    def hkv(self) -> int:             # key/value heads
+        return self.kv_heads or self.heads
 
     @property
     def tokens(self) -> int:          # T: video tokens per latent frame
+        return self.views * self.grid_h * self.grid_w
+
+    @property
+    def view_tokens(self) -> int:     # video tokens per view
         return self.grid_h * self.grid_w
 
     @property
@@ -97,4 +109,19 @@ BATCHED_RAGGED = Workload("bf16-16x20-h24-d128-F3-W12-R16-ragged", layers=1,
                           sink_frames=0, window_frames=12, steps=2, blocks=1,
                           dtype="bf16", ragged_window=(3, 12))
 
-ALL = [TINY_F32, SINGLE_480P, LARGE_ACTIONS, LONG_ROLLOUT, BATCHED_RAGGED]
+# 6: four-camera frames at 704x1280 (44x80 latent grid per view under the same
+#    16x spatial compression), 2 denoising steps (AlpaDreams write-up, section
+#    VIII: four-view model, two-step diffusion, 704x1280); one latent frame per
+#    block, 1 sink + 3 window frames; 16 heads of 128 (a 2B-parameter DiT,
+#    hidden 2048).  14080 query tokens x 70400 keys per call.
+MULTIVIEW_4 = Workload("bf16-4x44x80-h16-d128-F1-S1-W3", layers=28, rollouts=1,
+                       heads=16, head_dim=128, grid_h=44, grid_w=80, action_tokens=0,
+                       block_frames=1, sink_frames=1, window_frames=3, steps=2,
+                       blocks=5, dtype="bf16", views=4)
+
+# 7: the 480p shape with grouped-query attention (12 query heads, 4 key/value
+#    heads): a cache-semantics variant, not a configuration of the pages
+GQA_480P = SINGLE_480P.scaled(name="bf16-30x52-h12kv4-d128-F3-S1-W6-L30", kv_heads=4)
+
+ALL = [TINY_F32, SINGLE_480P, LARGE_ACTIONS, LONG_ROLLOUT, BATCHED_RAGGED, MULTIVIEW_4,
+       GQA_480P]

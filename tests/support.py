@@ -31,9 +31,9 @@ def views(cache, w):
     st = cache.storage
     L, R, slots = w.layers, w.rollouts, w.slots
     esz = 2 if w.dtype == "bf16" else 4
-    n_kv = L * R * slots * w.frame_tokens * w.heads * w.head_dim
+    n_kv = L * R * slots * w.frame_tokens * w.hkv * w.head_dim
     kv_dt = torch.int16 if esz == 2 else torch.float32
-    shape = (L, R, slots, w.frame_tokens, w.heads, w.head_dim)
+    shape = (L, R, slots, w.frame_tokens, w.hkv, w.head_dim)
     k = st[lay.k:lay.k + n_kv * esz].view(kv_dt).view(shape)
     v = st[lay.v:lay.v + n_kv * esz].view(kv_dt).view(shape)
     pos = st[lay.pos:lay.pos + L * R * slots * 4].view(torch.int32).view(L, R, slots)
@@ -45,16 +45,16 @@ def krot_view(cache, w):
     """The cache's committed keys rotated to their frame positions."""
     lay = cache.layout
     esz = 2 if w.dtype == "bf16" else 4
-    n_kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.heads * w.head_dim
+    n_kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.hkv * w.head_dim
     kv_dt = torch.int16 if esz == 2 else torch.float32
-    shape = (w.layers, w.rollouts, w.slots, w.frame_tokens, w.heads, w.head_dim)
+    shape = (w.layers, w.rollouts, w.slots, w.frame_tokens, w.hkv, w.head_dim)
     return cache.storage[lay.krot:lay.krot + n_kv * esz].view(kv_dt).view(shape)
 
 
 def check_rotated(got_storage: np.ndarray, raw: np.ndarray, t, w, what=""):
     """got = RoPE(raw) at frame positions t (one entry per frame), within one
     rounding to the storage dtype of the fp64 rotation."""
-    h, ww = oracle.token_coords(w.frame_tokens, w.tokens, w.grid_w)
+    h, ww = oracle.token_coords(w.frame_tokens, w.tokens, w.grid_w, w.view_tokens)
     t = np.asarray(t, dtype=np.float64)[:, None]
     ang = oracle.rope_angles(t, h[None, :], ww[None, :], w.head_dim, w.theta)[:, :, None, :]
     want = oracle.rope_rotate(oracle.values_f64(raw, w.dtype), ang)
@@ -93,7 +93,7 @@ def empty_like_q(w, n_rollouts, device="cuda"):
 def block_inputs(w, seed_parts, n_rollouts):
     """Seeded q, k, v of one attention call, storage form (numpy)."""
     qs = (n_rollouts, w.queries, w.heads, w.head_dim)
-    ks = (n_rollouts, w.block_frames * w.frame_tokens, w.heads, w.head_dim)
+    ks = (n_rollouts, w.block_frames * w.frame_tokens, w.hkv, w.head_dim)
     q = synth.normal(synth.seed_of(*seed_parts, 0), qs, w.dtype, w.value_scale)
     k = synth.normal(synth.seed_of(*seed_parts, 1), ks, w.dtype, w.value_scale)
     v = synth.normal(synth.seed_of(*seed_parts, 2), ks, w.dtype, w.value_scale)
@@ -119,7 +119,7 @@ class Lockstep:
         self.cache = new_cache(w, device)
         self.device = device
         self.orc = [[oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens,
-                                         w.heads, w.head_dim, w.dtype)
+                                         w.hkv, w.head_dim, w.dtype)
                      for _ in range(w.rollouts)] for _ in range(w.layers)]
 
     def attention(self, layer, q, k, v, n_rollouts=None, rows=None, with_lse=True,
@@ -138,7 +138,7 @@ class Lockstep:
             for r in range(nr):
                 want, want_lse = oracle.block_attention(
                     self.orc[layer][r], q[r], k[r], v[r], tokens=w.tokens,
-                    grid_w=w.grid_w, theta=w.theta, rows=rows)
+                    grid_w=w.grid_w, theta=w.theta, rows=rows, view_tokens=w.view_tokens)
                 sel = slice(None) if rows is None else np.asarray(rows)
                 errs.append(compare(got[r][sel], want[sel], w.dtype, f"{what} r={r}"))
                 if with_lse:
@@ -159,8 +159,8 @@ class Lockstep:
         for i, l in enumerate(layers):
             for r in range(nr):
                 nf = F if frames is None else int(frames[r])
-                kf = k_list[i][r].reshape(F, Tf, w.heads, w.head_dim)[:nf]
-                vf = v_list[i][r].reshape(F, Tf, w.heads, w.head_dim)[:nf]
+                kf = k_list[i][r].reshape(F, Tf, w.hkv, w.head_dim)[:nf]
+                vf = v_list[i][r].reshape(F, Tf, w.hkv, w.head_dim)[:nf]
                 self.orc[l][r].commit(kf, vf)
         torch.cuda.synchronize()
 

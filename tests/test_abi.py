@@ -34,13 +34,13 @@ def test_cache_bytes_and_layout():
         lay = fd.fd_cache_get_layout(desc)
         assert n == lay.total > 0
         esz = 2 if w.dtype == "bf16" else 4
-        kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.heads * w.head_dim * esz
+        kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.hkv * w.head_dim * esz
         assert lay.layer_kv_bytes * w.layers == kv
         regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.part, lay.cnt, lay.pos, lay.count,
                    lay.ttab, lay.htab, lay.wtab, lay.err]
         assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
         assert lay.v - lay.k >= kv and lay.krot - lay.v >= kv and lay.kblk - lay.krot >= kv
-        blk = w.layers * w.rollouts * w.block_frames * w.frame_tokens * w.heads * w.head_dim * esz
+        blk = w.layers * w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * esz
         assert lay.part - lay.kblk >= blk
         # partial results of split query-tile pairs: 148 CTAs x 2 slots per
         # layer, fp32 O [256][128] + max + sum; none for fp32 caches
@@ -91,9 +91,23 @@ def test_host_errors_before_any_device_call():
     assert lib.fd_block_attention(None, 0, 1, 16, 16, 16, 16, None, None) == 1
     assert lib.fd_cache_commit(None, 0, 1, 1, None, None, None, None) == 1
     assert lib.fd_cache_reset(None, None, 1, None) == 1
-    assert lib.fd_rope3d(None, 0, 1, 16, 4, None) == 1
+    assert lib.fd_rope3d(None, 0, 1, 16, 4, 1, None) == 1
     code = ctypes.c_int32()
     assert lib.fd_get_device_error(None, ctypes.byref(code)) == 1
     assert lib.fd_cache_destroy(None) == 1
     assert fd.fd_status_string(6) == "device-side wait gave up"
     assert fd.fd_launch_count() >= 0
+
+
+@pytest.mark.parametrize("heads,kv_heads,status", [(4, 3, 2), (4, 8, 2), (4, -1, 2),
+                                                   (4, 2, 0), (6, 1, 0), (4, 0, 0)])
+def test_grouped_query_heads_validated(heads, kv_heads, status):
+    w = SINGLE_480P.scaled(heads=heads, kv_heads=kv_heads, layers=1)
+    desc = fd.make_desc(w)
+    lay = fd.CacheLayout()
+    assert fd.load().fd_cache_get_layout(ctypes.byref(desc), ctypes.byref(lay)) == status
+    if status == 0:
+        # K and V regions hold Hkv heads
+        hkv = kv_heads or heads
+        kv = w.slots * w.frame_tokens * hkv * w.head_dim * 2
+        assert lay.layer_kv_bytes == kv

@@ -30,9 +30,11 @@ def _commit_block(ls, w, seed, layers=None, frames=None):
     ls.commit(layers, ks, vs, frames=frames)
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_commit_and_reset_bit_exact(dtype):
-    w = SMALL.scaled(dtype=dtype, grid_h=3, grid_w=5, action_tokens=2)
+@pytest.mark.parametrize("dtype,kv_heads,views", [("bf16", 0, 1), ("f32", 0, 1),
+                                                  ("bf16", 1, 1), ("bf16", 0, 2)])
+def test_commit_and_reset_bit_exact(dtype, kv_heads, views):
+    w = SMALL.scaled(dtype=dtype, grid_h=3, grid_w=5, action_tokens=2, kv_heads=kv_heads,
+                     views=views)
     ls = Lockstep(w)
     ls.check_cache_exact()
     rng = np.random.default_rng(5)
@@ -50,17 +52,20 @@ def test_commit_and_reset_bit_exact(dtype):
 
 @pytest.mark.parametrize("dtype,tokens", [("bf16", "T"), ("bf16", "Tf"), ("f32", "Tf")])
 def test_rope3d_matches_oracle(dtype, tokens):
-    w = SMALL.scaled(dtype=dtype, grid_h=5, grid_w=7, action_tokens=3, window_frames=4)
+    # keys carry Hkv = 1 head, queries H = 2; two camera views per frame
+    w = SMALL.scaled(dtype=dtype, grid_h=5, grid_w=7, action_tokens=3, window_frames=4,
+                     kv_heads=1, views=2)
     ls = Lockstep(w)
     for blk in range(3):
         _commit_block(ls, w, 200 + blk)
     Tx = w.tokens if tokens == "T" else w.frame_tokens
-    x = synth.normal(synth.seed_of(9, Tx), (w.rollouts, w.block_frames, Tx, w.heads, w.head_dim), dtype)
+    heads = w.heads if tokens == "T" else w.hkv
+    x = synth.normal(synth.seed_of(9, Tx), (w.rollouts, w.block_frames, Tx, heads, w.head_dim), dtype)
     xd = to_device(x)
-    fd.fd_rope3d(ls.cache, 1, w.rollouts, xd, Tx)
+    fd.fd_rope3d(ls.cache, 1, w.rollouts, xd, Tx, heads)
     torch.cuda.synchronize()
     got = oracle.values_f64(to_host(xd), dtype)
-    h, ww = oracle.token_coords(Tx, w.tokens, w.grid_w)
+    h, ww = oracle.token_coords(Tx, w.tokens, w.grid_w, w.view_tokens)
     for r in range(w.rollouts):
         n = ls.orc[1][r].n
         t = (n + np.arange(w.block_frames))[:, None]
@@ -74,9 +79,12 @@ def test_rope3d_matches_oracle(dtype, tokens):
             assert err.max() <= 1e-5
 
 
-def test_attention_f32_tiny_rollout():
-    """Tiny fp32 rollout: 20 blocks x 2 steps through a 3-frame window."""
-    w = TINY_F32
+@pytest.mark.parametrize("kv_heads,views", [(0, 1), (1, 1), (0, 2)])
+def test_attention_f32_tiny_rollout(kv_heads, views):
+    """Tiny fp32 rollout: 20 blocks x 2 steps through a 3-frame window (and
+    the same with grouped-query attention, one key/value head, and with two
+    camera views per frame)."""
+    w = TINY_F32.scaled(kv_heads=kv_heads, views=views)
     ls = Lockstep(w)
     for blk in range(w.blocks):
         for step in range(w.steps):
@@ -102,6 +110,9 @@ def test_single_key_returns_value_exactly_bf16():
     dict(action_tokens=4),                             # Tf=160 with action tokens
     dict(grid_h=16, grid_w=20, block_frames=3, window_frames=3, sink_frames=0),  # F = W
     dict(rollouts=4, sink_frames=2, window_frames=4),  # sinks straddled
+    dict(heads=4, kv_heads=2, action_tokens=4),        # grouped-query attention
+    dict(heads=3, kv_heads=1, rollouts=2),             # one key/value head
+    dict(views=3, grid_h=4, grid_w=5, action_tokens=2),  # three camera views
 ])
 def test_attention_bf16_rollout(shape):
     """Rollout through empty, partial, full and wrapped cache states."""

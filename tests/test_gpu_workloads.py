@@ -12,8 +12,9 @@ import torch
 import oracle
 from streaming_autoregressive_video_b200 import binding as fd
 from streaming_autoregressive_video_b200 import synth
-from streaming_autoregressive_video_b200.workloads import (BATCHED_RAGGED, LARGE_ACTIONS,
-                                                           LONG_ROLLOUT, SINGLE_480P)
+from streaming_autoregressive_video_b200.workloads import (BATCHED_RAGGED, GQA_480P,
+                                                           LARGE_ACTIONS, LONG_ROLLOUT,
+                                                           MULTIVIEW_4, SINGLE_480P)
 
 from support import Lockstep, block_inputs, compare, new_cache, out_values, to_device, \
     to_host, views
@@ -62,6 +63,19 @@ def test_large_model_with_action_tokens():
     (Tf = 1564): 4680 queries x 25024 keys, values N(0,1)*0.5."""
     w = LARGE_ACTIONS.scaled(layers=1)
     prefill_and_call(w, [0], seed=22)
+
+
+def test_multiview_four_cameras_704x1280():
+    """4 views of 44x80 per frame (14080 tokens), 16 heads, 1 sink + 3-frame
+    window (full): 14080 queries x 70400 keys."""
+    w = MULTIVIEW_4.scaled(layers=1)
+    prefill_and_call(w, [0], seed=25)
+
+
+def test_grouped_query_attention_480p():
+    """12 query heads over 4 key/value heads at the 480p shape."""
+    w = GQA_480P.scaled(layers=1)
+    prefill_and_call(w, [0], seed=26)
 
 
 def test_batched_ragged_rollouts():
