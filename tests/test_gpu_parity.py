@@ -95,6 +95,26 @@ def test_attention_f32_tiny_rollout(kv_heads, views):
     assert fd.fd_get_device_error(ls.cache) == 0
 
 
+def test_unsupported_bf16_head_dim_is_refused_cleanly():
+    """The tensor-core kernel handles d = 128 only: a bf16 cache with d = 64
+    commits and rotates, but attention returns FD_ERR_UNSUPPORTED without
+    launching anything, and the context stays usable."""
+    w = Workload("bf16-d64", layers=1, rollouts=1, heads=2, head_dim=64, grid_h=3, grid_w=4,
+                 action_tokens=0, block_frames=1, sink_frames=0, window_frames=2, steps=1,
+                 blocks=1, dtype="bf16")
+    ls = Lockstep(w)
+    q, k, v = block_inputs(w, (7, 0), 1)
+    _commit_block(ls, w, 500)
+    ls.check_cache_exact()
+    out = torch.empty((1, w.queries, w.heads, w.head_dim), dtype=torch.int16, device="cuda")
+    before = fd.fd_launch_count()
+    with pytest.raises(fd.FdError) as e:
+        fd.fd_block_attention(ls.cache, 0, 1, to_device(q), to_device(k), to_device(v), out)
+    assert e.value.status == 7
+    assert fd.fd_launch_count() == before
+    assert fd.fd_get_device_error(ls.cache) == 0
+
+
 def test_single_key_returns_value_exactly_bf16():
     w = Workload("one-key", layers=1, rollouts=1, heads=3, head_dim=128, grid_h=1, grid_w=1,
                  action_tokens=0, block_frames=1, sink_frames=0, window_frames=1, steps=1,
