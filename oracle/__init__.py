@@ -25,4 +25,5 @@ from .streaming_attention import (  # noqa: F401
     valid_slot_count,
     RolloutCache,
     block_attention,
+    combine_partials,
 )

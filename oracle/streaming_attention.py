@@ -59,6 +59,14 @@ R10 multi-view frames (a shape variant; the pages show four-camera models
     (Gh*Gw), and all views of a frame share t.  Views therefore differ only by
     content (any learned view embedding belongs to the model, before the
     attention).  V = 1 is R5.
+R11 context parallelism (a way to compute the same attention on N devices,
+    named by the pages without formulas): the key set splits into disjoint
+    parts; part i yields the softmax-normalised output O_i and log-sum-exp
+    lse_i over its own keys; the whole-set result is
+    O = sum_i exp(lse_i - M) O_i / sum_i exp(lse_i - M) and
+    lse = M + log sum_i exp(lse_i - M), M = max_i lse_i (a part with no keys
+    has lse = -inf and weight 0).  Parts here: cache slot s belongs to part
+    s mod N; the block's own keys belong to part 0.
 """
 from __future__ import annotations
 
@@ -211,7 +219,8 @@ class RolloutCache:
 # --------------------------------------------------------------------------
 def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
                     theta: float, heads=None, rows=None, row_chunk: int = 512,
-                    return_probs: bool = False, view_tokens: int = 0):
+                    return_probs: bool = False, view_tokens: int = 0,
+                    slot_part=None, include_block: bool = True):
     """Attention of the current block's queries of one (rollout, layer).
 
     q:    [F*T][H][d]    queries of the block, storage form, pre-RoPE
@@ -223,6 +232,10 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
            every row's softmax still runs over the whole key set
     view_tokens: video tokens per view of a multi-view frame (R10; 0 = one
            view of all `tokens`)
+    slot_part, include_block: attention over a part of the key set (R11):
+           only valid cache slots s with s mod N == r for slot_part = (N, r),
+           and the block's keys only if include_block; rows with no key get
+           out = 0 and lse = -inf
 
     Returns (out [F*T][H][d] fp64, lse [H][F*T] fp64 natural-log sum of exp of
     the scaled scores) and, with return_probs, a dict head -> P [F*T][Nk].
@@ -241,13 +254,21 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     n = cache.n
     nv = cache.valid_slots()
 
-    # coordinates of every key: valid cache slots in slot order, then the block
+    # the key set's slots (R11: possibly one part of it)
+    slots = np.arange(nv)
+    if slot_part is not None:
+        n_parts, part = slot_part
+        slots = slots[slots % n_parts == part]
+    nf_block = F if include_block else 0
+    ns = len(slots)
+
+    # coordinates of every key: the slots in slot order, then the block
     h_tok, w_tok = token_coords(Tf, T, grid_w, view_tokens)
-    t_cache = np.repeat(cache.pos[:nv].astype(np.float64), Tf)
-    t_block = np.repeat(np.arange(n, n + F, dtype=np.float64), Tf)
+    t_cache = np.repeat(cache.pos[slots].astype(np.float64), Tf)
+    t_block = np.repeat(np.arange(n, n + nf_block, dtype=np.float64), Tf)
     t_key = np.concatenate([t_cache, t_block])
-    h_key = np.tile(h_tok, nv + F)
-    w_key = np.tile(w_tok, nv + F)
+    h_key = np.tile(h_tok, ns + nf_block)
+    w_key = np.tile(w_tok, ns + nf_block)
     ang_k = rope_angles(t_key, h_key, w_key, d, theta)          # [Nk][d/2]
 
     # coordinates of the evaluated queries (video tokens only)
@@ -259,13 +280,18 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
     out = np.zeros((Mq, H, d), dtype=np.float64)
     lse = np.zeros((H, Mq), dtype=np.float64)
     probs = {}
+    if ns + nf_block == 0:  # no key at all (R11)
+        lse[:] = -np.inf
+        return (out, lse, probs) if return_probs else (out, lse)
     for hh in (range(H) if heads is None else heads):
         g = hh // group  # key/value head of this query head (R9)
         qh = rope_rotate(values_f64(q[rows, hh, :], dtype), ang_q)
-        kc = values_f64(cache.k[:nv, :, g, :], dtype).reshape(nv * Tf, d)
-        vc = values_f64(cache.v[:nv, :, g, :], dtype).reshape(nv * Tf, d)
-        kh = rope_rotate(np.concatenate([kc, values_f64(k[:, g, :], dtype)]), ang_k)
-        vh = np.concatenate([vc, values_f64(v[:, g, :], dtype)])
+        kc = values_f64(cache.k[slots, :, g, :], dtype).reshape(ns * Tf, d)
+        vc = values_f64(cache.v[slots, :, g, :], dtype).reshape(ns * Tf, d)
+        kb = values_f64(k[:, g, :], dtype)[:nf_block * Tf]
+        vb = values_f64(v[:, g, :], dtype)[:nf_block * Tf]
+        kh = rope_rotate(np.concatenate([kc, kb]), ang_k)
+        vh = np.concatenate([vc, vb])
         if return_probs:
             probs[hh] = np.zeros((Mq, kh.shape[0]), dtype=np.float64)
         for c0 in range(0, len(rows), row_chunk):
@@ -280,4 +306,28 @@ def block_attention(cache: RolloutCache, q, k, v, *, tokens: int, grid_w: int,
                 probs[hh][sel] = e / l
     if return_probs:
         return out, lse, probs
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# context parallelism (reading R11)
+# --------------------------------------------------------------------------
+def combine_partials(outs, lses):
+    """Whole-key-set attention from per-part results (R11).
+
+    outs: list of [Mq][H][d] fp64 outputs, each normalised over its part
+    lses: list of [H][Mq] fp64 log-sum-exp of the same parts (-inf: no keys)
+    Returns (out [Mq][H][d], lse [H][Mq]).
+    """
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])       # [N][H][Mq]
+    M = L.max(axis=0)                                                  # [H][Mq]
+    Msafe = np.where(np.isfinite(M), M, 0.0)
+    w = np.where(np.isfinite(L), np.exp(L - Msafe[None]), 0.0)          # [N][H][Mq]
+    tot = w.sum(axis=0)                                                # [H][Mq]
+    out = np.zeros_like(np.asarray(outs[0], dtype=np.float64))
+    for wi, oi in zip(w, outs):
+        out += np.asarray(oi, dtype=np.float64) * wi.T[:, :, None]
+    has = tot > 0
+    out = np.where(has.T[:, :, None], out / np.where(has, tot, 1.0).T[:, :, None], 0.0)
+    lse = np.where(has, Msafe + np.log(np.where(has, tot, 1.0)), -np.inf)
     return out, lse

@@ -450,3 +450,51 @@ def test_multiview_attention_is_equivariant_to_swapping_views():
     oc, _ = block_attention(b, q[perm[:T]], k[perm], v[perm], tokens=T, grid_w=gw,
                             theta=1.0e4)
     assert np.abs(oc - oa[perm[:T]]).max() > 1e-3
+
+
+# --------------------------------------------------------------------------
+# context parallelism (reading R11)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("N", [2, 3, 4])
+def test_parts_recombine_to_the_whole_key_set(N):
+    # cache slots split round-robin over N parts, the block's keys in part 0:
+    # recombining the parts' normalised outputs by their log-sum-exps gives the
+    # attention over the whole key set (an identity of the softmax)
+    rng = np.random.default_rng(51 + N)
+    S, W, F, T, H, d = 1, 4, 2, 6, 2, 12
+    c = RolloutCache(S, W, T, H, d, "f32")
+    for _ in range(4):
+        c.commit(rng.standard_normal((F, T, H, d)).astype(np.float32),
+                 rng.standard_normal((F, T, H, d)).astype(np.float32))
+    q = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    k = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    v = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    kw = dict(tokens=T, grid_w=3, theta=1.0e4)
+    full, full_lse = block_attention(c, q, k, v, **kw)
+    parts = [block_attention(c, q, k, v, slot_part=(N, r), include_block=(r == 0), **kw)
+             for r in range(N)]
+    out, lse = oracle.combine_partials([p[0] for p in parts], [p[1] for p in parts])
+    np.testing.assert_allclose(out, full, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, full_lse, rtol=0, atol=1e-12)
+
+
+def test_empty_part_has_no_weight():
+    rng = np.random.default_rng(57)
+    S, W, T, H, d = 0, 2, 4, 1, 12
+    c = RolloutCache(S, W, T, H, d, "f32")
+    c.commit(rng.standard_normal((1, T, H, d)).astype(np.float32),
+             rng.standard_normal((1, T, H, d)).astype(np.float32))
+    q = rng.standard_normal((T, H, d)).astype(np.float32)
+    k = rng.standard_normal((T, H, d)).astype(np.float32)
+    v = rng.standard_normal((T, H, d)).astype(np.float32)
+    kw = dict(tokens=T, grid_w=2, theta=1.0e4)
+    # one valid slot (slot 0): part 1 of 2 holds nothing and no block keys
+    o1, l1 = block_attention(c, q, k, v, slot_part=(2, 1), include_block=False, **kw)
+    assert np.all(o1 == 0) and np.all(np.isneginf(l1))
+    o0, l0 = block_attention(c, q, k, v, slot_part=(2, 0), include_block=True, **kw)
+    out, lse = oracle.combine_partials([o0, o1], [l0, l1])
+    np.testing.assert_array_equal(out, o0)
+    np.testing.assert_array_equal(lse, l0)
+    # no keys anywhere: zero rows, -inf
+    out, lse = oracle.combine_partials([o1, o1], [l1, l1])
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
