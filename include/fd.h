@@ -21,6 +21,8 @@
  *            historical clean frames and the current noisy frame via a KV cache.
  *   [DZ-SR]  "Single-GPU inference for DreamZero", Sequential requests: KV and
  *            frame positions carry over between requests; explicit reset.
+ *   [FD-CP]  "NVIDIA FlashDreams ...", section Multi-GPU Context Parallelism:
+ *            one rollout's inference sharded across several GPUs.
  *
  * Readings where the pages are silent (the same ones the test oracle states):
  *   - scores q.k/sqrt(d), softmax over the whole key set, no bias or mask
@@ -102,6 +104,12 @@ typedef struct {
                            * token i sits at (h, w) of i mod (grid_h*grid_w)
                            * and all views share t (no counterpart on the
                            * pages beyond their four-view models)           */
+  int32_t num_shards;     /* N context-parallel shards of the key set (0: 1)
+                           * ([FD-CP]); this cache stores the ring slots s
+                           * with s % N == shard_index at local index s / N,
+                           * every shard counts all committed frames, and the
+                           * block's own keys belong to shard 0              */
+  int32_t shard_index;    /* this cache's shard, 0 <= shard_index < N      */
 } fd_cache_desc;
 
 /* Byte offsets of the regions inside the caller's storage buffer.
@@ -267,6 +275,25 @@ fd_status fd_exp2_selfcheck(const float* x, float* y, int64_t n, void* stream);
  * fd_get_device_error (FD_ERR_DEVICE_TIMEOUT, code 0x501). */
 fd_status fd_selftest_bounded_wait(fd_cache* cache, int32_t limit_ms,
                                    void* stream);
+
+/* Context parallelism ([FD-CP]): rows of attention over a key set split into
+ * parts from each part's rows and log-sum-exp, e.g. the outputs of
+ * fd_block_attention on the N shards of one cache (gathered onto one device,
+ * by NCCL or a peer copy, before this call):
+ *   outs[i]: [n_rollouts][rows][heads][head_dim] of `dtype`, normalised over
+ *            part i's keys (device, host array of n_parts pointers)
+ *   lses[i]: [n_rollouts][heads][rows] fp32 natural-log sum of exponentials
+ *            of part i's scaled scores; -inf for a part with no key
+ *   out    : the whole-set rows, same layout as outs[i]; lse: its
+ *            log-sum-exp (or NULL)
+ * O = sum_i exp(lse_i - M) O_i / sum_i exp(lse_i - M), M = max_i lse_i,
+ * computed in fp32 and rounded once to `dtype`; rows no part has a key for
+ * become 0 with lse -inf.  1 <= n_parts <= 16.  No counterpart formula on the
+ * pages, which only name context parallelism. */
+fd_status fd_attention_combine(int32_t n_parts, const void* const* outs,
+                               const float* const* lses, int32_t n_rollouts,
+                               int32_t rows, int32_t heads, int32_t head_dim,
+                               int32_t dtype, void* out, float* lse, void* stream);
 
 /* Number of kernels this library has launched in this process. */
 uint64_t fd_launch_count(void);

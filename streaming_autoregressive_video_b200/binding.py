@@ -25,8 +25,8 @@ EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
            "fd_cache_reset", "fd_rope3d", "fd_block_attention",
            "fd_block_attention_static",
            "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
-           "fd_exp2_selfcheck", "fd_selftest_bounded_wait", "fd_launch_count",
-           "fd_status_string"]
+           "fd_exp2_selfcheck", "fd_selftest_bounded_wait", "fd_attention_combine",
+           "fd_launch_count", "fd_status_string"]
 
 
 class FdError(RuntimeError):
@@ -42,7 +42,8 @@ class CacheDesc(ctypes.Structure):
                 ("action_tokens", ctypes.c_int32), ("block_frames", ctypes.c_int32),
                 ("sink_frames", ctypes.c_int32), ("window_frames", ctypes.c_int32),
                 ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("num_kv_heads", ctypes.c_int32), ("num_views", ctypes.c_int32)]
+                ("num_kv_heads", ctypes.c_int32), ("num_views", ctypes.c_int32),
+                ("num_shards", ctypes.c_int32), ("shard_index", ctypes.c_int32)]
 
 
 class CacheLayout(ctypes.Structure):
@@ -90,6 +91,8 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
     lib.fd_get_device_error.argtypes = [vp, ctypes.POINTER(i32)]
     lib.fd_exp2_selfcheck.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.fd_selftest_bounded_wait.argtypes = [vp, i32, vp]
+    lib.fd_attention_combine.argtypes = [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
+                                         i32, i32, i32, vp, vp, vp]
     lib.fd_launch_count.argtypes = []
     lib.fd_launch_count.restype = ctypes.c_uint64
     lib.fd_status_string.argtypes = [i32]
@@ -124,13 +127,14 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def make_desc(w, dtype: Optional[str] = None) -> CacheDesc:
-    """CacheDesc of a workload (see workloads.Workload)."""
+def make_desc(w, dtype: Optional[str] = None, shards: int = 1, shard: int = 0) -> CacheDesc:
+    """CacheDesc of a workload (see workloads.Workload); `shards`/`shard`
+    select one context-parallel shard of its key set."""
     dt = dtype or w.dtype
     return CacheDesc(w.layers, w.rollouts, w.heads, w.head_dim, w.grid_h, w.grid_w,
                      w.action_tokens, w.block_frames, w.sink_frames, w.window_frames,
                      float(w.theta), FD_BF16 if dt == "bf16" else FD_F32,
-                     getattr(w, "kv_heads", 0), getattr(w, "views", 1))
+                     getattr(w, "kv_heads", 0), getattr(w, "views", 1), shards, shard)
 
 
 def fd_cache_bytes(desc: CacheDesc) -> int:
@@ -240,6 +244,18 @@ def fd_exp2_selfcheck(x, y, stream=None) -> None:
 def fd_selftest_bounded_wait(cache: Cache, limit_ms: int, stream=None) -> None:
     _check(load().fd_selftest_bounded_wait(cache.handle, limit_ms, _stream(stream)),
            "fd_selftest_bounded_wait")
+
+
+def fd_attention_combine(outs, lses, out, lse=None, stream=None) -> None:
+    """out (and lse) = log-sum-exp combination of per-part rows `outs` [R][Mq][H][d]
+    with their log-sum-exps `lses` [R][H][Mq] (device tensors)."""
+    n = len(outs)
+    R, Mq, H, d = out.shape
+    dt = FD_BF16 if out.element_size() == 2 else FD_F32
+    op = (ctypes.c_void_p * n)(*[_ptr(t) for t in outs])
+    lp = (ctypes.c_void_p * n)(*[_ptr(t) for t in lses])
+    _check(load().fd_attention_combine(n, op, lp, R, Mq, H, d, dt, _ptr(out), _ptr(lse),
+                                       _stream(stream)), "fd_attention_combine")
 
 
 def fd_get_device_error(cache: Cache) -> int:

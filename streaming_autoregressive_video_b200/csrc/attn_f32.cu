@@ -52,10 +52,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int r = blockIdx.z, h = blockIdx.y;
   const int q0 = blockIdx.x * kRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = p.count[r];
-  const int S = p.S, W = p.W;
-  const int nv = min(n, S) + min(max(n - S, 0), W);
-  const int n1 = nv * p.Tf, n2 = p.F * p.Tf;
+  const int nv = valid_slots_local(valid_slots_global(p.count[r], p.S, p.W), p.N, p.shard);
+  const int n1 = nv * p.Tf, n2 = p.shard == 0 ? p.F * p.Tf : 0;
   const float2* tt = p.ttab + (size_t)r * (p.slots + p.F) * p.pt;
   const float* qg = reinterpret_cast<const float*>(p.q);
   const float* kg = reinterpret_cast<const float*>(p.k);
@@ -164,12 +162,13 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int i = 0; i < kRowsPerWarp; ++i) {
     const int q = q0 + warp * kRowsPerWarp + i;
     if (q >= p.Mq) continue;
-    const float inv = 1.f / l[i];
+    // a shard may hold no key of this rollout: zero row, log-sum-exp -inf
+    const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
     float* dst = outg + (((size_t)r * p.Mq + q) * p.H + h) * D;
 #pragma unroll
     for (int e = 0; e < kPerLane; ++e) dst[lane + 32 * e] = o[i][e] * inv;
     if (p.lse != nullptr && lane == 0)
-      p.lse[((size_t)r * p.H + h) * p.Mq + q] = m[i] + logf(l[i]);
+      p.lse[((size_t)r * p.H + h) * p.Mq + q] = l[i] > 0.f ? m[i] + logf(l[i]) : -INFINITY;
   }
 }
 

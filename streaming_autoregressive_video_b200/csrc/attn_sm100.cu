@@ -158,10 +158,9 @@ struct TileCounts {
 
 __device__ __forceinline__ TileCounts tile_counts(const AttnParams& p, int r) {
   TileCounts t;
-  const int n = p.count[r];
-  const int nv = min(n, p.S) + min(max(n - p.S, 0), p.W);
+  const int nv = valid_slots_local(valid_slots_global(p.count[r], p.S, p.W), p.N, p.shard);
   t.n1 = nv * p.Tf;
-  t.n2 = p.F * p.Tf;
+  t.n2 = p.shard == 0 ? p.F * p.Tf : 0;  // the block's keys belong to shard 0
   t.nt1 = (t.n1 + kBN - 1) / kBN;
   t.nt = t.nt1 + (t.n2 + kBN - 1) / kBN;
   return t;
@@ -238,12 +237,13 @@ __device__ __forceinline__ Cursor cursor_init(const AttnParams& p, const Sched& 
 __device__ __forceinline__ bool next_piece(const AttnParams& p, const Sched& s,
                                            Cursor& c, Piece& pc) {
   const int per_r = p.H * p.nb;
-  if (c.w < s.W) {  // a whole unit
+  while (c.w < s.W) {  // a whole unit
     const int unit = c.w * p.G + blockIdx.x;
     ++c.w;
     pc.r = unit / per_r;
     const int u = unit - pc.r * per_r;
     pc.tc = tile_counts(p, pc.r);
+    if (pc.tc.nt == 0) continue;  // a shard with no key of this rollout
     pc.h = u / p.nb;
     pc.b = u - pc.h * p.nb;
     pc.kv0 = 0;

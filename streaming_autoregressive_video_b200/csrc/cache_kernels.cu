@@ -135,7 +135,9 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int l = p.layer0 + li, r = p.rollout0 + ri;
   const size_t lr = (size_t)l * c.R + r;
   const int n = c.count[lr];
-  const int slot = slot_of(n + f, c.S, c.W);
+  const int gslot = slot_of(n + f, c.S, c.W);
+  if (gslot % c.N != c.shard) return;  // another shard stores this frame
+  const int slot = gslot / c.N;          // local slot
   const uint64_t fvecs = c.frame_bytes / 16;
   const uint8_t* src_base = kv ? p.v[li] : p.k[li];
   const uint4* src = reinterpret_cast<const uint4*>(
@@ -186,7 +188,10 @@ __global__ void commit_meta_kernel(CacheView c, CommitParams p) {
   const int nf = p.frames[ri];
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int f = 0; f < nf; ++f) pos[slot_of(n + f, c.S, c.W)] = n + f;
+    for (int f = 0; f < nf; ++f) {
+      const int gslot = slot_of(n + f, c.S, c.W);
+      if (gslot % c.N == c.shard) pos[gslot / c.N] = n + f;
+    }
     c.count[lr] = n + nf;
   }
   __syncthreads();

@@ -66,8 +66,14 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   const size_t T = (size_t)views * d->grid_h * d->grid_w;
   const size_t Tf = T + (size_t)d->action_tokens;
   if (Tf > (1u << 24) || T * d->block_frames > (1u << 30)) return FD_ERR_SHAPE;
-  const size_t slots = (size_t)d->sink_frames + d->window_frames;
-  if (slots * Tf > (1u << 30)) return FD_ERR_SHAPE;
+  const size_t gslots = (size_t)d->sink_frames + d->window_frames;
+  if (gslots * Tf > (1u << 30)) return FD_ERR_SHAPE;
+  // context-parallel shard: ring slots s with s % N == shard_index, local s / N
+  const int32_t shards = d->num_shards == 0 ? 1 : d->num_shards;
+  if (shards < 1 || shards > 64 || (size_t)shards > gslots || d->shard_index < 0 ||
+      d->shard_index >= shards)
+    return FD_ERR_SHAPE;
+  const size_t slots = (gslots + shards - 1) / shards;  // local slots
   const size_t esz = d->dtype == FD_BF16 ? 2 : 4;
   const int d2 = d->head_dim / 2;
   const int p_hw = d->head_dim / 6;
@@ -254,7 +260,9 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.F = desc->block_frames;
   v.S = desc->sink_frames;
   v.W = desc->window_frames;
-  v.slots = v.S + v.W;
+  v.N = desc->num_shards == 0 ? 1 : desc->num_shards;
+  v.shard = desc->shard_index;
+  v.slots = (v.S + v.W + v.N - 1) / v.N;  // local slots of this shard
   v.nb = (v.F * v.T + 255) / 256;
   v.pt = lay.rope_pairs_t;
   v.ph = lay.rope_pairs_h;
@@ -404,6 +412,8 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.wtab = c.wtab;
   p.out = out;
   p.lse = lse;
+  p.N = c.N;
+  p.shard = c.shard;
   p.err = c.err;
   p.kc = c.krot + (size_t)layer * cache->layout.layer_kv_bytes;
   p.vc = c.v + (size_t)layer * cache->layout.layer_kv_bytes;
@@ -443,8 +453,13 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   } else if (c.d != 128 || !cache->have_maps) {
     return FD_ERR_UNSUPPORTED;
   }
-  st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
-  if (st != FD_OK) return st;
+  // a shard's result is only usable with its log-sum-exp (to be combined)
+  if (c.N > 1 && lse == nullptr) return FD_ERR_INVALID_ARG;
+  // the block's keys belong to shard 0; other shards never read them
+  if (c.shard == 0) {
+    st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
+    if (st != FD_OK) return st;
+  }
   if (cache->desc.dtype == FD_F32) return fd::cuda_status(fd::launch_attn_f32(p, s));
   CUtensorMap tm_q, tm_vb, tm_kb_work;
   const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
@@ -465,6 +480,12 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
     // the kernel's schedule arithmetic is 32-bit
     if (it_max * g >= ((int64_t)1 << 31)) return FD_ERR_UNSUPPORTED;
     p.G = (int)g;
+  }
+  if (c.shard != 0) {
+    // rollouts with no key on this shard get zero rows and lse = -inf here;
+    // the tensor-core kernel skips them
+    st = fd::cuda_status(fd::launch_attn_zero_keyless(p, s));
+    if (st != FD_OK) return st;
   }
   return fd::cuda_status(fd::launch_attn_bf16_sm100(
       tm_q, cache->tm_kc, cache->tm_vc, work != nullptr ? tm_kb_work : cache->tm_kb,
@@ -541,6 +562,39 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code) {
     return FD_ERR_DEVICE_TIMEOUT;
   }
   return FD_OK;
+}
+
+fd_status fd_attention_combine(int32_t n_parts, const void* const* outs,
+                               const float* const* lses, int32_t n_rollouts,
+                               int32_t rows, int32_t heads, int32_t head_dim,
+                               int32_t dtype, void* out, float* lse, void* stream) {
+  if (outs == nullptr || lses == nullptr || out == nullptr) return FD_ERR_INVALID_ARG;
+  if (n_parts < 1 || n_parts > fd::kCombineMaxParts) return FD_ERR_SHAPE;
+  if (dtype != FD_BF16 && dtype != FD_F32) return FD_ERR_DTYPE;
+  if (n_rollouts < 1 || rows < 1 || heads < 1 || head_dim < 1 || head_dim > 256)
+    return FD_ERR_SHAPE;
+  const size_t esz = dtype == FD_BF16 ? 2 : 4;
+  auto misaligned = [&](const void* ptr, size_t a) {
+    return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0;
+  };
+  fd::CombineParams p;
+  memset(&p, 0, sizeof(p));
+  for (int i = 0; i < n_parts; ++i) {
+    if (outs[i] == nullptr || lses[i] == nullptr) return FD_ERR_INVALID_ARG;
+    if (misaligned(outs[i], esz) || misaligned(lses[i], 4)) return FD_ERR_ALIGNMENT;
+    p.out[i] = outs[i];
+    p.lse[i] = lses[i];
+  }
+  if (misaligned(out, esz) || (lse != nullptr && misaligned(lse, 4))) return FD_ERR_ALIGNMENT;
+  p.n_parts = n_parts;
+  p.n_rollouts = n_rollouts;
+  p.Mq = rows;
+  p.H = heads;
+  p.d = head_dim;
+  p.esz = (int)esz;
+  p.dst = out;
+  p.dst_lse = lse;
+  return fd::cuda_status(fd::launch_combine(p, static_cast<cudaStream_t>(stream)));
 }
 
 fd_status fd_selftest_bounded_wait(fd_cache* cache, int32_t limit_ms,

@@ -30,6 +30,18 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
   return (uint32_t)(((uint64_t)n * f.m) >> 40);
 }
 
+// Valid cache frames of a rollout that committed n frames into a ring of S
+// sinks and W window slots: the slot prefix [0, nv).  Of these, shard `shard`
+// of N stores slots shard, shard + N, ... (local indices 0, 1, ...), which are
+// again a prefix of its local storage.
+__host__ __device__ __forceinline__ int valid_slots_global(int n, int S, int W) {
+  const int win = n - S > 0 ? n - S : 0;
+  return (n < S ? n : S) + (win < W ? win : W);
+}
+__host__ __device__ __forceinline__ int valid_slots_local(int nv, int N, int shard) {
+  return nv > shard ? (nv - shard + N - 1) / N : 0;
+}
+
 // Device pointers into one cache's storage plus its geometry.
 struct CacheView {
   uint8_t* k;
@@ -47,6 +59,10 @@ struct CacheView {
   int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz, nb;
   int Hkv;               // key/value heads (divides H)
   int Tv;                // video tokens per view (gh * gw); T = views * Tv
+  // Context-parallel shard: this cache stores ring slots s with s % N == shard
+  // at local index s / N; `slots` above counts local slots, S and W stay the
+  // ring's global sink and window counts, count[] the global frame counter.
+  int N, shard;
   double theta;
   uint64_t frame_bytes;  // Tf * Hkv * d * esz (one frame of K or V)
 };
@@ -100,6 +116,7 @@ struct AttnParams {
   int kv_group;          // H / Hkv: query head h reads key/value head h / kv_group
   int Tv;                // video tokens per view
   FastDiv div_Tv;
+  int N, shard;          // context-parallel shard of the key set (1, 0: whole)
   int G;                 // CTAs of the persistent launch
   int map_row0;          // layer * R: row offset of this layer in the cache maps
   int kb_row0;           // batch offset of rollout 0 in the rotated-block-key map
@@ -123,6 +140,19 @@ cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
                                    int n_rollouts, const void* k, void* out,
                                    cudaStream_t s);
 cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s);
+// bf16 output rows and log-sum-exp of rollouts with no key on this shard
+cudaError_t launch_attn_zero_keyless(const AttnParams& p, cudaStream_t s);
+// out = log-sum-exp weighted sum of n_parts partial results (context
+// parallelism); rows = n_rollouts * Mq, heads H, head dim d
+constexpr int kCombineMaxParts = 16;
+struct CombineParams {
+  const void* out[kCombineMaxParts];
+  const float* lse[kCombineMaxParts];
+  int n_parts, n_rollouts, Mq, H, d, esz;
+  void* dst;
+  float* dst_lse;
+};
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kc,
                                    const CUtensorMap& tm_vc,

@@ -111,3 +111,27 @@ def test_grouped_query_heads_validated(heads, kv_heads, status):
         hkv = kv_heads or heads
         kv = w.slots * w.frame_tokens * hkv * w.head_dim * 2
         assert lay.layer_kv_bytes == kv
+
+
+@pytest.mark.parametrize("shards,shard,status", [(2, 0, 0), (2, 1, 0), (7, 6, 0), (8, 0, 2),
+                                                 (2, 2, 2), (2, -1, 2), (0, 0, 0)])
+def test_shard_descriptor_validated(shards, shard, status):
+    # 480p ring: 1 sink + 6 window slots -> at most 7 shards
+    desc = fd.make_desc(SINGLE_480P.scaled(layers=1), shards=shards, shard=shard)
+    lay = fd.CacheLayout()
+    assert fd.load().fd_cache_get_layout(ctypes.byref(desc), ctypes.byref(lay)) == status
+    if status == 0:
+        n = max(shards, 1)
+        local = -(-7 // n)
+        assert lay.layer_kv_bytes == local * 1560 * 12 * 128 * 2
+
+
+def test_combine_host_errors():
+    lib = fd.load()
+    vp = ctypes.c_void_p
+    one = (vp * 1)(16)
+    assert lib.fd_attention_combine(0, one, one, 1, 1, 1, 8, 0, 16, None, None) == 2
+    assert lib.fd_attention_combine(17, one, one, 1, 1, 1, 8, 0, 16, None, None) == 2
+    assert lib.fd_attention_combine(1, one, one, 1, 1, 1, 8, 9, 16, None, None) == 3
+    assert lib.fd_attention_combine(1, None, one, 1, 1, 1, 8, 0, 16, None, None) == 1
+    assert lib.fd_attention_combine(1, one, one, 1, 1, 1, 8, 0, 17, None, None) == 8
