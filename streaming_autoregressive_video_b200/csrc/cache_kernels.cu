@@ -69,14 +69,24 @@ __global__ void cache_init_kernel(CacheView c) {
   if (threadIdx.x == 0) c.err[0] = 0;
 }
 
+// cos/sin of the kPairs rotation pairs from `pair0` on, for a token whose
+// t-section row is `tt_row` and whose grid coordinates are (hh, ww).
+template <int kPairs>
+__device__ __forceinline__ void rope_cs(float2 (&cs)[kPairs], int pair0, const CacheView& c,
+                                        const float2* tt_row, int hh, int ww) {
+#pragma unroll
+  for (int i = 0; i < kPairs; ++i) {
+    const int pair = pair0 + i;
+    if (pair < c.pt) cs[i] = __ldg(tt_row + pair);
+    else if (pair < c.pt + c.ph) cs[i] = __ldg(c.htab + hh * c.ph + (pair - c.pt));
+    else cs[i] = __ldg(c.wtab + ww * c.pw + (pair - c.pt - c.ph));
+  }
+}
+
 // 3D RoPE of the pairs held by one 16-byte vector (4 bf16 pairs or 2 fp32
-// pairs) whose first pair is `pair0`, for a token whose t-section cos/sin row
-// is `tt_row` and whose grid coordinates are (hh, ww).
+// pairs), given their cos/sin.
 template <typename Elem>
-__device__ __forceinline__ uint4 rotate16(uint4 u, int pair0,
-                                          const CacheView& c,
-                                          const float2* tt_row, int hh,
-                                          int ww) {
+__device__ __forceinline__ uint4 rotate16_cs(uint4 u, const float2 (&cs)[8 / sizeof(Elem)]) {
   constexpr int kPairs = 8 / sizeof(Elem);
   float vals[2 * kPairs];
   const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
@@ -92,14 +102,9 @@ __device__ __forceinline__ uint4 rotate16(uint4 u, int pair0,
   }
 #pragma unroll
   for (int i = 0; i < kPairs; ++i) {
-    const int pair = pair0 + i;
-    float2 cs;
-    if (pair < c.pt) cs = __ldg(tt_row + pair);
-    else if (pair < c.pt + c.ph) cs = __ldg(c.htab + hh * c.ph + (pair - c.pt));
-    else cs = __ldg(c.wtab + ww * c.pw + (pair - c.pt - c.ph));
     const float a = vals[2 * i], b = vals[2 * i + 1];
-    vals[2 * i] = a * cs.x - b * cs.y;
-    vals[2 * i + 1] = a * cs.y + b * cs.x;
+    vals[2 * i] = a * cs[i].x - b * cs[i].y;
+    vals[2 * i + 1] = a * cs[i].y + b * cs[i].x;
   }
   uint32_t o4[4];
   if constexpr (sizeof(Elem) == 2) {
@@ -113,6 +118,15 @@ __device__ __forceinline__ uint4 rotate16(uint4 u, int pair0,
     for (int i = 0; i < 4; ++i) o4[i] = __float_as_uint(vals[i]);
   }
   return make_uint4(o4[0], o4[1], o4[2], o4[3]);
+}
+
+// The same for a vector whose first pair is `pair0`, looking its cos/sin up.
+template <typename Elem>
+__device__ __forceinline__ uint4 rotate16(uint4 u, int pair0, const CacheView& c,
+                                          const float2* tt_row, int hh, int ww) {
+  float2 cs[8 / sizeof(Elem)];
+  rope_cs(cs, pair0, c, tt_row, hh, ww);
+  return rotate16_cs<Elem>(u, cs);
 }
 
 // One block copies a 64 KB chunk of one frame of K or V of one (layer,
@@ -258,6 +272,24 @@ __global__ void __launch_bounds__(256)
     const int ww = tok < c.T ? tv - hh * c.gw : 0;
     const uint4* src = reinterpret_cast<const uint4*>(in) + (size_t)row * row_chunks;
     uint4* dst = reinterpret_cast<uint4*>(out) + (size_t)row * row_chunks;
+    if (32 % cpr == 0) {
+      // every chunk a lane touches holds the same pairs (lane % cpr of each
+      // head row): their cos/sin are looked up once per token row, and up to
+      // 8 chunks per lane are loaded before any is rotated and stored
+      constexpr int kPairs = kPer / 2;
+      float2 cs[kPairs];
+      rope_cs(cs, (int)(lane % cpr) * kPairs, c, tt, hh, ww);
+      for (uint32_t base = lane; base < row_chunks; base += 32 * 8) {
+        uint4 buf[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (base + 32 * i < row_chunks) buf[i] = src[base + 32 * i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (base + 32 * i < row_chunks) dst[base + 32 * i] = rotate16_cs<Elem>(buf[i], cs);
+      }
+      continue;
+    }
     for (uint32_t ci = lane; ci < row_chunks; ci += 32) {
       const int pair0 = (int)(ci % cpr) * (kPer / 2);
       dst[ci] = rotate16<Elem>(src[ci], pair0, c, tt, hh, ww);
