@@ -427,9 +427,17 @@ __device__ __forceinline__ bool read_piece(const Meta* meta, int k, PieceInfo& p
   return true;
 }
 
-// KV iterations of ring entry k (what the MMA issuer needs of a piece).
-__device__ __forceinline__ bool read_piece_len(const Meta* meta, int k, int& n,
-                                               Shared* sh, int32_t* err, int site) {
+// Whether query tile 1 of pair b holds any query row (the last pair of a
+// head may end inside tile 0: tile 1 is then skipped altogether).
+__device__ __forceinline__ bool tile1_used(const AttnParams& p, int b) {
+  return b * 2 * kBM + kBM < p.Mq;
+}
+
+// KV iterations of ring entry k and whether its tile 1 is used (what the MMA
+// issuer needs of a piece).
+__device__ __forceinline__ bool read_piece_len(const Meta* meta, int k, int& n, bool& two,
+                                               const AttnParams& p, Shared* sh, int32_t* err,
+                                               int site) {
   const volatile PieceInfo* e = &meta->ring[k & 3];
   if (e->seq != k) {
     const uint64_t t0 = globaltimer_ns();
@@ -444,6 +452,7 @@ __device__ __forceinline__ bool read_piece_len(const Meta* meta, int k, int& n,
   }
   __threadfence_block();
   n = e->kv1 - e->kv0;
+  two = tile1_used(p, e->b);
   return true;
 }
 
@@ -647,23 +656,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         return wait_bar<true>(&sh->k_full[g % kKStages], (g / kKStages) & 1, sh, p.err,
                               kSiteMma);
       };
-      int g = 0;
+      // g counts the CTA's KV iterations (the K/V rings and tile 0's
+      // barriers), g1 only those of pieces whose tile 1 is used (its barriers)
+      int g = 0, g1 = 0;
       bool ok = true;
       for (int k = 0; k < n_pieces && ok; ++k) {
         int n = 0;
+        bool two = true;
         ok = wait_bar<true>(&sh->q_ready, k & 1, sh, p.err, kSiteMma) &&
-             read_piece_len(meta, k, n, sh, p.err, kSiteMma) && wait_k(g);
+             read_piece_len(meta, k, n, two, p, sh, p.err, kSiteMma) && wait_k(g);
         if (!ok) break;
         tc_fence_after();
         const int ks0 = g % kKStages;
         issue_s(0, ks0);
         mma_commit(&sh->s_full[0]);
-        issue_s(1, ks0);
-        mma_commit(&sh->s_full[1]);
+        if (two) {
+          issue_s(1, ks0);
+          mma_commit(&sh->s_full[1]);
+        }
         mma_commit(&sh->k_empty[ks0]);
         if (n == 1) mma_commit(&sh->q_empty);
         for (int jj = 0; jj < n; ++jj) {
-          const int gj = g + jj;
+          const int gj = g + jj, g1j = g1 + jj;
           const int vs = gj % kVStages;
           ok = wait_bar<true>(&sh->v_full[vs], (gj / kVStages) & 1, sh, p.err, kSiteMma) &&
                wait_bar<true>(&sh->p_full[0], gj & 1, sh, p.err, kSiteMma);
@@ -683,14 +697,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s(0, ks);
             mma_commit(&sh->s_full[0]);
           }
-          ok = wait_bar<true>(&sh->p_full[1], gj & 1, sh, p.err, kSiteMma);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(1, vs, jj > 0);
+          if (two) {
+            ok = wait_bar<true>(&sh->p_full[1], g1j & 1, sh, p.err, kSiteMma);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(1, vs, jj > 0);
+          }
           mma_commit(&sh->v_empty[vs]);
           if (more) {
-            issue_s(1, ks);
-            mma_commit(&sh->s_full[1]);
+            if (two) {
+              issue_s(1, ks);
+              mma_commit(&sh->s_full[1]);
+            }
             mma_commit(&sh->k_empty[ks]);
             if (jj + 2 == n) mma_commit(&sh->q_empty);  // last S products of the piece
           }
@@ -698,6 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mma_commit(&sh->o_full);
         g += n;
+        if (two) g1 += n;
       }
       if (!ok) {
         // wait for the tensor core to finish what was issued
@@ -767,21 +786,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
     const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
     const float sl2 = p.scale_log2;
-    int g = 0;
+    int g = 0;  // KV iterations this warpgroup's tile has run (its barriers' phases)
     uint32_t n_part = 0;
     bool ok = true;
     uint32_t sa[64], sb[64];
     for (int k = 0; k < n_pieces && ok; ++k) {
       int n, kv0, nt1, n1, n2;
       {
-        // the piece's first S product of this tile is done, so its ring
-        // entry is out
         PieceInfo pi;
-        ok = __all_sync(0xffffffffu,
-                        wait_bar<true>(&sh->s_full[x], g & 1, sh, p.err, kSiteSoftmax) &&
-                            read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
+        ok = __all_sync(0xffffffffu, read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
         if (!ok) break;
-        n = pi.kv1 - pi.kv0;
+        // tile 1 of a head's last pair may hold no query row: the tensor core
+        // computes nothing for it and this warpgroup skips the piece's loop
+        const bool used = x == 0 || tile1_used(p, pi.b);
+        n = used ? pi.kv1 - pi.kv0 : 0;
         kv0 = pi.kv0;
         nt1 = pi.nt1;
         n1 = pi.n1;
