@@ -256,3 +256,31 @@ def test_block_captured_in_cuda_graph_matches_eager():
     assert torch.equal(pe, pg) and torch.equal(ce, cg)
     assert torch.equal(ke, kg) and torch.equal(ve, vg)
     assert fd.fd_get_device_error(graphed.cache) == 0
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_random_shapes_rollout(seed):
+    """Seeded random geometries (heads and key/value heads, grid, views, action
+    tokens, block / sink / window sizes, rollouts, dtype and head size), a
+    short rollout with ragged commits through the cache, every call against
+    the oracle and the cache bit-exact."""
+    rng = np.random.default_rng(1000 + seed)
+    heads = int(rng.integers(1, 5))
+    kv = int(rng.choice([h for h in range(1, heads + 1) if heads % h == 0]))
+    F = int(rng.integers(1, 4))
+    dtype = "f32" if seed % 4 == 3 else "bf16"
+    d = int(rng.choice([32, 64])) if dtype == "f32" else 128
+    w = Workload(f"random-{seed}", layers=1, rollouts=int(rng.integers(1, 4)), heads=heads,
+                 head_dim=d, grid_h=int(rng.integers(1, 7)), grid_w=int(rng.integers(1, 10)),
+                 action_tokens=int(rng.choice([0, 1, 3])), block_frames=F,
+                 sink_frames=int(rng.integers(0, 3)), window_frames=F + int(rng.integers(0, 3)),
+                 steps=1, blocks=int(rng.integers(3, 6)), dtype=dtype,
+                 kv_heads=kv if kv != heads else 0, views=int(rng.choice([1, 1, 2])))
+    ls = Lockstep(w)
+    for blk in range(w.blocks):
+        q, k, v = block_inputs(w, (71, seed, blk), w.rollouts)
+        ls.attention(0, q, k, v, what=f"{w} blk {blk}")
+        frames = [int(x) for x in rng.integers(0, F + 1, w.rollouts)]
+        ls.commit([0], [k], [v], frames=frames)
+        ls.check_cache_exact()
+    assert fd.fd_get_device_error(ls.cache) == 0
