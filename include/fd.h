@@ -196,8 +196,11 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * For rollout r the key set is its valid cache slots (sinks + window, frame
  * positions from the slot table) plus all F*Tf block tokens at t = n_r + f.
  * The cache is read only: call it once per denoising step, then commit.
- * bf16 runs on tcgen05 tensor cores (fp32 accumulation, P rounded to bf16),
- * f32 on CUDA cores in fp32 (no TF32).  Tensor bases must be 16-byte aligned.
+ * bf16 with head_dim 128 runs on tcgen05 tensor cores (fp32 accumulation, P
+ * rounded to bf16); f32, and bf16 with head_dim 32, 64 or 96, on CUDA cores
+ * in fp32 arithmetic (no TF32; bf16 output rounded once).  Other head sizes
+ * return FD_ERR_UNSUPPORTED before any launch.  Tensor bases must be 16-byte
+ * aligned.
  * The bf16 kernel is persistent (one CTA per multiprocessor, at most 148)
  * and splits the call's KV iterations evenly over its CTAs; it returns
  * FD_ERR_UNSUPPORTED when n_rollouts x H x ceil(F*T/256) x (ceil((S+W)*Tf

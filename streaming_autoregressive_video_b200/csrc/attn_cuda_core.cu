@@ -1,4 +1,4 @@
-// fp32 block-causal chunk attention on CUDA cores (no TF32).
+// Block-causal chunk attention on CUDA cores, arithmetic in fp32 (no TF32).
 //
 // Same definition as the tensor-core kernel: for every query of the block,
 // softmax(q' k'^T / sqrt(d)) v over the rollout's valid cache tokens (sinks +
@@ -6,13 +6,16 @@
 // RoPE applied to q and k as they are staged ("Cosmos3-H-Dreams" model card,
 // Model Architecture: block-causal student with a KV cache; AlpaDreams GTC
 // 2026 write-up, section VII: next frame from historical clean frames and the
-// current noisy frame).  Used for fp32 caches, where the tolerance leaves no
-// room for TF32 rounding.
+// current noisy frame).  It serves fp32 caches, where the tolerance leaves no
+// room for TF32 rounding, and bf16 caches whose head size the tensor-core
+// kernel does not take (d = 32, 64, 96): bf16 values are widened to fp32 as
+// they are staged and the output is rounded to bf16 once, at the end.
 //
 // One CTA = (query tile of 32 rows, head, rollout); 8 warps x 4 rows.  Keys
 // are staged 64 at a time in shared memory, rotated in fp32; within a warp
 // lane j scores key j, then the warp forms the online softmax and each lane
 // accumulates d/32 output dimensions.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -40,9 +43,24 @@ __device__ __forceinline__ float2 rope_cs(const AttnParams& p,
   return p.wtab[kc.w * p.pw + (pair - p.pt - p.ph)];
 }
 
-template <int D>
+// Elements (2i, 2i+1) of a stored row as fp32: fp32 storage, or bf16 bit
+// patterns (the lower address in the low half of the 32-bit word).
+__device__ __forceinline__ float2 load_pair(const float* x) {
+  return *reinterpret_cast<const float2*>(x);
+}
+__device__ __forceinline__ float2 load_pair(const uint16_t* x) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(x);
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ void store_elem(float* x, float v) { *x = v; }
+__device__ __forceinline__ void store_elem(uint16_t* x, float v) {
+  *x = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// Elem: float (fp32 cache) or uint16_t (bf16 bit patterns)
+template <typename Elem, int D>
 __global__ void __launch_bounds__(kWarps * 32)
-    attn_f32_kernel(AttnParams p) {
+    attn_cuda_core_kernel(AttnParams p) {
   constexpr int kPerLane = D / 32;
   extern __shared__ float sm[];
   float* Qs = sm;                          // [kRows][D]
@@ -55,11 +73,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int nv = valid_slots_local(valid_slots_global(p.count[r], p.S, p.W), p.N, p.shard);
   const int n1 = nv * p.Tf, n2 = p.shard == 0 ? p.F * p.Tf : 0;
   const float2* tt = p.ttab + (size_t)r * (p.slots + p.F) * p.pt;
-  const float* qg = reinterpret_cast<const float*>(p.q);
-  const float* kg = reinterpret_cast<const float*>(p.k);
-  const float* vg = reinterpret_cast<const float*>(p.v);
-  const float* kcg = reinterpret_cast<const float*>(p.kc);
-  const float* vcg = reinterpret_cast<const float*>(p.vc);
+  const Elem* qg = static_cast<const Elem*>(p.q);
+  const Elem* kg = static_cast<const Elem*>(p.k);
+  const Elem* vg = static_cast<const Elem*>(p.v);
+  const Elem* kcg = reinterpret_cast<const Elem*>(p.kc);
+  const Elem* vcg = reinterpret_cast<const Elem*>(p.vc);
 
   // rotated queries
   for (int e = threadIdx.x; e < kRows * (D / 2); e += blockDim.x) {
@@ -69,10 +87,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (q < p.Mq) {
       const int f = q / p.T, tok = (q - f * p.T) % p.Tv;  // inside its view
       const KeyCoord kc{p.slots + f, tok / p.gw, tok % p.gw};
-      const float* src = qg + (((size_t)r * p.Mq + q) * p.H + h) * D + 2 * pair;
+      const float2 x = load_pair(qg + (((size_t)r * p.Mq + q) * p.H + h) * D + 2 * pair);
       const float2 cs = rope_cs(p, tt, pair, kc);
-      a = src[0] * cs.x - src[1] * cs.y;
-      b = src[0] * cs.y + src[1] * cs.x;
+      a = x.x * cs.x - x.y * cs.y;
+      b = x.x * cs.y + x.y * cs.x;
     }
     Qs[row * D + 2 * pair] = a;
     Qs[row * D + 2 * pair + 1] = b;
@@ -105,12 +123,12 @@ __global__ void __launch_bounds__(kWarps * 32)
             : (((size_t)r * p.F * p.Tf + key) * p.Hkv + hk) * D + 2 * pair;
         // keys arrive rotated: cached frames were rotated when committed, the
         // block's keys once per call before this kernel
-        const float* ks = (seg1 ? kcg : kg) + off;
-        const float* vs = (seg1 ? vcg : vg) + off;
-        a = ks[0];
-        b = ks[1];
-        va = vs[0];
-        vb = vs[1];
+        const float2 kx = load_pair((seg1 ? kcg : kg) + off);
+        const float2 vx = load_pair((seg1 ? vcg : vg) + off);
+        a = kx.x;
+        b = kx.y;
+        va = vx.x;
+        vb = vx.y;
       }
       Ks[kr * (D + 1) + 2 * pair] = a;
       Ks[kr * (D + 1) + 2 * pair + 1] = b;
@@ -157,48 +175,54 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
   }
 
-  float* outg = reinterpret_cast<float*>(p.out);
+  Elem* outg = static_cast<Elem*>(p.out);
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp; ++i) {
     const int q = q0 + warp * kRowsPerWarp + i;
     if (q >= p.Mq) continue;
     // a shard may hold no key of this rollout: zero row, log-sum-exp -inf
     const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
-    float* dst = outg + (((size_t)r * p.Mq + q) * p.H + h) * D;
+    Elem* dst = outg + (((size_t)r * p.Mq + q) * p.H + h) * D;
 #pragma unroll
-    for (int e = 0; e < kPerLane; ++e) dst[lane + 32 * e] = o[i][e] * inv;
+    for (int e = 0; e < kPerLane; ++e) store_elem(dst + lane + 32 * e, o[i][e] * inv);
     if (p.lse != nullptr && lane == 0)
       p.lse[((size_t)r * p.H + h) * p.Mq + q] = l[i] > 0.f ? m[i] + logf(l[i]) : -INFINITY;
   }
 }
 
-template <int D>
+template <typename Elem, int D>
 cudaError_t launch_d(const AttnParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (kRows * D + kKeys * (D + 1) + kKeys * D);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(
-        attn_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attn_cuda_core_kernel<Elem, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
         (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 grid((p.Mq + kRows - 1) / kRows, p.H, p.n_rollouts);
-  attn_f32_kernel<D><<<grid, kWarps * 32, smem, s>>>(p);
+  attn_cuda_core_kernel<Elem, D><<<grid, kWarps * 32, smem, s>>>(p);
   count_launch(1);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s) {
+template <typename Elem>
+cudaError_t launch_elem(const AttnParams& p, cudaStream_t s) {
   switch (p.d) {
-    case 32: return launch_d<32>(p, s);
-    case 64: return launch_d<64>(p, s);
-    case 96: return launch_d<96>(p, s);
-    case 128: return launch_d<128>(p, s);
+    case 32: return launch_d<Elem, 32>(p, s);
+    case 64: return launch_d<Elem, 64>(p, s);
+    case 96: return launch_d<Elem, 96>(p, s);
+    case 128: return launch_d<Elem, 128>(p, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_attn_cuda_core(const AttnParams& p, int esz, cudaStream_t s) {
+  if (esz == 2) return launch_elem<uint16_t>(p, s);
+  return launch_elem<float>(p, s);
 }
 
 }  // namespace fd

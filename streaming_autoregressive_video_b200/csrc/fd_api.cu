@@ -448,11 +448,11 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  if (cache->desc.dtype == FD_F32) {
-    if (c.d % 32 != 0 || c.d > 128) return FD_ERR_UNSUPPORTED;
-  } else if (c.d != 128 || !cache->have_maps) {
+  // bf16 with d = 128 runs on the tensor cores; fp32, and bf16 of the other
+  // head sizes, on CUDA cores
+  const bool tensor_cores = cache->desc.dtype == FD_BF16 && c.d == 128;
+  if (tensor_cores ? !cache->have_maps : (c.d % 32 != 0 || c.d > 128))
     return FD_ERR_UNSUPPORTED;
-  }
   // a shard's result is only usable with its log-sum-exp (to be combined)
   if (c.N > 1 && lse == nullptr) return FD_ERR_INVALID_ARG;
   // the block's keys belong to shard 0; other shards never read them
@@ -460,7 +460,7 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
     st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
     if (st != FD_OK) return st;
   }
-  if (cache->desc.dtype == FD_F32) return fd::cuda_status(fd::launch_attn_f32(p, s));
+  if (!tensor_cores) return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
   CUtensorMap tm_q, tm_vb, tm_kb_work;
   const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
   if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||

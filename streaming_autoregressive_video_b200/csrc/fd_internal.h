@@ -139,7 +139,9 @@ cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
 cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
                                    int n_rollouts, const void* k, void* out,
                                    cudaStream_t s);
-cudaError_t launch_attn_f32(const AttnParams& p, cudaStream_t s);
+// attention on CUDA cores in fp32 arithmetic: fp32 caches of any head size
+// d in {32, 64, 96, 128}; bf16 caches (esz = 2) whose d is not 128
+cudaError_t launch_attn_cuda_core(const AttnParams& p, int esz, cudaStream_t s);
 // bf16 output rows and log-sum-exp of rollouts with no key on this shard
 cudaError_t launch_attn_zero_keyless(const AttnParams& p, cudaStream_t s);
 // out = log-sum-exp weighted sum of n_parts partial results (context

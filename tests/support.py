@@ -51,19 +51,33 @@ def krot_view(cache, w):
     return cache.storage[lay.krot:lay.krot + n_kv * esz].view(kv_dt).view(shape)
 
 
+def rotated_bound(want: np.ndarray, raw: np.ndarray, dtype: str) -> np.ndarray:
+    """Error bound of a stored rotated value against the fp64 rotation.
+
+    The kernels rotate in fp32 with cos/sin rounded once to fp32: the value
+    before storage is off by at most about 3 * 2^-24 * (|x0| + |x1|) of its
+    input pair (x0, x1), which matters where the rotation cancels.  A bf16
+    value is then rounded once more (half an ulp, at most 2^-8 of the value).
+    The bound takes 2^-21 * (|x0| + |x1|) for the fp32 part (a factor 2
+    over the estimate)."""
+    x = np.abs(np.asarray(raw, dtype=np.float64))
+    pair = np.repeat(x[..., 0::2] + x[..., 1::2], 2, axis=-1)
+    if dtype == "bf16":
+        return np.abs(want) * 2.0 ** -8 + pair * 2.0 ** -21
+    return np.abs(want) * 1e-6 + 1e-6
+
+
 def check_rotated(got_storage: np.ndarray, raw: np.ndarray, t, w, what=""):
     """got = RoPE(raw) at frame positions t (one entry per frame), within one
-    rounding to the storage dtype of the fp64 rotation."""
+    rounding to the storage dtype of the fp32 rotation (rotated_bound)."""
     h, ww = oracle.token_coords(w.frame_tokens, w.tokens, w.grid_w, w.view_tokens)
     t = np.asarray(t, dtype=np.float64)[:, None]
     ang = oracle.rope_angles(t, h[None, :], ww[None, :], w.head_dim, w.theta)[:, :, None, :]
-    want = oracle.rope_rotate(oracle.values_f64(raw, w.dtype), ang)
+    raw64 = oracle.values_f64(raw, w.dtype)
+    want = oracle.rope_rotate(raw64, ang)
     got = oracle.values_f64(got_storage, w.dtype)
     err = np.abs(got - want)
-    if w.dtype == "bf16":
-        bound = np.abs(want) * 2.0 ** -8 + 1e-30
-    else:
-        bound = np.abs(want) * 1e-6 + 1e-6
+    bound = rotated_bound(want, raw64, w.dtype)
     assert np.all(err <= bound), f"{what}: rotated keys off by {float(err.max()):.3g}"
 
 

@@ -11,7 +11,8 @@ from streaming_autoregressive_video_b200 import binding as fd
 from streaming_autoregressive_video_b200 import synth
 from streaming_autoregressive_video_b200.workloads import TINY_F32, Workload
 
-from support import Lockstep, block_inputs, compare, to_device, to_host, views
+from support import (Lockstep, block_inputs, compare, rotated_bound, to_device, to_host,
+                     views)
 
 pytestmark = pytest.mark.gpu
 
@@ -70,11 +71,12 @@ def test_rope3d_matches_oracle(dtype, tokens):
         n = ls.orc[1][r].n
         t = (n + np.arange(w.block_frames))[:, None]
         ang = oracle.rope_angles(t, h[None, :], ww[None, :], w.head_dim, w.theta)[:, :, None, :]
-        want = oracle.rope_rotate(oracle.values_f64(x[r], dtype), ang)
+        raw = oracle.values_f64(x[r], dtype)
+        want = oracle.rope_rotate(raw, ang)
         err = np.abs(got[r] - want)
         if dtype == "bf16":
-            # one bf16 rounding of the rotated value
-            assert np.all(err <= np.abs(want) * 2.0 ** -8 + 1e-30)
+            # one bf16 rounding of the fp32 rotation
+            assert np.all(err <= rotated_bound(want, raw, dtype))
         else:
             assert err.max() <= 1e-5
 
@@ -95,17 +97,41 @@ def test_attention_f32_tiny_rollout(kv_heads, views):
     assert fd.fd_get_device_error(ls.cache) == 0
 
 
+@pytest.mark.parametrize("d,shape", [
+    (64, dict()),                                           # Tf=156, Mq=312
+    (64, dict(heads=4, kv_heads=2, action_tokens=4, views=2)),  # GQA, actions, 2 views
+    (32, dict(rollouts=2, sink_frames=2, window_frames=2)),     # sinks straddled
+    (96, dict(grid_h=5, grid_w=7, action_tokens=1)),        # d/2 = 48 pairs: t/h/w = 16/16/16
+])
+def test_attention_bf16_cuda_core_head_sizes(d, shape):
+    """bf16 caches with d != 128 run on the CUDA-core kernel (fp32 arithmetic
+    on the stored bf16 values): a rollout through empty, partial, full and
+    wrapped cache states against the oracle at the bf16 tolerance."""
+    w = SMALL.scaled(head_dim=d, blocks=5, **shape)
+    ls = Lockstep(w)
+    for blk in range(w.blocks):
+        for l in range(w.layers):
+            q, k, v = block_inputs(w, (8, blk, l), w.rollouts)
+            ls.attention(l, q, k, v, what=f"d {d} blk {blk} layer {l}")
+        _commit_block(ls, w, 700 + blk)
+        ls.check_cache_exact()
+        ls.check_rotated_keys()
+    assert fd.fd_get_device_error(ls.cache) == 0
+
+
 def test_unsupported_bf16_head_dim_is_refused_cleanly():
-    """The tensor-core kernel handles d = 128 only: a bf16 cache with d = 64
-    commits and rotates, but attention returns FD_ERR_UNSUPPORTED without
-    launching anything, and the context stays usable."""
-    w = Workload("bf16-d64", layers=1, rollouts=1, heads=2, head_dim=64, grid_h=3, grid_w=4,
+    """A head size that no attention kernel takes (d = 48: a multiple of 8, so
+    the cache accepts it, but not of 32): the cache commits and rotates, but
+    attention returns FD_ERR_UNSUPPORTED without launching anything, and the
+    context stays usable."""
+    w = Workload("bf16-d48", layers=1, rollouts=1, heads=2, head_dim=48, grid_h=3, grid_w=4,
                  action_tokens=0, block_frames=1, sink_frames=0, window_frames=2, steps=1,
                  blocks=1, dtype="bf16")
     ls = Lockstep(w)
     q, k, v = block_inputs(w, (7, 0), 1)
     _commit_block(ls, w, 500)
     ls.check_cache_exact()
+    ls.check_rotated_keys()
     out = torch.empty((1, w.queries, w.heads, w.head_dim), dtype=torch.int16, device="cuda")
     before = fd.fd_launch_count()
     with pytest.raises(fd.FdError) as e:
