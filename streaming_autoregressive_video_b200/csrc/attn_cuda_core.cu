@@ -193,14 +193,12 @@ __global__ void __launch_bounds__(kWarps * 32)
 template <typename Elem, int D>
 cudaError_t launch_d(const AttnParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float) * (kRows * D + kKeys * (D + 1) + kKeys * D);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(
-        attn_cuda_core_kernel<Elem, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce attr;
+  cudaError_t e = once_per_device(attr, [smem] {
+    return cudaFuncSetAttribute(attn_cuda_core_kernel<Elem, D>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((p.Mq + kRows - 1) / kRows, p.H, p.n_rollouts);
   attn_cuda_core_kernel<Elem, D><<<grid, kWarps * 32, smem, s>>>(p);
   count_launch(1);

@@ -1049,21 +1049,20 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kb,
                                    const CUtensorMap& tm_vb,
                                    const AttnParams& p, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
+  static PerDeviceOnce attr;
+  cudaError_t e = once_per_device(attr, [] {
     // The warpgroup register split (setmaxnreg) assumes the block launches
     // with exactly 128 registers per thread; refuse to launch otherwise, as
     // the increase would wait forever for registers that do not exist.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bf16_d128_sm100);
-    if (e != cudaSuccess) return e;
+    cudaError_t err = cudaFuncGetAttributes(&fa, attn_bf16_d128_sm100);
+    if (err != cudaSuccess) return err;
     if (fa.numRegs != 128) return cudaErrorNotSupported;
-    e = cudaFuncSetAttribute(attn_bf16_d128_sm100,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemMax);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return cudaFuncSetAttribute(attn_bf16_d128_sm100,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemMax);
+  });
+  if (e != cudaSuccess) return e;
   const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
                                         (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
   const size_t smem = kSmemFixed + tab;

@@ -21,16 +21,15 @@ namespace {
 // device address: the address comes from cudaGetSymbolAddress below.
 __device__ __align__(256) uint8_t g_block_work[FD_STATIC_WORK_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void* g_work_addr[kMaxDevices] = {};
+void* g_work_addr[fd::kMaxDevices] = {};
 
 // Device address of g_block_work on the current device: looked up once per
 // device, with that device current, on the first call made on it.
 fd_status work_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FD_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return FD_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= fd::kMaxDevices) return FD_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_work_addr[dev] == nullptr) {
     void* p = nullptr;

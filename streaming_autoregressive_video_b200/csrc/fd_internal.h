@@ -5,9 +5,34 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "fd.h"
 
 namespace fd {
+
+// Devices one process may drive (ordinals 0 .. kMaxDevices-1).
+constexpr int kMaxDevices = 64;
+
+// One-time setup per device.  Kernel attributes (cudaFuncSetAttribute) act
+// on the current device only, so a process that drives several GPUs sets
+// them once on each.  setup() runs until it succeeds once on a device; two
+// threads may both run it on first use (it must be idempotent).
+struct PerDeviceOnce {
+  std::atomic<bool> done[kMaxDevices];
+};
+
+template <typename Setup>
+cudaError_t once_per_device(PerDeviceOnce& once, Setup&& setup) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (once.done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess) once.done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 // Device error word: bits 0-7 kind, bits 8-15 site.
 enum DevErrKind : int32_t { kDevErrTimeout = 1, kDevErrArgument = 2 };
