@@ -45,6 +45,10 @@
  * Conventions for every call:
  *   - all pointers to tensors are DEVICE pointers on the device that owns the
  *     cache storage; host arrays are marked (host);
+ *   - a call on a cache needs that cache's device to be current (otherwise
+ *     FD_ERR_INVALID_ARG, nothing launched); one process may drive caches on
+ *     several devices (ordinals below 64), switching the current device
+ *     between calls;
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default);
  *     every call only enqueues work on it: no host synchronisation, no
  *     allocation, so a block of calls can be captured in a CUDA graph;
