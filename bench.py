@@ -463,7 +463,7 @@ def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
                 with torch.cuda.stream(d2h):
                     hout[l].copy_(dout[b], non_blocking=True)
                 freed[b].record(d2h)
-                h2d_bytes += 3 * hq[l].numel() * 2
+                h2d_bytes += (hq[l].numel() + hk[l].numel() + hv[l].numel()) * 2
                 d2h_bytes += hout[l].numel() * 2
                 i += 1
         fd.fd_cache_commit(cache, 0, L, R, klast, vlast, stream=stream)

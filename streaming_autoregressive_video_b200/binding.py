@@ -118,6 +118,48 @@ def _ptr(t) -> Optional[int]:
     return t.data_ptr()
 
 
+def _dev_ptr(t, nbytes: int, where: str, name: str, device=None) -> Optional[int]:
+    """Address of the tensor argument `name` after checking that the kernels
+    may read or write `nbytes` bytes there: a contiguous CUDA tensor (on
+    `device` when given) of at least that many bytes.  The C entry points take
+    bare addresses and cannot check this themselves; a host or short buffer
+    would otherwise reach a kernel.  Raw integer addresses pass unchecked (the
+    caller vouches for them), None stays None."""
+    if t is None or isinstance(t, int):
+        return t
+    if not getattr(t, "is_cuda", False):
+        raise FdError(1, f"{where}: {name} is not a CUDA tensor")
+    if device is not None and t.device != device:
+        raise FdError(1, f"{where}: {name} is on {t.device}, the cache on {device}")
+    if not t.is_contiguous():
+        raise FdError(1, f"{where}: {name} is not contiguous")
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise FdError(2, f"{where}: {name} holds {have} bytes, needs {nbytes}")
+    return t.data_ptr()
+
+
+class _Geom:
+    """Per-call tensor sizes of a cache's geometry (bytes per rollout)."""
+
+    def __init__(self, desc: "CacheDesc"):
+        self.esz = 2 if desc.dtype == FD_BF16 else 4
+        views = desc.num_views or 1
+        self.T = views * desc.grid_h * desc.grid_w
+        self.Tf = self.T + desc.action_tokens
+        self.F = desc.block_frames
+        self.H = desc.num_heads
+        self.Hkv = desc.num_kv_heads or desc.num_heads
+        self.d = desc.head_dim
+        self.q = self.F * self.T * self.H * self.d * self.esz      # q and out
+        self.kv = self.F * self.Tf * self.Hkv * self.d * self.esz  # block k and v
+        self.lse = self.H * self.F * self.T * 4
+
+
+def _device_of(cache: "Cache"):
+    return getattr(cache.storage, "device", None)
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -194,14 +236,26 @@ def fd_cache_reset(cache: Cache, rollout_ids: Sequence[int], stream=None) -> Non
 
 def fd_rope3d(cache: Cache, layer: int, n_rollouts: int, x, tokens_per_frame: int,
               heads: int, stream=None) -> None:
-    _check(load().fd_rope3d(cache.handle, layer, n_rollouts, _ptr(x), tokens_per_frame,
+    g = _Geom(cache.desc)
+    n = max(n_rollouts, 0) * g.F * max(tokens_per_frame, 0) * max(heads, 0) * g.d * g.esz
+    xp = _dev_ptr(x, n, "fd_rope3d", "x", _device_of(cache))
+    _check(load().fd_rope3d(cache.handle, layer, n_rollouts, xp, tokens_per_frame,
                             heads, _stream(stream)), "fd_rope3d")
+
+
+def _attention_ptrs(cache: Cache, n_rollouts: int, q, k, v, out, lse, where: str):
+    g = _Geom(cache.desc)
+    n = max(n_rollouts, 0)
+    dev = _device_of(cache)
+    return (_dev_ptr(q, n * g.q, where, "q", dev), _dev_ptr(k, n * g.kv, where, "k", dev),
+            _dev_ptr(v, n * g.kv, where, "v", dev), _dev_ptr(out, n * g.q, where, "out", dev),
+            _dev_ptr(lse, n * g.lse, where, "lse", dev))
 
 
 def fd_block_attention(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,
                        lse=None, stream=None) -> None:
-    _check(load().fd_block_attention(cache.handle, layer, n_rollouts, _ptr(q), _ptr(k),
-                                     _ptr(v), _ptr(out), _ptr(lse), _stream(stream)),
+    ptrs = _attention_ptrs(cache, n_rollouts, q, k, v, out, lse, "fd_block_attention")
+    _check(load().fd_block_attention(cache.handle, layer, n_rollouts, *ptrs, _stream(stream)),
            "fd_block_attention")
 
 
@@ -212,8 +266,8 @@ STATIC_WORK_BYTES = 32 << 20
 def fd_block_attention_static(cache: Cache, layer: int, n_rollouts: int, q, k, v, out,
                               lse=None, stream=None) -> None:
     """fd_block_attention with its work area in the library's static array."""
-    _check(load().fd_block_attention_static(cache.handle, layer, n_rollouts, _ptr(q),
-                                            _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+    ptrs = _attention_ptrs(cache, n_rollouts, q, k, v, out, lse, "fd_block_attention_static")
+    _check(load().fd_block_attention_static(cache.handle, layer, n_rollouts, *ptrs,
                                             _stream(stream)),
            "fd_block_attention_static")
 
@@ -222,8 +276,19 @@ def fd_cache_commit(cache: Cache, layer_begin: int, layer_end: int, n_rollouts: 
                     k_list, v_list, frames: Optional[Sequence[int]] = None,
                     stream=None) -> None:
     nl = layer_end - layer_begin
-    kp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in k_list])
-    vp = (ctypes.c_void_p * nl)(*[_ptr(t) for t in v_list])
+    if nl < 1 or len(k_list) != nl or len(v_list) != nl:
+        raise FdError(1, f"fd_cache_commit: {len(k_list)} k and {len(v_list)} v tensors "
+                         f"for {nl} layers")
+    if frames is not None and len(frames) != n_rollouts:
+        raise FdError(1, f"fd_cache_commit: {len(frames)} frame counts for {n_rollouts} "
+                         "rollouts")
+    g = _Geom(cache.desc)
+    nb = max(n_rollouts, 0) * g.kv
+    dev = _device_of(cache)
+    kp = (ctypes.c_void_p * nl)(*[_dev_ptr(t, nb, "fd_cache_commit", f"k[{i}]", dev)
+                                  for i, t in enumerate(k_list)])
+    vp = (ctypes.c_void_p * nl)(*[_dev_ptr(t, nb, "fd_cache_commit", f"v[{i}]", dev)
+                                  for i, t in enumerate(v_list)])
     fr = None if frames is None else (ctypes.c_int32 * n_rollouts)(*frames)
     _check(load().fd_cache_commit(cache.handle, layer_begin, layer_end, n_rollouts, fr,
                                   kp, vp, _stream(stream)), "fd_cache_commit")
@@ -237,7 +302,9 @@ def fd_cache_frames(cache: Cache, layer: int, rollout: int) -> int:
 
 
 def fd_exp2_selfcheck(x, y, stream=None) -> None:
-    _check(load().fd_exp2_selfcheck(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+    xp = _dev_ptr(x, x.numel() * 4, "fd_exp2_selfcheck", "x")
+    yp = _dev_ptr(y, 3 * x.numel() * 4, "fd_exp2_selfcheck", "y", x.device)
+    _check(load().fd_exp2_selfcheck(xp, yp, x.numel(), _stream(stream)),
            "fd_exp2_selfcheck")
 
 
@@ -250,10 +317,20 @@ def fd_attention_combine(outs, lses, out, lse=None, stream=None) -> None:
     """out (and lse) = log-sum-exp combination of per-part rows `outs` [R][Mq][H][d]
     with their log-sum-exps `lses` [R][H][Mq] (device tensors)."""
     n = len(outs)
+    if len(lses) != n:
+        raise FdError(1, f"fd_attention_combine: {n} row tensors, {len(lses)} lse tensors")
     R, Mq, H, d = out.shape
     dt = FD_BF16 if out.element_size() == 2 else FD_F32
-    op = (ctypes.c_void_p * n)(*[_ptr(t) for t in outs])
-    lp = (ctypes.c_void_p * n)(*[_ptr(t) for t in lses])
+    rows = R * Mq * H * d * out.element_size()
+    lse_bytes = R * H * Mq * 4
+    w = "fd_attention_combine"
+    dev = getattr(out, "device", None)
+    op = (ctypes.c_void_p * n)(*[_dev_ptr(t, rows, w, f"outs[{i}]", dev)
+                                 for i, t in enumerate(outs)])
+    lp = (ctypes.c_void_p * n)(*[_dev_ptr(t, lse_bytes, w, f"lses[{i}]", dev)
+                                 for i, t in enumerate(lses)])
+    _dev_ptr(out, rows, w, "out")
+    _dev_ptr(lse, lse_bytes, w, "lse", dev)
     _check(load().fd_attention_combine(n, op, lp, R, Mq, H, d, dt, _ptr(out), _ptr(lse),
                                        _stream(stream)), "fd_attention_combine")
 
