@@ -158,6 +158,42 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------
+# Workload description (both arms print the same config)
+# --------------------------------------------------------------------------
+def prefill_frames(w, rank):
+    """Frames committed per rollout before the timed block: the window is
+    filled (steady state), or for a ragged workload each rollout's fill is
+    drawn from the replica's seed."""
+    from streaming_autoregressive_video_b200 import synth
+    if w.ragged_window:
+        lo, hi = w.ragged_window
+        return [int(x) for x in
+                synth.ragged_fill(synth.seed_of(replica_seed_base(rank), 3), w.rollouts, lo, hi)]
+    return [w.block_frames * (-(-w.slots // w.block_frames) + 1)] * w.rollouts
+
+
+def keys_per_rollout(w, frames):
+    """Keys of one attention call per rollout: valid cache frames (sinks,
+    then at most W window frames) plus the block, Tf tokens each."""
+    S, W = w.sink_frames, w.window_frames
+    return [(min(n, S) + min(max(n - S, 0), W) + w.block_frames) * w.frame_tokens
+            for n in frames]
+
+
+def workload_config(w, world, rank=0):
+    nk = keys_per_rollout(w, prefill_frames(w, rank))
+    return {"workload": w.name, "rollouts_per_gpu": w.rollouts, "layers": w.layers,
+            "heads": w.heads, "kv_heads": w.hkv, "head_dim": w.head_dim,
+            "views": w.views, "grid": f"{w.grid_h}x{w.grid_w}",
+            "action_tokens": w.action_tokens, "block_frames": w.block_frames,
+            "sink_frames": w.sink_frames, "window_frames": w.window_frames,
+            "denoise_steps": w.steps, "keys_per_rollout": nk[0] if len(set(nk)) == 1 else nk,
+            "l2": "inputs larger than L2: every step reads all layers' caches and "
+                  "fresh q/k/v per (step, layer)",
+            "parallelism": f"replicas x{world}"}
+
+
+# --------------------------------------------------------------------------
 # CPU oracle timings (baseline / reference arm)
 # --------------------------------------------------------------------------
 def oracle_call_setup(w, heads):
@@ -245,7 +281,7 @@ def run_reference(args, w, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name}, "cpu_baseline": {
+        "config": workload_config(w, args.gpus), "cpu_baseline": {
             "value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": sample},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -282,26 +318,18 @@ def run_fd(args, w, rank, world, local_rank):
     # prefill every layer until the window is full (steady state)
     pk = [gen(synth.seed_of(base, 1, l), kshape) for l in range(L)]
     pv = [gen(synth.seed_of(base, 2, l), kshape) for l in range(L)]
-    if w.ragged_window:
-        lo, hi = w.ragged_window
-        fill = synth.ragged_fill(synth.seed_of(base, 3), R, lo, hi)
-        left = fill.copy()
-        while left.max() > 0:
-            fr = [int(min(F, x)) for x in left]
-            fd.fd_cache_commit(cache, 0, L, R, pk, pv, frames=fr)
-            left -= fr
-    else:
-        for _ in range(-(-w.slots // F) + 1):
-            fd.fd_cache_commit(cache, 0, L, R, pk, pv)
+    fill = prefill_frames(w, rank)
+    left = list(fill)
+    while max(left) > 0:
+        fr = [min(F, x) for x in left]
+        fd.fd_cache_commit(cache, 0, L, R, pk, pv, frames=fr)
+        left = [a - b for a, b in zip(left, fr)]
     torch.cuda.synchronize()
+    # the library's own frame counters agree with the described prefill
+    assert [fd.fd_cache_frames(cache, 0, r) for r in range(R)] == fill
 
     def nkeys():
-        out = []
-        for r in range(R):
-            n = fd.fd_cache_frames(cache, 0, r)
-            nv = min(n, w.sink_frames) + min(max(n - w.sink_frames, 0), w.window_frames)
-            out.append((nv + F) * Tf)
-        return out
+        return keys_per_rollout(w, fill)
 
     q = [[gen(synth.seed_of(base, 10, s, l), qshape) for l in range(L)] for s in range(S)]
     k = [[gen(synth.seed_of(base, 11, s, l), kshape) for l in range(L)] for s in range(S)]
@@ -392,14 +420,7 @@ def run_fd(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "rollouts_per_gpu": R, "layers": L, "heads": H,
-                   "head_dim": d, "grid": f"{w.grid_h}x{w.grid_w}",
-                   "action_tokens": w.action_tokens, "block_frames": F,
-                   "sink_frames": w.sink_frames, "window_frames": w.window_frames,
-                   "denoise_steps": S, "keys_per_rollout": nk[0] if len(set(nk)) == 1 else nk,
-                   "l2": "inputs larger than L2: every step reads all layers' caches and "
-                         "fresh q/k/v per (step, layer)",
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(w, world, rank),
         "latent_frames_per_s_per_layer": frames_per_s_layer,
         "roofline": roof,
         "commit_roofline": commit_roof,
