@@ -408,7 +408,7 @@ def run_fd(args, w, rank, world, local_rank):
             "flops_per_launch": flops_call, "launch_ms": attn_ms,
             "launch_covers": "fd_block_attention call: block-key RoPE pass + attention kernel"}
     # batched commit of all layers: read k, v; write K, V and rotated K
-    commit_bytes = 5.0 * L * R * F * Tf * H * d * 2
+    commit_bytes = 5.0 * L * R * F * Tf * w.hkv * d * 2
     commit_roof = {"bound": "hbm", "achieved": commit_bytes / (commit_ms * 1e-3) / 1e9,
                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "frac": commit_bytes / (commit_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
