@@ -208,7 +208,9 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * The bf16 kernel is persistent (one CTA per multiprocessor, at most 148)
  * and splits the call's KV iterations evenly over its CTAs; it returns
  * FD_ERR_UNSUPPORTED when n_rollouts x H x ceil(F*T/256) x (ceil((S+W)*Tf
- * /128) + ceil(F*Tf/128)) x CTAs reaches 2^31.  A query-tile pair split
+ * /128) + ceil(F*Tf/128)) x CTAs reaches 2^31, or when F*T x T reaches 2^40
+ * (its query-coordinate arithmetic), or when the RoPE tables of the call
+ * (S+W+F t-rows, the h and w tables) do not fit in shared memory.  A query-tile pair split
  * between CTAs is combined through the layer's `part` / `cnt` regions.
  * Device-side waits are bounded: a wait that gives up sets the error word
  * (fd_get_device_error) instead of hanging. */

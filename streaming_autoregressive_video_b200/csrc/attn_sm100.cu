@@ -1043,6 +1043,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+size_t attn_bf16_smem_bytes(const AttnParams& p) {
+  const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
+                                        (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
+  const size_t smem = kSmemFixed + tab;
+  return smem > kSmemMax ? 0 : smem;
+}
+
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kc,
                                    const CUtensorMap& tm_vc,
@@ -1063,10 +1070,8 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                 (int)kSmemMax);
   });
   if (e != cudaSuccess) return e;
-  const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
-                                        (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
-  const size_t smem = kSmemFixed + tab;
-  if (smem > kSmemMax) return cudaErrorNotSupported;
+  const size_t smem = attn_bf16_smem_bytes(p);
+  if (smem == 0) return cudaErrorNotSupported;
   if (p.G < 1 || p.G > kAttnMaxCtas) return cudaErrorInvalidValue;
   attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb,
                                                    tm_vb, p);

@@ -453,6 +453,15 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   const bool tensor_cores = cache->desc.dtype == FD_BF16 && c.d == 128;
   if (tensor_cores ? !cache->have_maps : (c.d % 32 != 0 || c.d > 128))
     return FD_ERR_UNSUPPORTED;
+  // The tensor-core kernel splits a query index q < Mq into (frame, token,
+  // h, w) with multiply-shift divisions (FastDiv), exact while n * divisor <
+  // 2^40: q / T, a token < T over Tv, a token < Tv over gw.
+  if (tensor_cores && ((uint64_t)p.Mq * c.T >= (1ull << 40) ||
+                       (uint64_t)c.T * c.Tv >= (1ull << 40) ||
+                       (uint64_t)c.Tv * c.gw >= (1ull << 40)))
+    return FD_ERR_UNSUPPORTED;
+  // and stages the call's RoPE tables in shared memory next to its tiles
+  if (tensor_cores && fd::attn_bf16_smem_bytes(p) == 0) return FD_ERR_UNSUPPORTED;
   // a shard's result is only usable with its log-sum-exp (to be combined)
   if (c.N > 1 && lse == nullptr) return FD_ERR_INVALID_ARG;
   // the block's keys belong to shard 0; other shards never read them

@@ -180,6 +180,9 @@ struct CombineParams {
   float* dst_lse;
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
+// Dynamic shared memory the tensor-core kernel needs for this call (its
+// fixed stages plus the call's RoPE tables), 0 if that exceeds the limit.
+size_t attn_bf16_smem_bytes(const AttnParams& p);
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kc,
                                    const CUtensorMap& tm_vc,
