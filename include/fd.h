@@ -186,7 +186,10 @@ fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
  * frame f of rollout r is at t = n_r + f with n_r that rollout's counter at
  * `layer`, i.e. the positions fd_block_attention gives the block.  This is the
  * same rotation fd_block_attention applies internally; it is exported for
- * callers that need rotated tensors and for tests. */
+ * callers that need rotated tensors and for tests.  n_rollouts x F x
+ * tokens_per_frame of 2^31 or more returns FD_ERR_UNSUPPORTED (the kernel
+ * counts token rows in 32 bits; fd_block_attention has the same limit for its
+ * block keys). */
 fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
                     void* x, int32_t tokens_per_frame, int32_t heads,
                     void* stream);

@@ -358,6 +358,7 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
   if (tokens_per_frame != v.T && tokens_per_frame != v.Tf) return FD_ERR_SHAPE;
   if (heads != v.H && heads != v.Hkv) return FD_ERR_SHAPE;
   if (!fd::aligned16(x)) return FD_ERR_ALIGNMENT;
+  if (!fd::rope_rows_ok(n_rollouts, v.F, tokens_per_frame)) return FD_ERR_UNSUPPORTED;
   fd_status st = fd::check_device(cache);
   if (st != FD_OK) return st;
   return fd::cuda_status(fd::launch_rope3d(v, layer, n_rollouts, x,
@@ -464,21 +465,19 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   if (tensor_cores && fd::attn_bf16_smem_bytes(p) == 0) return FD_ERR_UNSUPPORTED;
   // a shard's result is only usable with its log-sum-exp (to be combined)
   if (c.N > 1 && lse == nullptr) return FD_ERR_INVALID_ARG;
-  // the block's keys belong to shard 0; other shards never read them
-  if (c.shard == 0) {
-    st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
-    if (st != FD_OK) return st;
-  }
-  if (!tensor_cores) return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
+  // the RoPE pass walks the block's key rows with a 32-bit row counter
+  if (!fd::rope_rows_ok(n_rollouts, c.F, c.Tf)) return FD_ERR_UNSUPPORTED;
+  // Everything the tensor-core launch needs is prepared before the first
+  // launch of the call, so a refusal leaves nothing half done.
   CUtensorMap tm_q, tm_vb, tm_kb_work;
-  const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
-  if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
-      !fd::encode_bf16_map(&tm_vb, v_, c.d, c.Hkv, kb_rows, n_rollouts))
-    return FD_ERR_CUDA;
-  if (work != nullptr &&
-      !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.Hkv, kb_rows, n_rollouts))
-    return FD_ERR_CUDA;
-  {
+  if (tensor_cores) {
+    const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
+    if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
+        !fd::encode_bf16_map(&tm_vb, v_, c.d, c.Hkv, kb_rows, n_rollouts))
+      return FD_ERR_CUDA;
+    if (work != nullptr &&
+        !fd::encode_bf16_map(&tm_kb_work, work, c.d, c.Hkv, kb_rows, n_rollouts))
+      return FD_ERR_CUDA;
     // persistent grid: one CTA per multiprocessor, no more CTAs than KV
     // iterations the call can have (every rollout's cache full)
     const int64_t nt_max = ((int64_t)c.slots * c.Tf + 127) / 128 +
@@ -490,6 +489,12 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
     if (it_max * g >= ((int64_t)1 << 31)) return FD_ERR_UNSUPPORTED;
     p.G = (int)g;
   }
+  // the block's keys belong to shard 0; other shards never read them
+  if (c.shard == 0) {
+    st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
+    if (st != FD_OK) return st;
+  }
+  if (!tensor_cores) return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
   if (c.shard != 0) {
     // rollouts with no key on this shard get zero rows and lse = -inf here;
     // the tensor-core kernel skips them

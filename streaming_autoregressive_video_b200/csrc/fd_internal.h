@@ -55,6 +55,13 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
   return (uint32_t)(((uint64_t)n * f.m) >> 40);
 }
 
+// The RoPE pass walks token rows (rollout, frame, token) with a 32-bit
+// counter that steps by the grid's warp count: rows stay below 2^31 so the
+// counter cannot wrap.
+inline bool rope_rows_ok(int n_rollouts, int F, int tokens) {
+  return (uint64_t)n_rollouts * (uint64_t)F * (uint64_t)tokens < (1ull << 31);
+}
+
 // Valid cache frames of a rollout that committed n frames into a ring of S
 // sinks and W window slots: the slot prefix [0, nv).  Of these, shard `shard`
 // of N stores slots shard, shard + N, ... (local indices 0, 1, ...), which are
