@@ -136,3 +136,39 @@ def test_host_bound_keeps_the_arithmetic_in_32_bits():
         for x in (sk0, sk0 + I2 // 2, sk0 + I2 - 1):
             c = owner(x, sk0, I2, G)
             assert begin(c, sk0, I2, G) <= x < begin(c + 1, sk0, I2, G)
+
+
+# --------------------------------------------------------------------------
+# Multiply-shift division of the query coordinates: q / d computed as
+# (q * m) >> 40 with m = ceil(2^40 / d).  Exact whenever q * d < 2^40, the
+# bound the entry point enforces before launching the tensor-core kernel
+# (F*T x T, T x Tv, Tv x gw).
+# --------------------------------------------------------------------------
+def _fastdiv(n, d):
+    m = ((1 << 40) + d - 1) // d
+    return (n * m) >> 40
+
+
+@pytest.mark.parametrize("d", [1, 2, 3, 7, 52, 80, 1560, 1564, 3520, 14080, 65535, 1 << 20])
+def test_fastdiv_exact_below_the_bound(d):
+    rng = random.Random(d)
+    n_max = ((1 << 40) - 1) // d   # largest n with n * d < 2^40
+    ns = [0, 1, d - 1, d, d + 1, n_max, n_max - 1] + [rng.randint(0, n_max) for _ in range(20000)]
+    # every multiple of d and its neighbours near the top of the range
+    top = n_max // d * d
+    ns += [top - 1, top, min(top + 1, n_max)]
+    for n in ns:
+        assert _fastdiv(n, d) == n // d, (n, d)
+
+
+def test_fastdiv_fails_above_the_bound():
+    """The bound is needed: past it some quotient comes out one too high."""
+    d = 1560 * 64 + 1          # a frame of more than 2^16 tokens
+    m = ((1 << 40) + d - 1) // d
+    e = m * d - (1 << 40)      # rounding excess of m
+    assert e > 0
+    # the first multiple-minus-one of d whose excess reaches the next integer
+    n = d - 1
+    while (n * m) >> 40 == n // d:
+        n += d
+    assert n * d >= 1 << 40 and _fastdiv(n, d) == n // d + 1
