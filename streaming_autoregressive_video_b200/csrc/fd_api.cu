@@ -89,6 +89,10 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
     return FD_ERR_CAPACITY;
   lr = (size_t)d->num_layers * d->max_rollouts;
   size_t off = 0;
+  // Every region is kept below 2^56 bytes (far beyond any device memory), so
+  // the dozen regions summed below cannot wrap a 64-bit size.
+  constexpr size_t kRegionMax = (size_t)1 << 56;
+  if (kv > kRegionMax) return FD_ERR_CAPACITY;
   lay->k = off;
   off = align_up(off + kv);
   lay->v = off;
@@ -97,7 +101,7 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   off = align_up(off + kv);
   lay->kblk = off;
   size_t blk;
-  if (!mul_ok(frame * d->block_frames, lr, &blk)) return FD_ERR_CAPACITY;
+  if (!mul_ok(frame * d->block_frames, lr, &blk) || blk > kRegionMax) return FD_ERR_CAPACITY;
   off = align_up(off + blk);
   // partial results and arrival counters of the persistent bf16 kernel
   const bool tensor_path = d->dtype == FD_BF16;
@@ -108,7 +112,8 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
                              sizeof(float));
   lay->cnt = off;
   if (tensor_path) {
-    if (!mul_ok(lr * d->num_heads, pairs * sizeof(int32_t), &x)) return FD_ERR_CAPACITY;
+    if (!mul_ok(lr * d->num_heads, pairs * sizeof(int32_t), &x) || x > kRegionMax)
+      return FD_ERR_CAPACITY;
     off = align_up(off + x);
   }
   lay->pos = off;
@@ -116,7 +121,8 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   lay->count = off;
   off = align_up(off + lr * sizeof(int32_t));
   lay->ttab = off;
-  if (!mul_ok(lr * (slots + d->block_frames), (size_t)lay->rope_pairs_t * 8, &x))
+  if (!mul_ok(lr * (slots + d->block_frames), (size_t)lay->rope_pairs_t * 8, &x) ||
+      x > kRegionMax)
     return FD_ERR_CAPACITY;
   off = align_up(off + x);
   lay->htab = off;

@@ -135,3 +135,19 @@ def test_combine_host_errors():
     assert lib.fd_attention_combine(1, one, one, 1, 1, 1, 8, 9, 16, None, None) == 3
     assert lib.fd_attention_combine(1, None, one, 1, 1, 1, 8, 0, 16, None, None) == 1
     assert lib.fd_attention_combine(1, one, one, 1, 1, 1, 8, 0, 17, None, None) == 8
+
+
+def test_layout_regions_cannot_wrap_the_total():
+    """A geometry whose K region alone is 2^63 bytes (a 4096x4096 grid, 4096
+    heads of 256 fp32, 64 window slots, 1024 rollouts, 2 layers) is refused
+    with FD_ERR_CAPACITY: summed with V and the rotated keys it would wrap a
+    64-bit size and report a small storage requirement."""
+    desc = fd.CacheDesc(2, 1024, 4096, 256, 4096, 4096, 0, 1, 0, 64, 1.0e4, fd.FD_F32,
+                        0, 1, 1, 0)
+    lay = fd.CacheLayout()
+    assert fd.load().fd_cache_get_layout(ctypes.byref(desc), ctypes.byref(lay)) == 4
+    assert fd.fd_cache_bytes(desc) == 0
+    # one layer of one rollout of the same frame size still lays out
+    small = fd.CacheDesc(1, 1, 4, 256, 64, 64, 0, 1, 0, 64, 1.0e4, fd.FD_F32, 0, 1, 1, 0)
+    assert fd.load().fd_cache_get_layout(ctypes.byref(small), ctypes.byref(lay)) == 0
+    assert lay.total == fd.fd_cache_bytes(small) > 3 * lay.layer_kv_bytes
