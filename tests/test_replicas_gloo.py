@@ -81,7 +81,7 @@ def test_two_replicas_over_gloo(tmp_path):
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
 
 
-def _cp_rank_main(rank, port, out_dir):
+def _cp_rank_main(rank, port, out_dir, world, commits):
     """One rank of a context-parallel attention call over gloo: the rank's part
     of the key set (oracle, standing in for the shard's kernel), all-gather,
     combination (oracle)."""
@@ -94,13 +94,13 @@ def _cp_rank_main(rank, port, out_dir):
     import oracle
     from streaming_autoregressive_video_b200.context_parallel import ShardedBlockAttention
 
-    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+    dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
         rng = np.random.default_rng(71)   # the same inputs on every rank
         S, W, F, T, H, d = 1, 4, 2, 6, 2, 12
         c = oracle.RolloutCache(S, W, T, H, d, "f32")
-        for _ in range(3):
+        for _ in range(commits):
             c.commit(rng.standard_normal((F, T, H, d)).astype(np.float32),
                      rng.standard_normal((F, T, H, d)).astype(np.float32))
         q = rng.standard_normal((F * T, H, d)).astype(np.float32)
@@ -109,7 +109,7 @@ def _cp_rank_main(rank, port, out_dir):
         kw = dict(tokens=T, grid_w=3, theta=1.0e4)
 
         def attn(layer, n, q_, k_, v_, out, lse):
-            o, l = oracle.block_attention(c, q_[0], k_[0], v_[0], slot_part=(WORLD, rank),
+            o, l = oracle.block_attention(c, q_[0], k_[0], v_[0], slot_part=(world, rank),
                                           include_block=(rank == 0), **kw)
             out[0] = torch.from_numpy(o)
             lse[0] = torch.from_numpy(l)
@@ -119,7 +119,7 @@ def _cp_rank_main(rank, port, out_dir):
                                            [x[0].numpy() for x in lses])
             out[0] = torch.from_numpy(o)
 
-        cp = ShardedBlockAttention(None, WORLD, rank, attn_fn=attn, combine_fn=combine)
+        cp = ShardedBlockAttention(None, world, rank, attn_fn=attn, combine_fn=combine)
         out = torch.zeros((1, F * T, H, d), dtype=torch.float64)
         cp(0, 1, q[None], k[None], v[None], out)
         full, _ = oracle.block_attention(c, q, k, v, **kw)
@@ -131,13 +131,15 @@ def _cp_rank_main(rank, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_context_parallel_gather_and_combine_over_gloo(tmp_path):
-    """Two ranks, each holding half of the cache slots (the block's keys on
-    rank 0): after the all-gather and the combination every rank has the
-    attention over the whole key set."""
-    mp.start_processes(_cp_rank_main, args=(_free_port(), str(tmp_path)), nprocs=WORLD,
-                       join=True, start_method="spawn")
+@pytest.mark.parametrize("world,commits", [(2, 3), (3, 3), (3, 0)])
+def test_context_parallel_gather_and_combine_over_gloo(tmp_path, world, commits):
+    """N ranks, rank r holding the cache slots s with s mod N == r (the block's
+    keys on rank 0): after the all-gather and the combination every rank has
+    the attention over the whole key set.  With an empty cache (no commit)
+    every rank but 0 holds no key: its part weighs nothing."""
+    mp.start_processes(_cp_rank_main, args=(_free_port(), str(tmp_path), world, commits),
+                       nprocs=world, join=True, start_method="spawn")
     # the parts' log-sum-exps travel as fp32 (the library's type), hence the
     # fp32-level bound on an fp64 computation
-    for r in range(WORLD):
+    for r in range(world):
         assert json.load(open(tmp_path / f"cp{r}.json"))["err"] < 1e-6
