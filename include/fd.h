@@ -161,7 +161,16 @@ fd_status fd_cache_get_layout(const fd_cache_desc* desc, fd_cache_layout* out);
  * marks every slot empty, sets every counter to 0 and builds the RoPE tables,
  * then synchronises the device once.  The library allocates no device
  * memory, here or later: memory stays constant over unbounded rollouts
- * ([FD-BM], [C3-SI]).  The host object is freed by fd_cache_destroy. */
+ * ([FD-BM], [C3-SI]).  The host object is freed by fd_cache_destroy.
+ *
+ * Snapshot and restore: every piece of a cache's state (K, V, rotated K,
+ * slot positions, frame counters, RoPE tables) lives in the storage, so a
+ * snapshot is a copy of the fd_cache_bytes bytes taken between calls (after
+ * the stream's work is done), and a restore is fd_cache_create with the same
+ * descriptor followed by a copy of the snapshot over the new storage.  The
+ * calls then continue the snapshot's rollouts.  fd_cache_frames reads a host
+ * mirror of the counters that only this object's commits and resets
+ * update, so after a restore it counts from the restore. */
 fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
                           size_t bytes, fd_cache** out);
 

@@ -48,6 +48,7 @@ extern "C" fd_status fd_block_attention_static(fd_cache* cache, int32_t layer,
                                                const void* q, const void* k,
                                                const void* v, void* out,
                                                float* lse, void* stream) {
+  fd::NvtxRange nvtx_range("fd_block_attention_static");
   if (cache == nullptr || n_rollouts < 1) return FD_ERR_INVALID_ARG;
   if (fd::block_work_bytes(cache, n_rollouts) > (size_t)FD_STATIC_WORK_BYTES)
     return FD_ERR_CAPACITY;

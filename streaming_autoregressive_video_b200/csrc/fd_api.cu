@@ -211,6 +211,7 @@ fd_status fd_cache_get_layout(const fd_cache_desc* desc, fd_cache_layout* out) {
 
 fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
                           size_t bytes, fd_cache** out) {
+  fd::NvtxRange nvtx_range("fd_cache_create");
   if (out == nullptr) return FD_ERR_INVALID_ARG;
   *out = nullptr;
   fd_cache_layout lay;
@@ -332,6 +333,7 @@ fd_status fd_cache_frames(const fd_cache* cache, int32_t layer,
 
 fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
                          int32_t n_ids, void* stream) {
+  fd::NvtxRange nvtx_range("fd_cache_reset");
   if (cache == nullptr || (n_ids > 0 && rollout_ids == nullptr) || n_ids < 0)
     return FD_ERR_INVALID_ARG;
   const fd::CacheView& v = cache->view;
@@ -357,6 +359,7 @@ fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
 fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
                     void* x, int32_t tokens_per_frame, int32_t heads,
                     void* stream) {
+  fd::NvtxRange nvtx_range("fd_rope3d");
   if (cache == nullptr || x == nullptr) return FD_ERR_INVALID_ARG;
   const fd::CacheView& v = cache->view;
   if (layer < 0 || layer >= v.L || n_rollouts < 1 || n_rollouts > v.R)
@@ -376,6 +379,7 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
                              int32_t n_rollouts, const void* q, const void* k,
                              const void* v_, void* out, float* lse,
                              void* stream) {
+  fd::NvtxRange nvtx_range("fd_block_attention");
   return fd::block_attention_impl(cache, layer, n_rollouts, q, k, v_, out, lse,
                                   stream, nullptr);
 }
@@ -518,6 +522,7 @@ fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,
                           int32_t layer_end, int32_t n_rollouts,
                           const int32_t* frames, const void* const* k,
                           const void* const* v, void* stream) {
+  fd::NvtxRange nvtx_range("fd_cache_commit");
   if (cache == nullptr || k == nullptr || v == nullptr) return FD_ERR_INVALID_ARG;
   const fd::CacheView& c = cache->view;
   if (layer_begin < 0 || layer_end > c.L || layer_begin >= layer_end ||
@@ -588,6 +593,7 @@ fd_status fd_attention_combine(int32_t n_parts, const void* const* outs,
                                const float* const* lses, int32_t n_rollouts,
                                int32_t rows, int32_t heads, int32_t head_dim,
                                int32_t dtype, void* out, float* lse, void* stream) {
+  fd::NvtxRange nvtx_range("fd_attention_combine");
   if (outs == nullptr || lses == nullptr || out == nullptr) return FD_ERR_INVALID_ARG;
   if (n_parts < 1 || n_parts > fd::kCombineMaxParts) return FD_ERR_SHAPE;
   if (dtype != FD_BF16 && dtype != FD_F32) return FD_ERR_DTYPE;

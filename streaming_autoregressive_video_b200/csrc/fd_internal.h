@@ -7,9 +7,21 @@
 
 #include <atomic>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fd.h"
 
 namespace fd {
+
+// NVTX range over one entry point of the library, so that a profiler's
+// timeline shows each call (header-only NVTX v3: without an attached tool a
+// push or pop is one indirect call that returns at once).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Devices one process may drive (ordinals 0 .. kMaxDevices-1).
 constexpr int kMaxDevices = 64;
