@@ -13,7 +13,6 @@ h div (H/Hkv); views share t and repeat (h, w))."""
 import math
 
 import numpy as np
-import pytest
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st
 
@@ -104,3 +103,38 @@ def test_rolling_cache_equals_masked_full_history_random(case):
         vf = v.reshape(F, Tf, Hkv, d)[:nf]
         cache.commit(kf, vf)
         history += [(kf[f], vf[f]) for f in range(nf)]
+
+
+@settings(max_examples=30, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(rollouts(), st.integers(1, 5))
+def test_key_set_parts_recombine_random(case, N):
+    """Context parallelism ("NVIDIA FlashDreams ...", Multi-GPU Context
+    Parallelism; reading: cache slot s belongs to part s mod N, the block's
+    keys to part 0): the parts' rows merged by their log-sum-exps equal the
+    attention over the whole key set, for any fill of the ring."""
+    from oracle import combine_partials
+    S, W, F, views, gh, gw, A, H, Hkv, commits, seed = case
+    rng = np.random.default_rng(seed)
+    d, theta = 12, 1.0e4
+    Tv = gh * gw
+    T = views * Tv
+    Tf = T + A
+    vt = Tv if views > 1 else 0
+    cache = RolloutCache(S, W, Tf, Hkv, d, "f32")
+    for nf in commits:
+        cache.commit(rng.standard_normal((nf, Tf, Hkv, d)).astype(np.float32),
+                     rng.standard_normal((nf, Tf, Hkv, d)).astype(np.float32))
+    q = rng.standard_normal((F * T, H, d)).astype(np.float32)
+    k = rng.standard_normal((F * Tf, Hkv, d)).astype(np.float32)
+    v = rng.standard_normal((F * Tf, Hkv, d)).astype(np.float32)
+    kw = dict(tokens=T, grid_w=gw, theta=theta, view_tokens=vt)
+    whole, whole_lse = block_attention(cache, q, k, v, **kw)
+    outs, lses = [], []
+    for part in range(N):
+        o, l = block_attention(cache, q, k, v, slot_part=(N, part),
+                               include_block=(part == 0), **kw)
+        outs.append(o)
+        lses.append(l)
+    got, got_lse = combine_partials(outs, lses)
+    np.testing.assert_allclose(got, whole, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got_lse, whole_lse, rtol=0, atol=1e-12)
