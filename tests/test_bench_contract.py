@@ -1,0 +1,67 @@
+"""bench.py's JSON line on the CPU: the GPU arm's host code runs with CUDA
+and the library replaced by stand-ins (tests/bench_stub.py, in a subprocess),
+and the line it prints carries every key of the bench contract.  The
+reference arm runs for real (the oracle on the host)."""
+import json
+import os
+import subprocess
+import sys
+import types
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from streaming_autoregressive_video_b200.workloads import Workload  # noqa: E402
+
+
+def _stub_line(workload):
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "bench_stub.py"),
+                          workload], capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    return json.loads(res.stdout.strip().splitlines()[-1])
+
+
+@pytest.mark.parametrize("workload", ["480p", "gqa", "ragged", "multiview"])
+def test_gpu_arm_line_keeps_the_contract(workload):
+    line = _stub_line(workload)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "gpu_launches", "clocks", "e2e"):
+        assert key in line, key
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["scaling"] == "weak" and line["n_gpus"] == 1 and line["warmup"] >= 3
+    assert line["config"]["workload"] == bench.workloads()[workload].name
+    roof = line["roofline"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in roof, key
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    e2e = line["e2e"]
+    for key in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert key in e2e, key
+    w0 = bench.workloads()[workload]
+    w = w0.scaled(layers=min(w0.layers, 2))   # as bench_stub.py runs it
+    # every call copies q, k, v in and out back: bytes from the tensors' sizes
+    q = w.rollouts * w.queries * w.heads * w.head_dim * 2
+    kv = w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * 2
+    calls = w.steps * w.layers
+    assert e2e["h2d_bytes_per_step"] == calls * (q + 2 * kv)
+    assert e2e["d2h_bytes_per_step"] == calls * q
+    assert line["gpu_launches"] > 0
+    # commit bytes: read k, v; write K, V and rotated K, with Hkv heads
+    assert line["commit_roofline"]["algorithmic_bytes_per_launch"] == 5 * w.layers * kv
+
+
+def test_reference_arm_line_matches_the_gpu_arm_config(capsys):
+    w = Workload("contract-tiny", layers=2, rollouts=1, heads=2, head_dim=16, grid_h=3,
+                 grid_w=4, action_tokens=1, block_frames=1, sink_frames=1,
+                 window_frames=2, steps=1, blocks=1, dtype="bf16")
+    bench.run_reference(types.SimpleNamespace(steps=1, warmup=0, gpus=1), w, 0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config(w, 1)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
