@@ -1,9 +1,11 @@
-"""ctypes binding of libfd.so: argument marshalling only.
+"""ctypes binding of libfd.so: argument marshalling and argument checks only.
 
-Every function here has the name of a C entry point in include/fd.h, converts
-Python / torch arguments into plain pointers and sizes, calls the library and
-raises FdError on a non-OK status.  No step of the computation runs here; if
-the library cannot be loaded the call fails loudly.
+Every function here has the name of a C entry point in include/fd.h, checks
+that each tensor argument is a contiguous CUDA tensor (on the cache's device)
+holding at least the bytes the call reads or writes, converts Python / torch
+arguments into plain pointers and sizes, calls the library and raises FdError
+on a non-OK status.  No step of the computation runs here; if the library
+cannot be loaded the call fails loudly.
 """
 from __future__ import annotations
 
