@@ -24,6 +24,8 @@ from .streaming_attention import (  # noqa: F401
     slot_of,
     valid_slot_count,
     RolloutCache,
+    window_boundary_reached,
+    start_window,
     block_attention,
     combine_partials,
 )

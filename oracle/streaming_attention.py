@@ -59,6 +59,16 @@ R10 multi-view frames (a shape variant; the pages show four-camera models
     (Gh*Gw), and all views of a frame share t.  Views therefore differ only by
     content (any learned view embedding belongs to the model, before the
     attention).  V = 1 is R5.
+R12 window-boundary reset ("Single-GPU inference for DreamZero", Sequential
+    requests; a second cache policy next to the ring of R3): the cache's
+    S + W slots hold one local-attention window of consecutive frames that
+    is never evicted frame by frame.  Before a block of F frames, if the
+    window cannot take it (n + F > S + W), the old frames are released
+    (reset: n = 0, every slot empty), the conditioning is re-encoded and
+    committed first at positions 0 .. c-1, and the block follows at t = c.
+    Inside a window no slot is ever reused, so the ring of R3 never wraps
+    and every attention call sees exactly the frames committed since the
+    last reset.
 R11 context parallelism (a way to compute the same attention on N devices,
     named by the pages without formulas): the key set splits into disjoint
     parts; part i yields the softmax-normalised output O_i and log-sum-exp
@@ -212,6 +222,19 @@ class RolloutCache:
 
     def valid_slots(self) -> int:
         return valid_slot_count(self.n, self.S, self.W)
+
+
+def window_boundary_reached(n: int, frames: int, S: int, W: int) -> bool:
+    """R12: the next block of `frames` frames does not fit in the window of
+    S + W slots after n committed frames, so the window restarts."""
+    return n + frames > S + W
+
+
+def start_window(cache: "RolloutCache", cond_k: np.ndarray, cond_v: np.ndarray) -> None:
+    """R12: release the window's frames and commit the re-encoded conditioning
+    frames ([c][Tf][H][d], storage form) at positions 0 .. c-1."""
+    cache.reset()
+    cache.commit(cond_k, cond_v)
 
 
 # --------------------------------------------------------------------------

@@ -145,3 +145,34 @@ def test_worked_attention_fixture_catches_mistakes(mistake):
         assert np.allclose(out, g["want_out"], rtol=0, atol=1e-12)
     else:
         assert not np.allclose(out, g["want_out"], rtol=0, atol=1e-6)
+
+
+def test_window_reset_fixture():
+    """The window-boundary policy (R12) follows the hand-worked sequences:
+    when the window restarts, which positions the block gets, which slots its
+    attention sees and the counter after its commit."""
+    caches, n_rows = {}, 0
+    for head, tail in _rows("window_reset.txt"):
+        S, W, F, c, blk = (int(x) for x in head)
+        n0, restart, n1, t_blk, seen, n2 = tail.split()
+        if (S, W, F, c) not in caches:
+            cache = oracle.RolloutCache(S, W, 1, 1, 2, "f32")
+            cond = np.zeros((c, 1, 1, 2), np.float32)
+            oracle.start_window(cache, cond, cond)          # a new sequence
+            caches[(S, W, F, c)] = cache
+        cache = caches[(S, W, F, c)]
+        assert cache.n == int(n0), (S, W, F, c, blk)
+        hit = oracle.window_boundary_reached(cache.n, F, S, W)
+        assert hit == bool(int(restart)), (S, W, F, c, blk)
+        if hit:
+            cond = np.zeros((c, 1, 1, 2), np.float32)
+            oracle.start_window(cache, cond, cond)
+        assert cache.n == int(n1)
+        assert [cache.n + f for f in range(F)] == [int(x) for x in t_blk.split(",")]
+        nv = cache.valid_slots()
+        assert [f"{s}:{cache.pos[s]}" for s in range(nv)] == seen.split(","), (S, W, blk)
+        frames = np.full((F, 1, 1, 2), 7, np.float32)
+        cache.commit(frames, frames)
+        assert cache.n == int(n2)
+        n_rows += 1
+    assert n_rows == 14

@@ -498,3 +498,49 @@ def test_empty_part_has_no_weight():
     # no keys anywhere: zero rows, -inf
     out, lse = oracle.combine_partials([o1, o1], [l1, l1])
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+@pytest.mark.parametrize("S,W,F,c", [(1, 4, 2, 1), (0, 3, 1, 2), (2, 3, 1, 1)])
+def test_window_reset_equals_attention_over_the_current_window(S, W, F, c):
+    """R12: with the window-boundary policy every attention call equals the
+    brute-force attention over the frames committed since the window's start
+    (conditioning at t = 0 .. c-1, then the blocks), positions counted from
+    that start: earlier windows leave no trace."""
+    from oracle import start_window, window_boundary_reached
+    rng = np.random.default_rng(40 + S + W + F + c)
+    gh, gw, H, d, theta = 2, 2, 2, 12, 1.0e4
+    T = gh * gw
+    Tf = T
+    cache = RolloutCache(S, W, Tf, H, d, "f32")
+    window = []                       # (k, v) of the frames of the current window
+
+    def new_window():
+        ck = rng.standard_normal((c, Tf, H, d)).astype(np.float32)
+        cv = rng.standard_normal((c, Tf, H, d)).astype(np.float32)
+        start_window(cache, ck, cv)
+        window[:] = [(ck[f].astype(np.float64), cv[f].astype(np.float64)) for f in range(c)]
+
+    new_window()
+    restarts = 0
+    for blk in range(7):
+        if window_boundary_reached(cache.n, F, S, W):
+            new_window()
+            restarts += 1
+        n = cache.n
+        assert n == len(window)
+        q = rng.standard_normal((F * T, H, d)).astype(np.float32)
+        k = rng.standard_normal((F * Tf, H, d)).astype(np.float32)
+        v = rng.standard_normal((F * Tf, H, d)).astype(np.float32)
+        out, lse = block_attention(cache, q, k, v, tokens=T, grid_w=gw, theta=theta)
+        # every frame of the window is visible: a sink + window mask as wide
+        # as the whole window
+        ref, ref_lse = _brute_force_block(window, n, n, 0, q.astype(np.float64),
+                                          k.astype(np.float64), v.astype(np.float64),
+                                          T, Tf, gw, theta)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+        kf, vf = k.reshape(F, Tf, H, d), v.reshape(F, Tf, H, d)
+        cache.commit(kf, vf)
+        window += [(kf[f].astype(np.float64), vf[f].astype(np.float64)) for f in range(F)]
+        assert cache.n <= S + W   # the ring never wraps under this policy
+    assert restarts >= 1
