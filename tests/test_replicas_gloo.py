@@ -83,8 +83,9 @@ def test_two_replicas_over_gloo(tmp_path):
 
 def _cp_rank_main(rank, port, out_dir, world, commits):
     """One rank of a context-parallel attention call over gloo: the rank's part
-    of the key set (oracle, standing in for the shard's kernel), all-gather,
-    combination (oracle)."""
+    of the key set (oracle, standing in for the shard's kernel), the exchange
+    of row chunks, the combination of this rank's chunk (oracle) and, for the
+    full output, the gather of the merged chunks."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
 
@@ -92,7 +93,8 @@ def _cp_rank_main(rank, port, out_dir, world, commits):
     import torch
 
     import oracle
-    from streaming_autoregressive_video_b200.context_parallel import ShardedBlockAttention
+    from streaming_autoregressive_video_b200.context_parallel import (ShardedBlockAttention,
+                                                                      row_chunks)
 
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
@@ -118,28 +120,45 @@ def _cp_rank_main(rank, port, out_dir, world, commits):
             o, l = oracle.combine_partials([x[0].numpy() for x in outs],
                                            [x[0].numpy() for x in lses])
             out[0] = torch.from_numpy(o)
+            if lse is not None:
+                lse[0] = torch.from_numpy(l)
 
         cp = ShardedBlockAttention(None, world, rank, attn_fn=attn, combine_fn=combine)
+        full, full_lse = oracle.block_attention(c, q, k, v, **kw)
         out = torch.zeros((1, F * T, H, d), dtype=torch.float64)
-        cp(0, 1, q[None], k[None], v[None], out)
-        full, _ = oracle.block_attention(c, q, k, v, **kw)
+        lse = torch.zeros((1, H, F * T), dtype=torch.float64)
+        assert cp(0, 1, q[None], k[None], v[None], out, lse) == (0, F * T)
         err = float(np.abs(out[0].numpy() - full).max())
+        err_lse = float(np.abs(lse[0].numpy() - full_lse).max())
+        # only this rank's chunk of rows
+        out2 = torch.zeros_like(out)
+        lse2 = torch.zeros_like(lse)
+        q0, q1 = cp(0, 1, q[None], k[None], v[None], out2, lse2, rows_only=True)
+        assert (q0, q1) == row_chunks(F * T, world)[rank]
+        err_rows = float(np.abs(out2[0, q0:q1].numpy() - full[q0:q1]).max())
+        untouched = bool((out2[0, :q0] == 0).all() and (out2[0, q1:] == 0).all())
         with open(os.path.join(out_dir, f"cp{rank}.json"), "w") as f:
-            json.dump({"err": err}, f)
+            json.dump({"err": err, "err_lse": err_lse, "err_rows": err_rows,
+                       "untouched": untouched}, f)
         dist.barrier()
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,commits", [(2, 3), (3, 3), (3, 0)])
+@pytest.mark.parametrize("world,commits", [(2, 3), (3, 3), (3, 0), (5, 3)])
 def test_context_parallel_gather_and_combine_over_gloo(tmp_path, world, commits):
     """N ranks, rank r holding the cache slots s with s mod N == r (the block's
-    keys on rank 0): after the all-gather and the combination every rank has
-    the attention over the whole key set.  With an empty cache (no commit)
-    every rank but 0 holds no key: its part weighs nothing."""
+    keys on rank 0): after the exchange of row chunks and the combination
+    every rank has the attention over the whole key set for its chunk of
+    query rows (rows_only) or, after the gather of the merged chunks, for
+    every row.  With an empty cache (no commit) every rank but 0 holds no
+    key: its part weighs nothing.  Five ranks over 12 rows give unequal
+    chunks (the padded gather)."""
     mp.start_processes(_cp_rank_main, args=(_free_port(), str(tmp_path), world, commits),
                        nprocs=world, join=True, start_method="spawn")
     # the parts' log-sum-exps travel as fp32 (the library's type), hence the
     # fp32-level bound on an fp64 computation
     for r in range(world):
-        assert json.load(open(tmp_path / f"cp{r}.json"))["err"] < 1e-6
+        res = json.load(open(tmp_path / f"cp{r}.json"))
+        assert res["err"] < 1e-6 and res["err_rows"] < 1e-6 and res["err_lse"] < 1e-6
+        assert res["untouched"]
