@@ -114,6 +114,14 @@ typedef struct {
                            * every shard counts all committed frames, and the
                            * block's own keys belong to shard 0              */
   int32_t shard_index;    /* this cache's shard, 0 <= shard_index < N      */
+  int32_t num_work_sets;  /* Wk per-call work areas (0: 1), 1 <= Wk <= L: an
+                           * attention call on layer l uses work set l mod
+                           * Wk, and two attention calls on this cache may
+                           * run at the same time on the GPU only when their
+                           * layers differ modulo Wk.  One set (the default)
+                           * keeps the storage to what one call at a time
+                           * needs; Wk = L lets calls on any two layers
+                           * overlap (no counterpart on the pages)          */
 } fd_cache_desc;
 
 /* Byte offsets of the regions inside the caller's storage buffer.
@@ -123,15 +131,14 @@ typedef struct {
  *          position never change, so its rotation is computed once instead
  *          of at every attention call); derived data, not part of the
  *          cache's observable state
- *   kblk : [L][R][F*Tf][Hkv][d] work area of fd_block_attention: the current
- *          block's keys rotated once per call, read by every query tile
- *          (one region per layer, so calls on different layers may run
- *          concurrently; calls on the same layer must be ordered)
- *   part : [L][148][2][256*128 + 512] float work area of the bf16 attention
+ *   kblk : [Wk][R][F*Tf][Hkv][d] work area of fd_block_attention: the
+ *          current block's keys rotated once per call, read by every query
+ *          tile (one set per work set, see num_work_sets)
+ *   part : [Wk][148][2][256*128 + 512] float work area of the bf16 attention
  *          kernel: a CTA whose share of the work ends or begins inside a
  *          query tile pair leaves its partial result there (unnormalised
  *          output rows, running max, row sum); empty (size 0) for fp32
- *   cnt  : [L][R][H][ceil(F*T/256)] int32 arrival counters of those split
+ *   cnt  : [Wk][R][H][ceil(F*T/256)] int32 arrival counters of those split
  *          tile pairs; zero between calls (the last arriving CTA combines
  *          the partial results and clears its counter)
  *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
@@ -150,10 +157,15 @@ typedef struct {
 typedef struct fd_cache fd_cache;
 
 /* Bytes of device storage a cache with this geometry needs; 0 if the
- * descriptor is invalid.  Pure host function. */
+ * descriptor is invalid.  Pure host function.  The storage is bounded by the
+ * geometry alone, whatever the length of the rollouts ([FD-BM], [C3-SI]:
+ * bounded, static-shape cache); its regions are those of fd_cache_layout
+ * (the cache's reading: K/V as committed plus positions, see the readings
+ * at the top of this file). */
 size_t fd_cache_bytes(const fd_cache_desc* desc);
 
-/* Region offsets of the storage layout above.  Pure host function. */
+/* Region offsets of the storage layout above ([FD-BM], [C3-SI]; the regions
+ * follow the readings at the top of this file).  Pure host function. */
 fd_status fd_cache_get_layout(const fd_cache_desc* desc, fd_cache_layout* out);
 
 /* Bind a cache object to caller-owned device storage of at least
@@ -188,7 +200,11 @@ fd_status fd_cache_layout_of(const fd_cache* cache, fd_cache_layout* out);
 fd_status fd_cache_reset(fd_cache* cache, const int32_t* rollout_ids,
                          int32_t n_ids, void* stream);
 
-/* 3D RoPE in place on a block tensor x of rollouts 0..n_rollouts-1:
+/* 3D RoPE in place on a block tensor x of rollouts 0..n_rollouts-1.  The
+ * pages name no positional encoding; this is the 3D (t,h,w) RoPE reading at
+ * the top of this file (pair layout, t | h | w sections, frequencies), with
+ * t the block's frames since the last reset ([DZ-SR]: frame positions carry
+ * over between requests):
  *   x: [n_rollouts][F][tokens_per_frame][heads][d] of the cache dtype;
  *   tokens_per_frame = T (queries) or Tf (keys, action tokens at (t,0,0));
  *   heads = num_heads (queries) or Hkv (keys); anything else FD_ERR_SHAPE;
@@ -212,9 +228,9 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * For rollout r the key set is its valid cache slots (sinks + window, frame
  * positions from the slot table) plus all F*Tf block tokens at t = n_r + f.
  * The cache is read only: call it once per denoising step, then commit.
- * bf16 with head_dim 128 runs on tcgen05 tensor cores (fp32 accumulation, P
- * rounded to bf16); f32, and bf16 with head_dim 32, 64 or 96, on CUDA cores
- * in fp32 arithmetic (no TF32; bf16 output rounded once).  Other head sizes
+ * bf16 with head_dim 128 or 64 runs on tcgen05 tensor cores (fp32
+ * accumulation, P rounded to bf16); f32, and bf16 with head_dim 32 or 96, on
+ * CUDA cores in fp32 arithmetic (no TF32; bf16 output rounded once).  Other head sizes
  * return FD_ERR_UNSUPPORTED before any launch.  Tensor bases must be 16-byte
  * aligned.
  * The bf16 kernel is persistent (one CTA per multiprocessor, at most 148)
@@ -240,8 +256,9 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
  * fd_block_attention; the work area for the block's rotated keys is instead a
  * static device array of FD_STATIC_WORK_BYTES inside this library, which
  * every GPU that loads the library holds until the process exits.
- *   - FD_ERR_CAPACITY (before any launch) when n_rollouts*F*Tf*H*d*element
- *     size exceeds FD_STATIC_WORK_BYTES;
+ *   - FD_ERR_CAPACITY (before any launch) when n_rollouts*F*Tf*Hkv*d*element
+ *     size (the block's rotated keys, Hkv key/value heads) exceeds
+ *     FD_STATIC_WORK_BYTES;
  *   - the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress), so make that first call before any stream
  *     capture on that device;
@@ -268,6 +285,19 @@ fd_status fd_cache_commit(fd_cache* cache, int32_t layer_begin,
                           int32_t layer_end, int32_t n_rollouts,
                           const int32_t* frames, const void* const* k,
                           const void* const* v, void* stream);
+
+/* Window-boundary policy of [DZ-SR], a second way to bound the cache next to
+ * the rolling ring: the S + W slots hold one local-attention window of
+ * consecutive frames; when the next block of `frames` frames does not fit
+ * (n + frames > S + W, n the rollout's counter at `layer`), the window
+ * restarts: the caller releases the old frames with fd_cache_reset, commits
+ * the re-encoded conditioning frames (they take positions 0, 1, ...) with
+ * fd_cache_commit, and then runs the block.  Used this way the ring never
+ * wraps.  Sets *reached to 1 in that case and to 0 otherwise.  Host only:
+ * reads the host mirror of the counter (fd_cache_frames); nothing is
+ * launched.  frames in [1, F]. */
+fd_status fd_cache_window_full(const fd_cache* cache, int32_t layer,
+                               int32_t rollout, int32_t frames, int32_t* reached);
 
 /* Host mirror of a rollout's counter (updated by commit/reset calls). */
 fd_status fd_cache_frames(const fd_cache* cache, int32_t layer,

@@ -26,7 +26,8 @@ EXPORTS = ["fd_cache_bytes", "fd_cache_get_layout", "fd_cache_create",
            "fd_cache_destroy", "fd_cache_get_desc", "fd_cache_layout_of",
            "fd_cache_reset", "fd_rope3d", "fd_block_attention",
            "fd_block_attention_static",
-           "fd_cache_commit", "fd_cache_frames", "fd_get_device_error",
+           "fd_cache_commit", "fd_cache_frames", "fd_cache_window_full",
+           "fd_get_device_error",
            "fd_exp2_selfcheck", "fd_selftest_bounded_wait", "fd_attention_combine",
            "fd_launch_count", "fd_status_string"]
 
@@ -45,7 +46,8 @@ class CacheDesc(ctypes.Structure):
                 ("sink_frames", ctypes.c_int32), ("window_frames", ctypes.c_int32),
                 ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("num_views", ctypes.c_int32),
-                ("num_shards", ctypes.c_int32), ("shard_index", ctypes.c_int32)]
+                ("num_shards", ctypes.c_int32), ("shard_index", ctypes.c_int32),
+                ("num_work_sets", ctypes.c_int32)]
 
 
 class CacheLayout(ctypes.Structure):
@@ -90,6 +92,7 @@ def load(path: Optional[str] = None, build_if_missing: bool = True) -> ctypes.CD
     lib.fd_cache_commit.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32),
                                     ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
     lib.fd_cache_frames.argtypes = [vp, i32, i32, ctypes.POINTER(ctypes.c_int64)]
+    lib.fd_cache_window_full.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32)]
     lib.fd_get_device_error.argtypes = [vp, ctypes.POINTER(i32)]
     lib.fd_exp2_selfcheck.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.fd_selftest_bounded_wait.argtypes = [vp, i32, vp]
@@ -171,14 +174,18 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def make_desc(w, dtype: Optional[str] = None, shards: int = 1, shard: int = 0) -> CacheDesc:
+def make_desc(w, dtype: Optional[str] = None, shards: int = 1, shard: int = 0,
+              work_sets: int = 1) -> CacheDesc:
     """CacheDesc of a workload (see workloads.Workload); `shards`/`shard`
-    select one context-parallel shard of its key set."""
+    select one context-parallel shard of its key set; `work_sets` is the
+    number of per-call work areas (attention calls whose layers differ modulo
+    it may run at the same time)."""
     dt = dtype or w.dtype
     return CacheDesc(w.layers, w.rollouts, w.heads, w.head_dim, w.grid_h, w.grid_w,
                      w.action_tokens, w.block_frames, w.sink_frames, w.window_frames,
                      float(w.theta), FD_BF16 if dt == "bf16" else FD_F32,
-                     getattr(w, "kv_heads", 0), getattr(w, "views", 1), shards, shard)
+                     getattr(w, "kv_heads", 0), getattr(w, "views", 1), shards, shard,
+                     work_sets)
 
 
 def fd_cache_bytes(desc: CacheDesc) -> int:
@@ -301,6 +308,15 @@ def fd_cache_frames(cache: Cache, layer: int, rollout: int) -> int:
     _check(load().fd_cache_frames(cache.handle, layer, rollout, ctypes.byref(n)),
            "fd_cache_frames")
     return n.value
+
+
+def fd_cache_window_full(cache: Cache, layer: int, rollout: int, frames: int) -> bool:
+    """Whether the next block of `frames` frames restarts the rollout's window
+    (the window-boundary policy)."""
+    r = ctypes.c_int32()
+    _check(load().fd_cache_window_full(cache.handle, layer, rollout, frames, ctypes.byref(r)),
+           "fd_cache_window_full")
+    return bool(r.value)
 
 
 def fd_exp2_selfcheck(x, y, stream=None) -> None:

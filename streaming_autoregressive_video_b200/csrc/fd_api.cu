@@ -23,8 +23,8 @@ struct fd_cache {
   int device;
   int sms;                      // multiprocessors of the device
   std::vector<int64_t> host_n;  // [L][R] mirror of the device counters
-  CUtensorMap tm_kc, tm_vc;     // bf16 caches: (d, H, slots*Tf, L*R)
-  CUtensorMap tm_kb;            // rotated block keys: (d, H, F*Tf, L*R)
+  CUtensorMap tm_kc, tm_vc;     // bf16 caches: (d, Hkv, slots*Tf, L*R)
+  CUtensorMap tm_kb;            // rotated block keys: (d, Hkv, F*Tf, work_sets*R)
   bool have_maps;
 };
 
@@ -74,6 +74,10 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
       d->shard_index >= shards)
     return FD_ERR_SHAPE;
   const size_t slots = (gslots + shards - 1) / shards;  // local slots
+  // per-call work areas (rotated block keys, split-pair partials, counters)
+  const int32_t sets = d->num_work_sets == 0 ? 1 : d->num_work_sets;
+  if (sets < 1 || sets > d->num_layers) return FD_ERR_SHAPE;
+  const size_t ws_r = (size_t)sets * d->max_rollouts;
   const size_t esz = d->dtype == FD_BF16 ? 2 : 4;
   const int d2 = d->head_dim / 2;
   const int p_hw = d->head_dim / 6;
@@ -101,18 +105,17 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   off = align_up(off + kv);
   lay->kblk = off;
   size_t blk;
-  if (!mul_ok(frame * d->block_frames, lr, &blk) || blk > kRegionMax) return FD_ERR_CAPACITY;
+  if (!mul_ok(frame * d->block_frames, ws_r, &blk) || blk > kRegionMax) return FD_ERR_CAPACITY;
   off = align_up(off + blk);
   // partial results and arrival counters of the persistent bf16 kernel
   const bool tensor_path = d->dtype == FD_BF16;
   const size_t pairs = (T * d->block_frames + 255) / 256;
   lay->part = off;
   if (tensor_path)
-    off = align_up(off + (size_t)d->num_layers * kAttnMaxCtas * 2 * kPartSlotFloats *
-                             sizeof(float));
+    off = align_up(off + (size_t)sets * kAttnMaxCtas * 2 * kPartSlotFloats * sizeof(float));
   lay->cnt = off;
   if (tensor_path) {
-    if (!mul_ok(lr * d->num_heads, pairs * sizeof(int32_t), &x) || x > kRegionMax)
+    if (!mul_ok(ws_r * d->num_heads, pairs * sizeof(int32_t), &x) || x > kRegionMax)
       return FD_ERR_CAPACITY;
     off = align_up(off + x);
   }
@@ -270,6 +273,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.N = desc->num_shards == 0 ? 1 : desc->num_shards;
   v.shard = desc->shard_index;
   v.slots = (v.S + v.W + v.N - 1) / v.N;  // local slots of this shard
+  v.work_sets = desc->num_work_sets == 0 ? 1 : desc->num_work_sets;
   v.nb = (v.F * v.T + 255) / 256;
   v.pt = lay.rope_pairs_t;
   v.ph = lay.rope_pairs_h;
@@ -285,7 +289,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
     if (!fd::encode_bf16_map(&c->tm_kc, v.krot, v.d, v.Hkv, rows, batch) ||
         !fd::encode_bf16_map(&c->tm_vc, v.v, v.d, v.Hkv, rows, batch) ||
         !fd::encode_bf16_map(&c->tm_kb, v.kblk, v.d, v.Hkv, (uint64_t)v.F * v.Tf,
-                             batch)) {
+                             (uint64_t)v.work_sets * v.R)) {
       // only the tensor-core path needs the maps; keep going without them
       c->have_maps = false;
     } else {
@@ -328,6 +332,17 @@ fd_status fd_cache_frames(const fd_cache* cache, int32_t layer,
       rollout >= cache->view.R)
     return FD_ERR_INVALID_ARG;
   *n = cache->host_n[(size_t)layer * cache->view.R + rollout];
+  return FD_OK;
+}
+
+fd_status fd_cache_window_full(const fd_cache* cache, int32_t layer,
+                               int32_t rollout, int32_t frames, int32_t* reached) {
+  if (cache == nullptr || reached == nullptr) return FD_ERR_INVALID_ARG;
+  const fd::CacheView& v = cache->view;
+  if (layer < 0 || layer >= v.L || rollout < 0 || rollout >= v.R) return FD_ERR_INVALID_ARG;
+  if (frames < 1 || frames > v.F) return FD_ERR_INVALID_ARG;
+  const int64_t n = cache->host_n[(size_t)layer * v.R + rollout];
+  *reached = n + frames > (int64_t)v.S + v.W ? 1 : 0;
   return FD_OK;
 }
 
@@ -409,11 +424,13 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   fd::AttnParams p;
   memset(&p, 0, sizeof(p));
   p.q = q;
-  // the block's keys, rotated once for all query tiles (see fd.h, kblk),
-  // in the layer's work area of the cache or in the caller's `work`
+  // the call's work set: the block's keys, rotated once for all query tiles
+  // (see fd.h, kblk), the split-pair partials and their counters; the keys
+  // go to the caller's `work` instead when one is given
+  const int ws = layer % c.work_sets;
   void* kblk = work != nullptr
       ? work
-      : static_cast<void*>(c.kblk + (size_t)layer * c.R * c.F * c.frame_bytes);
+      : static_cast<void*>(c.kblk + (size_t)ws * c.R * c.F * c.frame_bytes);
   p.k = kblk;
   p.v = v_;
   p.pos = c.pos + (size_t)layer * c.R * c.slots;
@@ -428,8 +445,8 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.err = c.err;
   p.kc = c.krot + (size_t)layer * cache->layout.layer_kv_bytes;
   p.vc = c.v + (size_t)layer * cache->layout.layer_kv_bytes;
-  p.part = c.part + (size_t)layer * fd::kAttnMaxCtas * 2 * fd::kPartSlotFloats;
-  p.cnt = c.cnt + (size_t)layer * c.R * c.H * c.nb;
+  p.part = c.part + (size_t)ws * fd::kAttnMaxCtas * 2 * fd::kPartSlotFloats;
+  p.cnt = c.cnt + (size_t)ws * c.R * c.H * c.nb;
   p.nb = c.nb;
   p.H = c.H;
   p.Hkv = c.Hkv;
@@ -449,7 +466,7 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.pw = c.pw;
   p.n_rollouts = n_rollouts;
   p.map_row0 = layer * c.R;
-  p.kb_row0 = work != nullptr ? 0 : layer * c.R;
+  p.kb_row0 = work != nullptr ? 0 : ws * c.R;
   p.div_T = fd::make_fastdiv((uint32_t)c.T);
   p.div_Tf = fd::make_fastdiv((uint32_t)c.Tf);
   p.div_gw = fd::make_fastdiv((uint32_t)c.gw);
@@ -459,9 +476,9 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  // bf16 with d = 128 runs on the tensor cores; fp32, and bf16 of the other
-  // head sizes, on CUDA cores
-  const bool tensor_cores = cache->desc.dtype == FD_BF16 && c.d == 128;
+  // bf16 with d = 128 or 64 runs on the tensor cores; fp32, and bf16 of the
+  // other head sizes, on CUDA cores
+  const bool tensor_cores = cache->desc.dtype == FD_BF16 && (c.d == 128 || c.d == 64);
   if (tensor_cores ? !cache->have_maps : (c.d % 32 != 0 || c.d > 128))
     return FD_ERR_UNSUPPORTED;
   // The tensor-core kernel splits a query index q < Mq into (frame, token,

@@ -91,14 +91,14 @@ struct CacheView {
   uint8_t* k;
   uint8_t* v;
   uint8_t* krot;  // committed keys rotated to their frame's position
-  uint8_t* kblk;  // per-layer work area: the block's keys rotated per call
+  uint8_t* kblk;  // work areas: the block's keys rotated per call
   int32_t* pos;
   int32_t* count;
   float2* ttab;
   float2* htab;
   float2* wtab;
-  float* part;    // [L][kAttnMaxCtas][2][kPartSlotFloats] (bf16 caches)
-  int32_t* cnt;   // [L][R][H][nb] (bf16 caches)
+  float* part;    // [work_sets][kAttnMaxCtas][2][kPartSlotFloats] (bf16 caches)
+  int32_t* cnt;   // [work_sets][R][H][nb] (bf16 caches)
   int32_t* err;
   int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz, nb;
   int Hkv;               // key/value heads (divides H)
@@ -107,13 +107,14 @@ struct CacheView {
   // at local index s / N; `slots` above counts local slots, S and W stay the
   // ring's global sink and window counts, count[] the global frame counter.
   int N, shard;
+  int work_sets;  // per-call work areas; layer l uses set l % work_sets
   double theta;
   uint64_t frame_bytes;  // Tf * Hkv * d * esz (one frame of K or V)
 };
 
 // Persistent tensor-core attention: at most this many CTAs, each with two
 // partial-result slots of kPartSlotFloats floats (O [256][128], m [256],
-// l [256]) per layer.
+// l [256]) per work set.
 constexpr int kAttnMaxCtas = 148;
 constexpr size_t kPartSlotFloats = 256 * 128 + 2 * 256;
 
@@ -184,7 +185,7 @@ cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
                                    int n_rollouts, const void* k, void* out,
                                    cudaStream_t s);
 // attention on CUDA cores in fp32 arithmetic: fp32 caches of any head size
-// d in {32, 64, 96, 128}; bf16 caches (esz = 2) whose d is not 128
+// d in {32, 64, 96, 128}; bf16 caches (esz = 2) whose d is 32 or 96
 cudaError_t launch_attn_cuda_core(const AttnParams& p, int esz, cudaStream_t s);
 // bf16 output rows and log-sum-exp of rollouts with no key on this shard
 cudaError_t launch_attn_zero_keyless(const AttnParams& p, cudaStream_t s);
@@ -214,7 +215,7 @@ cudaError_t launch_bounded_wait_selftest(int32_t* err, uint64_t limit_ns,
                                          cudaStream_t s);
 
 // Shared body of the attention entry points.  `work` is a device area for the
-// block's rotated keys ([n_rollouts][F*Tf][H][d], block_work_bytes bytes,
+// block's rotated keys ([n_rollouts][F*Tf][Hkv][d], block_work_bytes bytes,
 // 16-byte aligned) or nullptr for the layer's work area in the cache storage.
 fd_status block_attention_impl(fd_cache* cache, int32_t layer,
                                int32_t n_rollouts, const void* q,

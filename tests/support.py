@@ -15,8 +15,8 @@ TOL_BF16_MEAN = 2e-3
 TOL_F32_MAX = 1e-4
 
 
-def new_cache(w, device="cuda", shards=1, shard=0):
-    desc = fd.make_desc(w, shards=shards, shard=shard)
+def new_cache(w, device="cuda", shards=1, shard=0, work_sets=1):
+    desc = fd.make_desc(w, shards=shards, shard=shard, work_sets=work_sets)
     nbytes = fd.fd_cache_bytes(desc)
     assert nbytes > 0
     storage = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)

@@ -40,15 +40,23 @@ def test_cache_bytes_and_layout():
                    lay.ttab, lay.htab, lay.wtab, lay.err]
         assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
         assert lay.v - lay.k >= kv and lay.krot - lay.v >= kv and lay.kblk - lay.krot >= kv
-        blk = w.layers * w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * esz
-        assert lay.part - lay.kblk >= blk
-        # partial results of split query-tile pairs: 148 CTAs x 2 slots per
-        # layer, fp32 O [256][128] + max + sum; none for fp32 caches
-        part = w.layers * 148 * 2 * (256 * 128 + 512) * 4 if w.dtype == "bf16" else 0
+        # one work set by default: the block's rotated keys, the split-pair
+        # partial results (148 CTAs x 2 slots, fp32 O [256][128] + max + sum)
+        # and their counters, for one call at a time; none of the latter two
+        # for fp32 caches
+        blk = w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * esz
+        assert blk <= lay.part - lay.kblk < blk + 1024
+        part = 148 * 2 * (256 * 128 + 512) * 4 if w.dtype == "bf16" else 0
         assert part <= lay.cnt - lay.part < part + 1024
         pairs = -(-w.block_frames * w.tokens // 256)
-        cnt = w.layers * w.rollouts * w.heads * pairs * 4 if w.dtype == "bf16" else 0
+        cnt = w.rollouts * w.heads * pairs * 4 if w.dtype == "bf16" else 0
         assert cnt <= lay.pos - lay.cnt < cnt + 1024
+        # one work set per layer multiplies the three by L and nothing else
+        lay_l = fd.fd_cache_get_layout(fd.make_desc(w, work_sets=w.layers))
+        assert lay_l.part - lay_l.kblk >= w.layers * blk
+        assert lay_l.cnt - lay_l.part >= w.layers * part
+        assert lay_l.pos - lay_l.cnt >= w.layers * cnt
+        assert (lay_l.total - lay.total) - (w.layers - 1) * (blk + part + cnt) < 3 * 1024
         assert (lay.rope_pairs_t, lay.rope_pairs_h, lay.rope_pairs_w) == \
             (w.head_dim // 2 - 2 * (w.head_dim // 6), w.head_dim // 6, w.head_dim // 6)
 
@@ -56,10 +64,27 @@ def test_cache_bytes_and_layout():
 def test_single_480p_cache_is_about_3_gb():
     n = fd.fd_cache_bytes(fd.make_desc(SINGLE_480P))
     # 30 layers x 7 slots x 1560 tokens x 12 heads x 128 x 2 B x (K, V, rotated K)
-    # + the per-layer work area for the block's rotated keys (3 frames)
-    # + the per-layer partial-result slots of the attention kernel
-    part = 30 * 148 * 2 * (256 * 128 + 512) * 4
-    assert abs(n - 30 * (7 * 3 + 3) * 1560 * 12 * 128 * 2 - part) < 1 << 20
+    # + one work area for the block's rotated keys (3 frames)
+    # + one set of partial-result slots of the attention kernel
+    part = 148 * 2 * (256 * 128 + 512) * 4
+    assert abs(n - (30 * 7 * 3 + 3) * 1560 * 12 * 128 * 2 - part) < 1 << 20
+    assert n <= 3.1e9
+    # K and V as the method keeps them: 2.01 GB
+    assert 30 * 7 * 2 * 1560 * 12 * 128 * 2 == 2012774400
+
+
+def test_large_model_cache_holds_little_beyond_its_keys_and_values():
+    from streaming_autoregressive_video_b200.workloads import LARGE_ACTIONS as w
+    n = fd.fd_cache_bytes(fd.make_desc(w))
+    kv = 2 * w.layers * w.slots * w.frame_tokens * w.heads * w.head_dim * 2  # K and V
+    # K and V, the rotated keys (half of that again) and one work set
+    assert n <= 1.5 * kv + 0.2e9 and n <= 25.5e9
+
+
+@pytest.mark.parametrize("sets", [-1, 31])
+def test_work_sets_outside_one_to_layers_rejected(sets):
+    desc = fd.make_desc(SINGLE_480P, work_sets=sets)
+    assert fd.fd_cache_bytes(desc) == 0
 
 
 @pytest.mark.parametrize("field,value,status", [
