@@ -129,22 +129,33 @@ __device__ __forceinline__ uint4 rotate16(uint4 u, int pair0, const CacheView& c
   return rotate16_cs<Elem>(u, cs);
 }
 
-// One block copies a 64 KB chunk of one frame of K or V of one (layer,
-// rollout) into the frame's ring slot; K chunks also go, rotated to the
-// frame's position t = n + f, into the rotated-key region.  16-byte vectors,
-// 16 per thread in flight.  grid = (chunks per frame, nl * nr * 2 * F).
+// Commit copy: every CTA takes a run of token rows of one frame of one
+// (layer, rollout); one warp per token row.  For its row a warp loads the
+// block's K and V chunks (16-byte vectors, up to 2 x 8 per lane in flight),
+// then stores K and V into the frame's ring slot and K, rotated to the frame's
+// position t = n + f, into the rotated-key region.  K and V of a row travel
+// together, so every CTA does the same work (per row: two reads and three
+// writes of a row's size).  Index arithmetic
+// is per row (token -> (h, w)); inside a row the lanes step through 32-bit
+// chunk indices, and when every chunk a lane touches holds the same rotation
+// pairs (32 is a multiple of the chunks per head row) their cos/sin are looked
+// up once per row.  grid = (ceil(Tf / rows per CTA), nl * nr * F).
 constexpr int kCopyThreads = 256;
-constexpr int kCopyVecs = 16;
+constexpr int kCopyVecs = 16;  // 16-byte vectors per thread of the reset kernel
+constexpr int kCommitWarps = kCopyThreads / 32;
+constexpr int kCommitRowsPerWarp = 8;
+constexpr int kCommitRowsPerCta = kCommitWarps * kCommitRowsPerWarp;
+constexpr int kCommitBatch = 8;  // chunks per lane and tensor in flight
 
-template <typename Elem>
-__global__ void __launch_bounds__(kCopyThreads)
+template <typename Elem, bool kFixedPairs>
+__global__ void __launch_bounds__(kCopyThreads, 2)
     commit_copy_kernel(CacheView c, CommitParams p) {
-  constexpr int kPer = 16 / sizeof(Elem);
+  constexpr int kPer = 16 / sizeof(Elem);  // elements per 16-byte chunk
+  constexpr int kPairs = kPer / 2;         // rotation pairs per chunk
   const int job = blockIdx.y;
   const int f = job % c.F;
-  const int kv = (job / c.F) & 1;
-  const int ri = (job / c.F / 2) % p.nr;
-  const int li = job / c.F / 2 / p.nr;
+  const int ri = (job / c.F) % p.nr;
+  const int li = job / c.F / p.nr;
   if (f >= p.frames[ri]) return;
   const int l = p.layer0 + li, r = p.rollout0 + ri;
   const size_t lr = (size_t)l * c.R + r;
@@ -152,43 +163,59 @@ __global__ void __launch_bounds__(kCopyThreads)
   const int gslot = slot_of(n + f, c.S, c.W);
   if (gslot % c.N != c.shard) return;  // another shard stores this frame
   const int slot = gslot / c.N;          // local slot
-  const uint64_t fvecs = c.frame_bytes / 16;
-  const uint8_t* src_base = kv ? p.v[li] : p.k[li];
-  const uint4* src = reinterpret_cast<const uint4*>(
-      src_base + ((uint64_t)r * c.F + f) * c.frame_bytes);
+  const uint32_t cpr = (uint32_t)c.d / kPer;      // chunks per head row
+  const uint32_t row_chunks = cpr * (uint32_t)c.Hkv;  // chunks per token row
+  const uint64_t src_off = ((uint64_t)r * c.F + f) * c.frame_bytes;
   const uint64_t dst_off = (lr * c.slots + slot) * c.frame_bytes;
-  uint4* dst = reinterpret_cast<uint4*>((kv ? c.v : c.k) + dst_off);
-  const uint64_t v0 = (uint64_t)blockIdx.x * kCopyThreads * kCopyVecs + threadIdx.x;
-  uint4 buf[kCopyVecs];
-#pragma unroll
-  for (int i = 0; i < kCopyVecs; ++i) {
-    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
-    if (vi < fvecs) buf[i] = __ldcs(src + vi);
-  }
-#pragma unroll
-  for (int i = 0; i < kCopyVecs; ++i) {
-    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
-    if (vi < fvecs) dst[vi] = buf[i];
-  }
-  if (kv) return;
-  // rotated keys: the ttab row slots + f holds frame n + f (the next block)
+  const uint4* ksrc = reinterpret_cast<const uint4*>(p.k[li] + src_off);
+  const uint4* vsrc = reinterpret_cast<const uint4*>(p.v[li] + src_off);
+  uint4* kdst = reinterpret_cast<uint4*>(c.k + dst_off);
+  uint4* vdst = reinterpret_cast<uint4*>(c.v + dst_off);
   uint4* rdst = reinterpret_cast<uint4*>(c.krot + dst_off);
+  // the ttab row slots + f holds frame n + f (the next block's frame f)
   const float2* tt_row = c.ttab + (lr * (c.slots + c.F) + c.slots + f) * c.pt;
-  const uint32_t vec_per_row = c.d / kPer;
-  const uint32_t vec_per_tok = vec_per_row * c.Hkv;
-#pragma unroll
-  for (int i = 0; i < kCopyVecs; ++i) {
-    const uint64_t vi = v0 + (uint64_t)i * kCopyThreads;
-    if (vi >= fvecs) continue;
-    const uint32_t tok = (uint32_t)(vi / vec_per_tok);
-    const int pair0 = (int)(vi % vec_per_row) * (kPer / 2);
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = threadIdx.x & 31;
+  // kFixedPairs: 32 % cpr == 0 (chosen by the host)
+  constexpr int kBatch = kFixedPairs ? kCommitBatch : kCommitBatch / 2;
+  const int row_end = min(c.Tf, (int)(blockIdx.x + 1) * kCommitRowsPerCta);
+  for (int tok = blockIdx.x * kCommitRowsPerCta + warp; tok < row_end; tok += kCommitWarps) {
     int hh = 0, ww = 0;
-    if ((int)tok < c.T) {
-      const int tv = (int)tok % c.Tv;  // position inside the token's view
+    if (tok < c.T) {
+      const int tv = tok % c.Tv;  // position inside the token's view
       hh = tv / c.gw;
       ww = tv - hh * c.gw;
     }
-    rdst[vi] = rotate16<Elem>(buf[i], pair0, c, tt_row, hh, ww);
+    const uint64_t row = (uint64_t)tok * row_chunks;
+    const uint4* ks = ksrc + row;
+    const uint4* vs = vsrc + row;
+    uint4* kd = kdst + row;
+    uint4* vd = vdst + row;
+    uint4* rd = rdst + row;
+    float2 cs[kPairs];
+    if (kFixedPairs) rope_cs(cs, (int)(lane % cpr) * kPairs, c, tt_row, hh, ww);
+    for (uint32_t c0 = lane; c0 < row_chunks; c0 += 32 * kBatch) {
+      uint4 kb[kBatch], vb[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const uint32_t ci = c0 + 32 * i;
+        if (ci < row_chunks) {
+          kb[i] = __ldcs(ks + ci);
+          vb[i] = __ldcs(vs + ci);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const uint32_t ci = c0 + 32 * i;
+        if (ci < row_chunks) {
+          kd[ci] = kb[i];
+          vd[ci] = vb[i];
+          rd[ci] = kFixedPairs
+                       ? rotate16_cs<Elem>(kb[i], cs)
+                       : rotate16<Elem>(kb[i], (int)(ci % cpr) * kPairs, c, tt_row, hh, ww);
+        }
+      }
+    }
   }
 }
 
@@ -321,14 +348,17 @@ cudaError_t launch_cache_init(const CacheView& c, cudaStream_t s) {
 
 cudaError_t launch_commit(const CacheView& c, const CommitParams& p,
                           cudaStream_t s) {
-  const uint64_t fvecs = c.frame_bytes / 16;
-  const uint64_t chunks = (fvecs + kCopyThreads * kCopyVecs - 1) /
-                          (kCopyThreads * kCopyVecs);
-  dim3 grid((unsigned)chunks, (unsigned)(p.nl * p.nr * 2 * c.F));
-  if (c.esz == 2)
-    commit_copy_kernel<uint16_t><<<grid, kCopyThreads, 0, s>>>(c, p);
-  else
-    commit_copy_kernel<float><<<grid, kCopyThreads, 0, s>>>(c, p);
+  const unsigned row_blocks = (unsigned)((c.Tf + kCommitRowsPerCta - 1) / kCommitRowsPerCta);
+  dim3 grid(row_blocks, (unsigned)(p.nl * p.nr * c.F));
+  // whether every chunk a lane touches holds the same rotation pairs
+  const bool fixed = 32 % (c.d * c.esz / 16) == 0;
+  if (c.esz == 2) {
+    if (fixed) commit_copy_kernel<uint16_t, true><<<grid, kCopyThreads, 0, s>>>(c, p);
+    else commit_copy_kernel<uint16_t, false><<<grid, kCopyThreads, 0, s>>>(c, p);
+  } else {
+    if (fixed) commit_copy_kernel<float, true><<<grid, kCopyThreads, 0, s>>>(c, p);
+    else commit_copy_kernel<float, false><<<grid, kCopyThreads, 0, s>>>(c, p);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   commit_meta_kernel<<<p.nl * p.nr, 128, 0, s>>>(c, p);
