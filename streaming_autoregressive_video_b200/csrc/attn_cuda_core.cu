@@ -8,7 +8,7 @@
 // 2026 write-up, section VII: next frame from historical clean frames and the
 // current noisy frame).  It serves fp32 caches, where the tolerance leaves no
 // room for TF32 rounding, and bf16 caches whose head size the tensor-core
-// kernel does not take (d = 32, 64, 96): bf16 values are widened to fp32 as
+// kernel does not take (d = 32, 96): bf16 values are widened to fp32 as
 // they are staged and the output is rounded to bf16 once, at the end.
 //
 // One CTA = (query tile of 32 rows, head, rollout); 8 warps x 4 rows.  Keys

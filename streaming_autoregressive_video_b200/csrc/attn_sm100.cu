@@ -69,29 +69,27 @@ using namespace sm100;
 constexpr int kThreads = 512;
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
-constexpr int kD = 128;   // head dim handled by this kernel
-constexpr uint32_t kTile = kBM * kD * 2;  // 32 KB (bf16)
-constexpr uint32_t kHalf = kTile / 2;     // one 64-column, 128-byte-swizzled half
+// one 64-column, 128-byte-swizzled half of a tile: 128 rows x 128 bytes
+constexpr uint32_t kHalf = kBM * 64 * 2;
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = 2 * kTile;
-constexpr uint32_t kOffV = kOffK + kKStages * kTile;
-constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 // Every kPolyEvery-th pair of exponentials on the FMA pipe (0: all on MUFU).
 // With one warpgroup per query tile the MUFU unit is not the limit and the
 // polynomial's extra instructions cost more than they save (measured: 505 us
 // per 480p call all on MUFU, 521 us with every second pair on the FMA pipe).
 constexpr int kPolyEvery = 0;
+// Exponentials as packed pairs on MUFU (ex2.approx.ftz.bf16x2): the argument
+// pair is rounded to bf16 and one instruction returns both weights as bf16,
+// already in the layout the PV product reads.
+constexpr bool kExpPairs = false;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
 
-// TMEM columns
+// TMEM columns: S0 at 0, S1 at 128 (128 keys each), O0 at 256, O1 at 256 + D
 constexpr uint32_t kColS0 = 0, kColO0 = 256;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD, true);
 
 struct Shared {
   uint64_t q_full, q_ready, q_empty;
@@ -107,12 +105,29 @@ struct Shared {
   int32_t last;       // this piece arrived last: it writes the unit's rows
 };
 
-// RoPE tables follow the barriers; the dynamic size adds them per launch.
-constexpr uint32_t kOffMeta = kOffShared + 256;  // struct Meta
-constexpr uint32_t kOffTab = kOffMeta + 256;
 static_assert(sizeof(Shared) <= 256, "barrier block");
 constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
-constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + 1024: base alignment slack
+
+// Shared-memory layout and per-head-size constants of the kernel for head
+// size D (64 or 128): Q (two tiles), K and V stages of 128 rows x D bf16, each
+// tile stored as D/64 column halves of 128 rows x 128 bytes (one 128-byte
+// swizzle atom per row), then the barriers, the piece ring and the RoPE
+// tables (the dynamic size adds the tables per launch).
+template <int D>
+struct Geo {
+  static_assert(D == 64 || D == 128, "head size of the tensor-core kernel");
+  static constexpr uint32_t kTile = kBM * D * 2;  // 32 KB (D = 128) or 16 KB
+  static constexpr int kHalves = D / 64;
+  static constexpr int kChunks = D / 8;           // 16-byte chunks per row
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = 2 * kTile;
+  static constexpr uint32_t kOffV = kOffK + kKStages * kTile;
+  static constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
+  static constexpr uint32_t kOffMeta = kOffShared + 256;  // struct Meta
+  static constexpr uint32_t kOffTab = kOffMeta + 256;
+  static constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + base alignment slack
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
+};
 
 // Site codes for the device error word.
 enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4,
@@ -317,12 +332,13 @@ struct RopeLane {
   int half, chunk, row0;
 };
 
+template <int D>
 __device__ __forceinline__ RopeLane rope_lane(const AttnParams& p, int tid) {
   RopeLane rl;
-  const int cc = tid & 15;
+  const int cc = tid % Geo<D>::kChunks;
   rl.half = cc >> 3;
   rl.chunk = cc & 7;
-  rl.row0 = tid >> 4;
+  rl.row0 = tid / Geo<D>::kChunks;
   const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
@@ -364,13 +380,16 @@ __device__ __forceinline__ void rotate_chunk(uint8_t* tile, int row,
 }
 
 // Rotate the 128 query rows of a Q tile (rows past Mq are zero: skipped).
+// The 128 threads cover 128 / kChunks rows per pass.
+template <int D>
 __device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
                                             const RopeLane& rl,
                                             const float2* tab,
                                             const AttnParams& p) {
+  constexpr int kRowsPerPass = 128 / Geo<D>::kChunks;
 #pragma unroll 4
-  for (int m = 0; m < 16; ++m) {
-    const int row = rl.row0 + 8 * m;
+  for (int m = 0; m < Geo<D>::kChunks; ++m) {
+    const int row = rl.row0 + kRowsPerPass * m;
     const int q = qrow0 + row;
     if (q >= p.Mq) continue;
     const int f = (int)fast_div((uint32_t)q, p.div_T);
@@ -456,18 +475,18 @@ __device__ __forceinline__ bool read_piece_len(const Meta* meta, int k, int& n, 
   return true;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_bf16_d128_sm100(const __grid_constant__ CUtensorMap tm_q,
-                         const __grid_constant__ CUtensorMap tm_kc,
-                         const __grid_constant__ CUtensorMap tm_vc,
-                         const __grid_constant__ CUtensorMap tm_kb,
-                         const __grid_constant__ CUtensorMap tm_vb,
-                         const __grid_constant__ AttnParams p) {
+template <int D>
+__device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtensorMap& tm_kc,
+                                          const CUtensorMap& tm_vc, const CUtensorMap& tm_kb,
+                                          const CUtensorMap& tm_vb, const AttnParams& p) {
+  using G = Geo<D>;
+  constexpr uint32_t kTile = G::kTile;
+  constexpr uint32_t kOffQ = G::kOffQ, kOffK = G::kOffK, kOffV = G::kOffV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Shared* sh = reinterpret_cast<Shared*>(smem + kOffShared);
-  Meta* meta = reinterpret_cast<Meta*>(smem + kOffMeta);
+  Shared* sh = reinterpret_cast<Shared*>(smem + G::kOffShared);
+  Meta* meta = reinterpret_cast<Meta*>(smem + G::kOffMeta);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -565,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e->seq = k;
         mbar_arrive_expect_tx(&sh->q_full, 2 * kTile);
         for (int t = 0; t < 2; ++t)
-          for (int hf = 0; hf < 2; ++hf)
+          for (int hf = 0; hf < G::kHalves; ++hf)
             tma_load_4d(smem + kOffQ + t * kTile + hf * kHalf, &tm_q, &sh->q_full,
                         hf * 64, pc.h, pc.b * 2 * kBM + t * kBM, pc.r);
         issued_q = k + 1;
@@ -589,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&sh->k_full[ks], kTile);
-          for (int hf = 0; hf < 2; ++hf)
+          for (int hf = 0; hf < G::kHalves; ++hf)
             tma_load_4d(smem + kOffK + ks * kTile + hf * kHalf, mk,
                         &sh->k_full[ks], hf * 64, hkv, key0, ck3);
           issued_k = g + 1;
@@ -601,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&sh->v_full[vs], kTile);
-          for (int hf = 0; hf < 2; ++hf)
+          for (int hf = 0; hf < G::kHalves; ++hf)
             tma_load_4d(smem + kOffV + vs * kTile + hf * kHalf, mv,
                         &sh->v_full[vs], hf * 64, hkv, key0, cv3);
           issued_v = g + 1;
@@ -636,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t a = q_lo + x * (kTile >> 4), b = k_lo + ks * (kTile >> 4);
         asm volatile("" : "+r"(a), "+r"(b));
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t step = (kk >> 2) * (kHalf >> 4) + (kk & 3) * 2;  // 32 B per k-step
           mma_ss_lo(tmem + kColS0 + x * 128, a + step, b + step, desc_hi, kIdescQK, kk > 0);
         }
@@ -646,8 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("" : "+r"(b));
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_ts_lo(tmem + kColO0 + x * 128, tmem + kColS0 + x * 128 + kk * 8,
-                    b + kk * (2048 >> 4), desc_hi, kIdescPV, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_lo(tmem + kColO0 + x * D, tmem + kColS0 + x * 128 + kk * 8,
+                    b + kk * (2048 >> 4), desc_hi, G::kIdescPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       // K tiles arrive rotated (cache keys at commit, block keys once per
@@ -732,9 +751,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<72>();
     // ------------------------------------------------------------ RoPE
     const int tid = threadIdx.x - 128;
-    const RopeLane rl = rope_lane(p, tid);
+    const RopeLane rl = rope_lane<D>(p, tid);
     // this rollout's t table and the static h / w tables, in shared memory
-    float2* st = reinterpret_cast<float2*>(smem + kOffTab);
+    float2* st = reinterpret_cast<float2*>(smem + G::kOffTab);
     const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph, n_w = p.gw * p.pw;
     int staged = -1;
     uint32_t n_stage = 0;
@@ -764,8 +783,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         staged = pi.r;
       }
       const int qrow0 = pi.b * 2 * kBM;
-      rope_q_tile(smem + kOffQ, qrow0, rl, st, p);
-      rope_q_tile(smem + kOffQ + kTile, qrow0 + kBM, rl, st, p);
+      rope_q_tile<D>(smem + kOffQ, qrow0, rl, st, p);
+      rope_q_tile<D>(smem + kOffQ + kTile, qrow0 + kBM, rl, st, p);
       fence_proxy_async_smem();
       mbar_arrive(&sh->q_ready);
     }
@@ -784,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row_t = wq * 32 + lane;  // row within the tile
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS0 + x * 128;
-    const uint32_t tO = tmem + lane_off + kColO0 + x * 128;
+    const uint32_t tO = tmem + lane_off + kColO0 + x * D;
     const float sl2 = p.scale_log2;
     int g = 0;  // KV iterations this warpgroup's tile has run (its barriers' phases)
     uint32_t n_part = 0;
@@ -841,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jj > 0 && __any_sync(0xffffffffu, need)) {
           const float alpha = need ? ex2_approx(m - m_tile) : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < D / 16; ++c) {
             uint32_t r16[16];
             tmem_ld16(tO + c * 16, r16);
 #pragma unroll
@@ -869,6 +888,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) {
             const uint64_t x2 = f2_fma(
                 f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
+            if constexpr (kExpPairs) {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              const uint32_t pb = ex2_bf16x2(pack_bf16(x0, x1));
+              pk[i] = pb;
+              ls2 = f2_add(ls2, f2_pack(__uint_as_float(pb << 16),
+                                        __uint_as_float(pb & 0xFFFF0000u)));
+              continue;
+            }
             uint64_t e2;
             constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
             if (kPolyEvery > 0 && full && (i % kEvery) == kEvery - 1) {
@@ -922,16 +950,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 (pi.U0 + pi.kv0 == meta->my_begin ? 0 : 1)) * kPartSlotFloats;
         uint32_t rr[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, rr);
-          float4* dst = reinterpret_cast<float4*>(part + (size_t)row * kD + c * 32);
+          float4* dst = reinterpret_cast<float4*>(part + (size_t)row * D + c * 32);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             dst[i] = make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
                                  __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3]));
         }
-        part[2 * kBM * kD + row] = m;
-        part[2 * kBM * kD + 2 * kBM + row] = l;
+        part[2 * kBM * D + row] = m;
+        part[2 * kBM * D + 2 * kBM + row] = l;
         __threadfence();
         mbar_arrive(&sh->part_bar);
         if (threadIdx.x == 256) {
@@ -968,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (write_rows) {
         // row = sum over pieces i of O_i 2^(m_i - M) / sum of l_i 2^(m_i - M),
         // M the largest max; this CTA's own piece comes from TMEM
-        constexpr size_t kOffM = 2 * kBM * kD, kOffL = kOffM + 2 * kBM;
+        constexpr size_t kOffM = 2 * kBM * D, kOffL = kOffM + 2 * kBM;
         const int qrow = pi.b * 2 * kBM + row;
         auto skip = [&](int c) {
           return c != (int)blockIdx.x && cta_begin(c, sd, p.G) == cta_begin(c + 1, sd, p.G);
@@ -989,10 +1017,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float inv_l = 1.f / L;
         uint16_t* out = static_cast<uint16_t*>(p.out) +
-                        (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * kD;
+                        (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * D;
         uint32_t rr[32];
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, rr);
           float acc[32];
 #pragma unroll
@@ -1005,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int i = 0; i < 32; ++i) acc[i] += w * __uint_as_float(rr[i]);
             } else {
               const float4* src = reinterpret_cast<const float4*>(
-                  part_slot(p, c2, pi.U0, sd) + (size_t)row * kD + c * 32);
+                  part_slot(p, c2, pi.U0, sd) + (size_t)row * D + c * 32);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const float4 f = __ldcg(src + i);
@@ -1041,12 +1069,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// The kernels for head sizes 128 and 64 (the same body, instantiated).
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_d128_sm100(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_kc,
+                         const __grid_constant__ CUtensorMap tm_vc,
+                         const __grid_constant__ CUtensorMap tm_kb,
+                         const __grid_constant__ CUtensorMap tm_vb,
+                         const __grid_constant__ AttnParams p) {
+  attn_body<128>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_bf16_d64_sm100(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_kc,
+                        const __grid_constant__ CUtensorMap tm_vc,
+                        const __grid_constant__ CUtensorMap tm_kb,
+                        const __grid_constant__ CUtensorMap tm_vb,
+                        const __grid_constant__ AttnParams p) {
+  attn_body<64>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
+}
+
+using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                            const CUtensorMap, const CUtensorMap, const AttnParams);
+
+// The warpgroup register split (setmaxnreg) assumes the block launches with
+// exactly 128 registers per thread; refuse to launch otherwise, as the
+// increase would wait forever for registers that do not exist.
+cudaError_t prepare_kernel(AttnKernel k) {
+  cudaFuncAttributes fa;
+  cudaError_t err = cudaFuncGetAttributes(&fa, k);
+  if (err != cudaSuccess) return err;
+  if (fa.numRegs != 128) return cudaErrorNotSupported;
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kSmemMax);
+}
+
 }  // namespace
 
 size_t attn_bf16_smem_bytes(const AttnParams& p) {
+  if (p.d != 64 && p.d != 128) return 0;
   const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
                                         (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
-  const size_t smem = kSmemFixed + tab;
+  const size_t fixed = p.d == 128 ? Geo<128>::kSmemFixed : Geo<64>::kSmemFixed;
+  const size_t smem = fixed + tab;
   return smem > kSmemMax ? 0 : smem;
 }
 
@@ -1058,23 +1124,17 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const AttnParams& p, cudaStream_t s) {
   static PerDeviceOnce attr;
   cudaError_t e = once_per_device(attr, [] {
-    // The warpgroup register split (setmaxnreg) assumes the block launches
-    // with exactly 128 registers per thread; refuse to launch otherwise, as
-    // the increase would wait forever for registers that do not exist.
-    cudaFuncAttributes fa;
-    cudaError_t err = cudaFuncGetAttributes(&fa, attn_bf16_d128_sm100);
-    if (err != cudaSuccess) return err;
-    if (fa.numRegs != 128) return cudaErrorNotSupported;
-    return cudaFuncSetAttribute(attn_bf16_d128_sm100,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kSmemMax);
+    cudaError_t err = prepare_kernel(attn_bf16_d128_sm100);
+    return err == cudaSuccess ? prepare_kernel(attn_bf16_d64_sm100) : err;
   });
   if (e != cudaSuccess) return e;
   const size_t smem = attn_bf16_smem_bytes(p);
   if (smem == 0) return cudaErrorNotSupported;
   if (p.G < 1 || p.G > kAttnMaxCtas) return cudaErrorInvalidValue;
-  attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb,
-                                                   tm_vb, p);
+  if (p.d == 128)
+    attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
+  else
+    attn_bf16_d64_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
   count_launch(1);
   return cudaGetLastError();
 }

@@ -103,10 +103,11 @@ def test_attention_f32_tiny_rollout(kv_heads, views):
     (32, dict(rollouts=2, sink_frames=2, window_frames=2)),     # sinks straddled
     (96, dict(grid_h=5, grid_w=7, action_tokens=1)),        # d/2 = 48 pairs: t/h/w = 16/16/16
 ])
-def test_attention_bf16_cuda_core_head_sizes(d, shape):
-    """bf16 caches with d != 128 run on the CUDA-core kernel (fp32 arithmetic
-    on the stored bf16 values): a rollout through empty, partial, full and
-    wrapped cache states against the oracle at the bf16 tolerance."""
+def test_attention_bf16_head_sizes(d, shape):
+    """bf16 caches with d = 64 run on the tensor-core kernel's 64-column
+    instance, d = 32 and 96 on the CUDA-core kernel (fp32 arithmetic on the
+    stored bf16 values): a rollout through empty, partial, full and wrapped
+    cache states against the oracle at the bf16 tolerance."""
     w = SMALL.scaled(head_dim=d, blocks=5, **shape)
     ls = Lockstep(w)
     for blk in range(w.blocks):
@@ -116,6 +117,25 @@ def test_attention_bf16_cuda_core_head_sizes(d, shape):
         _commit_block(ls, w, 700 + blk)
         ls.check_cache_exact()
         ls.check_rotated_keys()
+    assert fd.fd_get_device_error(ls.cache) == 0
+
+
+def test_attention_bf16_d64_tensor_cores_480p_shape():
+    """The d = 64 tensor-core instance at the 480p frame shape (30x52 grid,
+    3-frame blocks, 1 sink + 6 window frames, cache full): many query-tile
+    pairs per head, split between CTAs, against the oracle on sampled rows of
+    every head (rows from every query tile, the ragged last one included)."""
+    from streaming_autoregressive_video_b200.workloads import SINGLE_480P
+    w = SINGLE_480P.scaled(name="480p-d64", head_dim=64, heads=4, layers=1)
+    ls = Lockstep(w)
+    for blk in range(3):
+        _commit_block(ls, w, 900 + blk)
+    ls.check_cache_exact()
+    ls.check_rotated_keys()
+    rows = np.unique(np.concatenate([np.arange(0, w.queries, 37), [w.queries - 1]]))
+    for step in range(2):
+        q, k, v = block_inputs(w, (901, step), 1)
+        ls.attention(0, q, k, v, rows=rows, what=f"480p d64 step {step}")
     assert fd.fd_get_device_error(ls.cache) == 0
 
 
