@@ -8,7 +8,7 @@ into every layer's ring buffer.  The cache is full (steady state) before the
 timed region, so every call attends to sinks + the whole window + the block.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fd|reference]
-                    [--workload 480p|large|long|ragged|multiview|gqa]
+                    [--workload 480p|tiny|large|long|ragged|multiview|gqa|d64]
 
 N > 1 runs one independent replica per GPU (the path has no exchange step):
 value = work of all ranks / max-over-ranks time ("scaling": "weak").
@@ -36,13 +36,16 @@ METRIC = ("chunk-attention TFLOP/s & latent-frames/s per layer; "
 PROFILE = os.path.join(ROOT, "profiles", "attn_bf16_d128_sm100.480p.md")
 KERNEL_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
                           "attn_sm100.cu")
+COMMIT_PROFILE = os.path.join(ROOT, "profiles", "commit_copy_kernel.480p_l30.md")
+COMMIT_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
+                          "cache_kernels.cu")
 
 
 def workloads():
     from streaming_autoregressive_video_b200 import workloads as wl
-    return {"480p": wl.SINGLE_480P, "large": wl.LARGE_ACTIONS,
+    return {"480p": wl.SINGLE_480P, "tiny": wl.TINY_F32, "large": wl.LARGE_ACTIONS,
             "long": wl.LONG_ROLLOUT, "ragged": wl.BATCHED_RAGGED,
-            "multiview": wl.MULTIVIEW_4, "gqa": wl.GQA_480P}
+            "multiview": wl.MULTIVIEW_4, "gqa": wl.GQA_480P, "d64": wl.D64_480P}
 
 
 def parse_args():
@@ -54,6 +57,8 @@ def parse_args():
     ap.add_argument("--workload", default="480p")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the finalize-overlap and other-workload measurements")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases only)")
     return ap.parse_args()
@@ -88,12 +93,12 @@ def measured_peaks():
             "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def profile_traffic():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+def _traffic_from(profile, source):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel source (sha256 recorded in the summary)."""
     try:
-        text = open(PROFILE).read()
-        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+        text = open(profile).read()
+        src = hashlib.sha256(open(source, "rb").read()).hexdigest()
     except OSError:
         return None
     m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
@@ -101,6 +106,14 @@ def profile_traffic():
     if not m_sha or not m_tr or m_sha.group(1) != src:
         return None
     return float(m_tr.group(1))
+
+
+def profile_traffic():
+    return _traffic_from(PROFILE, KERNEL_SRC)
+
+
+def commit_traffic():
+    return _traffic_from(COMMIT_PROFILE, COMMIT_SRC)
 
 
 class ClockSampler:
@@ -199,22 +212,36 @@ def workload_config(w, world, rank=0):
 def oracle_call_setup(w, heads):
     import oracle
     from streaming_autoregressive_video_b200 import synth
+    dt = w.dtype
     c = oracle.RolloutCache(w.sink_frames, w.window_frames, w.frame_tokens, w.hkv,
-                            w.head_dim, "bf16")
+                            w.head_dim, dt)
     ks = (w.block_frames, w.frame_tokens, w.hkv, w.head_dim)
     n_commits = -(-w.slots // w.block_frames) + 1
     for b in range(n_commits):
-        c.commit(synth.normal(synth.seed_of(7, b, 0), ks, "bf16", w.value_scale),
-                 synth.normal(synth.seed_of(7, b, 1), ks, "bf16", w.value_scale))
-    q = synth.normal(synth.seed_of(7, 99, 0), (w.queries, w.heads, w.head_dim), "bf16", w.value_scale)
-    k = synth.normal(synth.seed_of(7, 99, 1), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), "bf16", w.value_scale)
-    v = synth.normal(synth.seed_of(7, 99, 2), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), "bf16", w.value_scale)
+        c.commit(synth.normal(synth.seed_of(7, b, 0), ks, dt, w.value_scale),
+                 synth.normal(synth.seed_of(7, b, 1), ks, dt, w.value_scale))
+    q = synth.normal(synth.seed_of(7, 99, 0), (w.queries, w.heads, w.head_dim), dt, w.value_scale)
+    k = synth.normal(synth.seed_of(7, 99, 1), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), dt, w.value_scale)
+    v = synth.normal(synth.seed_of(7, 99, 2), (w.block_frames * w.frame_tokens, w.hkv, w.head_dim), dt, w.value_scale)
     nk = (c.valid_slots() + w.block_frames) * w.frame_tokens
 
     def call():
         oracle.block_attention(c, q, k, v, tokens=w.tokens, grid_w=w.grid_w,
                                theta=w.theta, heads=heads, view_tokens=w.view_tokens)
     return call, 4.0 * len(heads) * w.head_dim * w.queries * nk
+
+
+def cpu_model():
+    """Model name of the host CPU (first entry of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def oracle_threads():
@@ -257,7 +284,7 @@ def cpu_baseline(w):
     call()
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"one full attention call ({w.heads} heads x {w.queries} queries, "
                       f"cache full) in fp64 numpy, {dt:.1f} s"}
 
@@ -283,7 +310,7 @@ def run_reference(args, w, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus), "cpu_baseline": {
             "value": val, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": sample},
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(), "sample": sample},
         "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0}}), flush=True)
 
@@ -291,136 +318,306 @@ def run_reference(args, w, rank):
 # --------------------------------------------------------------------------
 # CUDA path
 # --------------------------------------------------------------------------
-def run_fd(args, w, rank, world, local_rank):
-    import torch
-    import torch.distributed as dist
-    from streaming_autoregressive_video_b200 import binding as fd
-    from streaming_autoregressive_video_b200 import synth
+class Rollout:
+    """One workload on the device: a cache prefilled to steady state (or to
+    its ragged fill), and fresh q/k/v per (denoising step, layer)."""
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    fd.load(build_if_missing=(rank == 0))
-    L, R, S = w.layers, w.rollouts, w.steps
-    F, Tf, H, d = w.block_frames, w.frame_tokens, w.heads, w.head_dim
-    desc = fd.make_desc(w)
-    nbytes = fd.fd_cache_bytes(desc)
-    raw = torch.empty(nbytes + 1024, dtype=torch.uint8, device=dev)
-    off = (-raw.data_ptr()) % 1024
-    storage = raw[off:off + nbytes]
-    cache = fd.fd_cache_create(desc, storage)
+    def __init__(self, w, dev, rank):
+        import torch
+        from streaming_autoregressive_video_b200 import binding as fd
+        from streaming_autoregressive_video_b200 import synth
 
-    def gen(seed, shape):
-        return synth.normal_device(seed, shape, "bf16", dev, w.value_scale).view(torch.int16)
+        self.w, self.dev = w, dev
+        L, R, S = w.layers, w.rollouts, w.steps
+        F, Tf, H, d = w.block_frames, w.frame_tokens, w.heads, w.head_dim
+        self.desc = fd.make_desc(w)
+        self.cache_bytes = fd.fd_cache_bytes(self.desc)
+        raw = torch.empty(self.cache_bytes + 1024, dtype=torch.uint8, device=dev)
+        off = (-raw.data_ptr()) % 1024
+        self.cache = fd.fd_cache_create(self.desc, raw[off:off + self.cache_bytes])
+        self.esz = 2 if w.dtype == "bf16" else 4
+        tdt = torch.int16 if w.dtype == "bf16" else torch.float32
 
-    qshape = (R, w.queries, H, d)
-    kshape = (R, F * Tf, w.hkv, d)
-    base = replica_seed_base(rank)
-    # prefill every layer until the window is full (steady state)
-    pk = [gen(synth.seed_of(base, 1, l), kshape) for l in range(L)]
-    pv = [gen(synth.seed_of(base, 2, l), kshape) for l in range(L)]
-    fill = prefill_frames(w, rank)
-    left = list(fill)
-    while max(left) > 0:
-        fr = [min(F, x) for x in left]
-        fd.fd_cache_commit(cache, 0, L, R, pk, pv, frames=fr)
-        left = [a - b for a, b in zip(left, fr)]
-    torch.cuda.synchronize()
-    # the library's own frame counters agree with the described prefill
-    assert [fd.fd_cache_frames(cache, 0, r) for r in range(R)] == fill
+        def gen(seed, shape):
+            t = synth.normal_device(seed, shape, w.dtype, dev, w.value_scale)
+            return t.view(torch.int16) if w.dtype == "bf16" else t
 
-    def nkeys():
-        return keys_per_rollout(w, fill)
+        self.qshape = (R, w.queries, H, d)
+        self.kshape = (R, F * Tf, w.hkv, d)
+        base = replica_seed_base(rank)
+        pk = [gen(synth.seed_of(base, 1, l), self.kshape) for l in range(L)]
+        pv = [gen(synth.seed_of(base, 2, l), self.kshape) for l in range(L)]
+        self.fill = prefill_frames(w, rank)
+        left = list(self.fill)
+        while max(left) > 0:
+            fr = [min(F, x) for x in left]
+            fd.fd_cache_commit(self.cache, 0, L, R, pk, pv, frames=fr)
+            left = [a - b for a, b in zip(left, fr)]
+        torch.cuda.synchronize()
+        # the library's own frame counters agree with the described prefill
+        assert [fd.fd_cache_frames(self.cache, 0, r) for r in range(R)] == self.fill
+        del pk, pv
+        self.q = [[gen(synth.seed_of(base, 10, s, l), self.qshape) for l in range(L)]
+                  for s in range(S)]
+        self.k = [[gen(synth.seed_of(base, 11, s, l), self.kshape) for l in range(L)]
+                  for s in range(S)]
+        self.v = [[gen(synth.seed_of(base, 12, s, l), self.kshape) for l in range(L)]
+                  for s in range(S)]
+        self.outs = [torch.empty(self.qshape, dtype=tdt, device=dev) for _ in range(L)]
+        self.stream = torch.cuda.current_stream(dev)
+        self.nk = keys_per_rollout(w, self.fill)
+        self.flops_call = attn_flops(w, self.nk)
+        self.bytes_call = attn_bytes(w, self.nk, self.esz)
+        self.kv_bytes = 2 * w.layers * w.rollouts * w.slots * Tf * w.hkv * d * self.esz
+        # one block's commit: read k, v; write K, V and the rotated K
+        self.commit_bytes = 5.0 * L * R * F * Tf * w.hkv * d * self.esz
 
-    q = [[gen(synth.seed_of(base, 10, s, l), qshape) for l in range(L)] for s in range(S)]
-    k = [[gen(synth.seed_of(base, 11, s, l), kshape) for l in range(L)] for s in range(S)]
-    v = [[gen(synth.seed_of(base, 12, s, l), kshape) for l in range(L)] for s in range(S)]
-    outs = [torch.empty(qshape, dtype=torch.int16, device=dev) for _ in range(L)]
-    stream = torch.cuda.current_stream(dev)
-
-    def timed(fn, evs):
+    def _timed(self, fn, evs):
+        import torch
         if evs is None:
             fn()
             return
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+        a.record(self.stream)
         fn()
-        b.record(stream)
+        b.record(self.stream)
         evs.append((a, b))
 
-    def step(evs=None, cevs=None):
+    def step(self, evs=None, cevs=None):
+        """One block: every denoising step through every layer, then one
+        batched commit of the last step's k/v into every layer."""
+        from streaming_autoregressive_video_b200 import binding as fd
+        w, c = self.w, self.cache
+        L, R, S = w.layers, w.rollouts, w.steps
         for s in range(S):
             for l in range(L):
-                timed(lambda: fd.fd_block_attention(cache, l, R, q[s][l], k[s][l], v[s][l],
-                                                    outs[l], stream=stream), evs)
-        timed(lambda: fd.fd_cache_commit(cache, 0, L, R, k[S - 1], v[S - 1], stream=stream),
-              cevs)
+                self._timed(lambda: fd.fd_block_attention(
+                    c, l, R, self.q[s][l], self.k[s][l], self.v[s][l], self.outs[l],
+                    stream=self.stream), evs)
+        self._timed(lambda: fd.fd_cache_commit(c, 0, L, R, self.k[S - 1], self.v[S - 1],
+                                               stream=self.stream), cevs)
+
+    def step_side_commits(self, aux, attn_done, commit_done):
+        """The same block with finalize() in the background: layer l's commit
+        runs on stream `aux` once its last-step attention is done, and the next
+        block's first call on layer l waits for it."""
+        from streaming_autoregressive_video_b200 import binding as fd
+        w, c = self.w, self.cache
+        L, R, S = w.layers, w.rollouts, w.steps
+        for s in range(S):
+            for l in range(L):
+                if s == 0:
+                    self.stream.wait_event(commit_done[l])
+                fd.fd_block_attention(c, l, R, self.q[s][l], self.k[s][l], self.v[s][l],
+                                      self.outs[l], stream=self.stream)
+                if s == S - 1:
+                    attn_done[l].record(self.stream)
+                    aux.wait_event(attn_done[l])
+                    fd.fd_cache_commit(c, l, l + 1, R, [self.k[s][l]], [self.v[s][l]],
+                                       stream=aux)
+                    commit_done[l].record(aux)
+
+    def check(self):
+        from streaming_autoregressive_video_b200 import binding as fd
+        err = fd.fd_get_device_error(self.cache)
+        assert err == 0, f"device error word {err:#x}"
+
+
+def time_steps(ro, steps, warmup, world=1, barrier=None):
+    """Device time of `steps` blocks after `warmup` untimed ones: (ms per
+    step, mean ms per attention call, mean ms per commit)."""
+    import torch
+    for _ in range(warmup):
+        ro.step()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    evs, cevs = [], []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ro.stream)
+    for _ in range(steps):
+        ro.step(evs, cevs)
+    e1.record(ro.stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    ms_step = e0.elapsed_time(e1) / steps
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+    commit_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
+    return ms_step, attn_ms, commit_ms
+
+
+def finalize_overlap(ro, steps):
+    """Step time with one batched commit after the block (serial) and with
+    each layer's commit on a second stream right after its last attention
+    call (finalize() in the background)."""
+    import torch
+    serial = time_steps(ro, steps, 2)[0]
+    aux = torch.cuda.Stream(ro.dev)
+    L = ro.w.layers
+    attn_done = [torch.cuda.Event() for _ in range(L)]
+    commit_done = [torch.cuda.Event() for _ in range(L)]
+    for e in commit_done:
+        e.record(ro.stream)
+    for _ in range(2):
+        ro.step_side_commits(aux, attn_done, commit_done)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ro.stream)
+    for _ in range(steps):
+        ro.step_side_commits(aux, attn_done, commit_done)
+    for e in commit_done:
+        ro.stream.wait_event(e)
+    e1.record(ro.stream)
+    torch.cuda.synchronize()
+    ro.check()
+    return {"ms_per_step_batched_commit": serial,
+            "ms_per_step_side_stream_commits": e0.elapsed_time(e1) / steps,
+            "steps": steps, "layers": L,
+            "how": "per-layer fd_cache_commit on a second stream after the layer's "
+                   "last-step attention (event-ordered), against one batched commit "
+                   "after the block on the same stream"}
+
+
+# secondary workloads timed in the default run: name -> (workload key,
+# layers, steps); layers > 1 give each call its own cache so the K/V come
+# from HBM rather than from L2 (each call has the workload's shape)
+OTHER_CONFIGS = {"tiny": ("tiny", 1, 40), "large": ("large", 4, 4),
+                 "long": ("long", 8, 10), "ragged": ("ragged", 1, 10),
+                 "d64": ("d64", 4, 4)}
+
+
+def other_configs(dev, rank):
+    """Per-call time, TFLOP/s and roofline fraction of the other workloads,
+    each with the clocks seen while it ran."""
+    import gc
+    import torch
+    peaks, src = measured_peaks()
+    res = {}
+    for name, (key, layers, steps) in OTHER_CONFIGS.items():
+        w = workloads()[key]
+        if layers != w.layers:
+            w = w.scaled(layers=layers, name=f"{w.name}-L{layers}")
+        ro = Rollout(w, dev, rank)
+        sampler = ClockSampler(dev.index or 0)
+        sampler.start()
+        ms_step, attn_ms, commit_ms = time_steps(ro, steps, 3)
+        clocks = sampler.stop()
+        ro.check()
+        tf = ro.flops_call / (attn_ms * 1e-3) / 1e12
+        gbs = ro.bytes_call / (attn_ms * 1e-3) / 1e9
+        entry = {"workload": w.name, "dtype": w.dtype, "steps": steps, "layers": layers,
+                 "ms_per_call": attn_ms, "ms_per_step": ms_step, "commit_ms": commit_ms,
+                 "tflops_per_call": tf, "hbm_gbs_per_call": gbs,
+                 "latent_frames_per_s_per_layer":
+                     w.rollouts * w.block_frames * w.layers / (ms_step * 1e-3),
+                 "frac_of_burst_bf16": tf / peaks["bf16_tflops"],
+                 "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                 "commit_frac_of_hbm": ro.commit_bytes / (commit_ms * 1e-3) / 1e9
+                                       / peaks["hbm_gbs"],
+                 "cache_bytes": ro.cache_bytes, "kv_bytes": ro.kv_bytes,
+                 "clocks": clocks}
+        if w.dtype != "bf16":
+            entry["bound"] = "latency (CUDA-core fp32 kernel, launch-sized work)"
+            entry["us_per_call"] = attn_ms * 1e3
+        res[name] = entry
+        del ro
+        gc.collect()
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_fd(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from streaming_autoregressive_video_b200 import binding as fd
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fd.load(build_if_missing=(rank == 0))
+    ro = Rollout(w, dev, rank)
+    L, R, S, F = w.layers, w.rollouts, w.steps, w.block_frames
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     for _ in range(max(3, args.warmup)):
-        step()
+        ro.step()
     torch.cuda.synchronize()
-    nk = nkeys()  # steady state: constant over the timed steps when uniform
-    flops_call = attn_flops(w, nk)
-    bytes_call = attn_bytes(w, nk)
     sampler = ClockSampler(local_rank)
     sampler.start()
-    barrier()
-    torch.cuda.synchronize()
     launches0 = fd.fd_launch_count()
-    evs, cevs = [], []
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step(evs, cevs)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    clocks = sampler.stop()
+    ms_step, attn_ms, commit_ms = time_steps(ro, args.steps, 0, world, barrier)
     launches = fd.fd_launch_count() - launches0
-    ms_step = e0.elapsed_time(e1) / args.steps
-    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
-    commit_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
+    clocks = sampler.stop()
     ms_step, attn_ms, commit_ms = max_over_ranks([ms_step, attn_ms, commit_ms], world, dev)
-    err = fd.fd_get_device_error(cache)
-    assert err == 0, f"device error word {err:#x}"
+    ro.check()
 
-    flops_step = flops_call * S * L
+    flops_step = ro.flops_call * S * L
     value = job_rate(flops_step, world, ms_step) / 1e12
     frames_per_s_layer = job_rate(R * F * L, world, ms_step)
 
     # ---------------- end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world)
+        e2e = run_e2e(args, w, ro.cache, dev, ro.stream, ro.q, ro.k, ro.v, ro.outs,
+                      flops_step, world)
+    overlap = None
+    if not args.no_extra and world == 1:
+        overlap = finalize_overlap(ro, 5)
 
     if rank != 0:
         return
     peaks, src = measured_peaks()
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    achieved = flops_call / (attn_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": profile_traffic(),
-            "kernel": "attn_bf16_d128_sm100", "peak_source": f"{src} bf16_tflops_sustained",
-            "algorithmic_bytes_per_launch": bytes_call,
-            "flops_per_launch": flops_call, "launch_ms": attn_ms,
-            "launch_covers": "fd_block_attention call: block-key RoPE pass + attention kernel"}
+    dtype = "bf16" if w.dtype == "bf16" else "f32"
+    line_extra = {}
+    if w.dtype == "bf16":
+        # the attention kernel runs for a step of tens of ms between host
+        # syncs, not for seconds: its fraction is quoted against the burst
+        # bf16 figure, and against the sustained one for context
+        peak = peaks["bf16_tflops"]
+        achieved = ro.flops_call / (attn_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                # the committed ncu capture is of the 480p call
+                "traffic": profile_traffic() if w.name == workloads()["480p"].name else None,
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+                "kernel": f"attn_bf16_d{w.head_dim}_sm100",
+                "peak_source": f"{src} bf16_tflops (burst)",
+                "algorithmic_bytes_per_launch": ro.bytes_call,
+                "flops_per_launch": ro.flops_call, "launch_ms": attn_ms,
+                "launch_covers": "fd_block_attention call: block-key RoPE pass + attention "
+                                 "kernel"}
+    else:
+        achieved = ro.bytes_call / (attn_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "attn_cuda_core_kernel", "peak_source": f"{src} hbm_gbs",
+                "algorithmic_bytes_per_launch": ro.bytes_call, "launch_ms": attn_ms,
+                "note": "fp32 CUDA-core kernel on a launch-sized call: latency bound",
+                "us_per_call": attn_ms * 1e3}
     # batched commit of all layers: read k, v; write K, V and rotated K
-    commit_bytes = 5.0 * L * R * F * Tf * w.hkv * d * 2
-    commit_roof = {"bound": "hbm", "achieved": commit_bytes / (commit_ms * 1e-3) / 1e9,
-                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                   "frac": commit_bytes / (commit_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                   "traffic": None, "kernel": "commit_copy_kernel + commit_meta_kernel",
-                   "peak_source": f"{src} hbm_gbs", "algorithmic_bytes_per_launch": commit_bytes,
+    commit_gbs = ro.commit_bytes / (commit_ms * 1e-3) / 1e9
+    commit_roof = {"bound": "hbm", "achieved": commit_gbs, "peak": peaks["hbm_gbs"],
+                   "unit": "GB/s", "frac": commit_gbs / peaks["hbm_gbs"],
+                   "traffic": commit_traffic() if w.name == workloads()["480p"].name else None,
+                   "frac_4stream": 0.8 * commit_gbs / peaks["hbm_gbs"],
+                   "kernel": "commit_copy_kernel + commit_meta_kernel",
+                   "peak_source": f"{src} hbm_gbs",
+                   "algorithmic_bytes_per_launch": ro.commit_bytes,
+                   "bytes_counted": "read k, v; write K, V, rotated K (5 element streams); "
+                                    "frac_4stream counts only read k, v + write K, V",
                    "launch_ms": commit_ms, "layers_per_launch": L}
+    cfg = workload_config(w, world, rank)
+    cfg.update(cache_bytes=ro.cache_bytes, kv_bytes=ro.kv_bytes)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world, rank),
+        "dtype": dtype, "data": "synthetic",
+        "config": cfg,
         "latent_frames_per_s_per_layer": frames_per_s_layer,
         "roofline": roof,
         "commit_roofline": commit_roof,
@@ -428,6 +625,12 @@ def run_fd(args, w, rank, world, local_rank):
         "clocks": clocks,
         "e2e": e2e,
     }
+    line.update(line_extra)
+    if overlap is not None:
+        line["finalize_overlap"] = overlap
+    if world == 1 and not args.no_extra and args.workload == "480p":
+        del ro
+        line["other_configs"] = other_configs(dev, rank)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -436,7 +639,10 @@ def run_fd(args, w, rank, world, local_rank):
 def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
     """Same steps through the C ABI with the q/k/v of every call copied from
     pinned host memory and every output copied back, inside the timed region.
-    Copies run on their own streams so they overlap the kernels."""
+    Copies run on their own streams so they overlap the kernels.  The host
+    buffers hold the first denoising step's q/k/v of every layer and are sent
+    again at every step and block: the copies move the bytes of fresh inputs,
+    which is what the end-to-end figure measures."""
     import torch
     import torch.distributed as dist
     from streaming_autoregressive_video_b200 import binding as fd
@@ -445,7 +651,7 @@ def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
     hq = [t.cpu().pin_memory() for t in q[0]]
     hk = [t.cpu().pin_memory() for t in k[0]]
     hv = [t.cpu().pin_memory() for t in v[0]]
-    hout = [torch.empty(outs[0].shape, dtype=torch.int16).pin_memory() for _ in range(L)]
+    hout = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory() for _ in range(L)]
     nbuf = 2
     dq = [torch.empty_like(q[0][0]) for _ in range(nbuf)]
     dk = [torch.empty_like(k[0][0]) for _ in range(nbuf)]
@@ -484,8 +690,8 @@ def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
                 with torch.cuda.stream(d2h):
                     hout[l].copy_(dout[b], non_blocking=True)
                 freed[b].record(d2h)
-                h2d_bytes += (hq[l].numel() + hk[l].numel() + hv[l].numel()) * 2
-                d2h_bytes += hout[l].numel() * 2
+                h2d_bytes += sum(t.numel() * t.element_size() for t in (hq[l], hk[l], hv[l]))
+                d2h_bytes += hout[l].numel() * hout[l].element_size()
                 i += 1
         fd.fd_cache_commit(cache, 0, L, R, klast, vlast, stream=stream)
 

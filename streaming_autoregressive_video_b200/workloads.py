@@ -123,5 +123,9 @@ MULTIVIEW_4 = Workload("bf16-4x44x80-h16-d128-F1-S1-W3", layers=28, rollouts=1,
 #    heads): a cache-semantics variant, not a configuration of the pages
 GQA_480P = SINGLE_480P.scaled(name="bf16-30x52-h12kv4-d128-F3-S1-W6-L30", kv_heads=4)
 
+# 8: the 480p shape with head size 64 (the test matrix's second head size; 24
+#    heads of 64 keep the 1536-wide model of the 12 x 128 workload)
+D64_480P = SINGLE_480P.scaled(name="bf16-30x52-h24-d64-F3-S1-W6-L30", head_dim=64, heads=24)
+
 ALL = [TINY_F32, SINGLE_480P, LARGE_ACTIONS, LONG_ROLLOUT, BATCHED_RAGGED, MULTIVIEW_4,
-       GQA_480P]
+       GQA_480P, D64_480P]

@@ -47,13 +47,16 @@ class _Stream:
         pass
 
 
+torch.cuda.empty_cache = lambda: None
+
+
 torch.cuda.Event = _Event
 torch.cuda.Stream = _Stream
 torch.cuda.current_stream = lambda *a: _Stream()
 torch.cuda.stream = lambda s: contextlib.nullcontext()
 torch.Tensor.pin_memory = lambda self: self
 synth.normal_device = lambda seed, shape, dtype, dev, scale=1.0: torch.zeros(
-    shape, dtype=torch.bfloat16)
+    shape, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
 
 _state = {"n": None, "launches": 0}
 
@@ -109,5 +112,5 @@ if __name__ == "__main__":
     layers = int(sys.argv[2]) if len(sys.argv) > 2 else 2
     w = w.scaled(layers=min(w.layers, layers))
     args = types.SimpleNamespace(steps=2, warmup=3, no_e2e=False, no_cpu_baseline=True,
-                                 gpus=1)
+                                 gpus=1, no_extra=False, workload=sys.argv[1])
     bench.run_fd(args, w, 0, 1, 0)

@@ -24,7 +24,7 @@ def _stub_line(workload):
     return json.loads(res.stdout.strip().splitlines()[-1])
 
 
-@pytest.mark.parametrize("workload", ["480p", "gqa", "ragged", "multiview"])
+@pytest.mark.parametrize("workload", ["480p", "gqa", "ragged", "multiview", "tiny"])
 def test_gpu_arm_line_keeps_the_contract(workload):
     line = _stub_line(workload)
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
@@ -37,22 +37,50 @@ def test_gpu_arm_line_keeps_the_contract(workload):
     roof = line["roofline"]
     for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert key in roof, key
-    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+    w0 = bench.workloads()[workload]
+    if w0.dtype == "bf16":
+        assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s"
+        assert line["dtype"] == "bf16"
+    else:
+        assert roof["bound"] == "hbm" and roof["unit"] == "GB/s" and line["dtype"] == "f32"
     assert roof["frac"] == pytest.approx(roof["achieved"] / roof["peak"])
+    esz = 2 if w0.dtype == "bf16" else 4
     e2e = line["e2e"]
     for key in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
         assert key in e2e, key
-    w0 = bench.workloads()[workload]
     w = w0.scaled(layers=min(w0.layers, 2))   # as bench_stub.py runs it
     # every call copies q, k, v in and out back: bytes from the tensors' sizes
-    q = w.rollouts * w.queries * w.heads * w.head_dim * 2
-    kv = w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * 2
+    q = w.rollouts * w.queries * w.heads * w.head_dim * esz
+    kv = w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * esz
     calls = w.steps * w.layers
     assert e2e["h2d_bytes_per_step"] == calls * (q + 2 * kv)
     assert e2e["d2h_bytes_per_step"] == calls * q
     assert line["gpu_launches"] > 0
     # commit bytes: read k, v; write K, V and rotated K, with Hkv heads
     assert line["commit_roofline"]["algorithmic_bytes_per_launch"] == 5 * w.layers * kv
+    assert line["commit_roofline"]["frac_4stream"] == pytest.approx(
+        0.8 * line["commit_roofline"]["frac"])
+    # the cache's storage and the K/V the method keeps
+    assert line["config"]["cache_bytes"] == fd_cache_bytes(w)
+    assert line["config"]["kv_bytes"] == 2 * w.layers * w.rollouts * w.slots * \
+        w.frame_tokens * w.hkv * w.head_dim * esz
+    fo = line["finalize_overlap"]
+    assert fo["layers"] == w.layers and fo["ms_per_step_side_stream_commits"] > 0
+    if workload == "480p":
+        oc = line["other_configs"]
+        assert sorted(oc) == ["d64", "large", "long", "ragged", "tiny"]
+        for name, e in oc.items():
+            for key in ("ms_per_call", "tflops_per_call", "frac_of_burst_bf16", "clocks",
+                        "commit_frac_of_hbm", "workload"):
+                assert key in e, (name, key)
+        assert oc["tiny"]["dtype"] == "f32" and "us_per_call" in oc["tiny"]
+    else:
+        assert "other_configs" not in line
+
+
+def fd_cache_bytes(w):
+    from streaming_autoregressive_video_b200 import binding as fd
+    return fd.fd_cache_bytes(fd.make_desc(w))
 
 
 def test_reference_arm_line_matches_the_gpu_arm_config(capsys):
