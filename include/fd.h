@@ -39,8 +39,9 @@
  *   - the cache stores K/V as committed (pre-RoPE) plus an int32 frame
  *     position per slot; a cached key's rotation depends only on that
  *     position, so the commit also stores it rotated (krot).  Each attention
- *     call rotates the block's keys once into a work area (kblk) that all
- *     query tiles read, and rotates each query tile as it is loaded.
+ *     call on the tensor cores rotates the block's keys once into a work area
+ *     (kblk) that all query tiles read, and rotates each query tile as it is
+ *     loaded (the CUDA-core kernel rotates both as it stages them).
  *
  * Conventions for every call:
  *   - all pointers to tensors are DEVICE pointers on the device that owns the
@@ -253,9 +254,10 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
  * carved from a pool or arena someone else sizes, or a process that may not
  * call cudaMalloc at all (it can synchronise the device, which a real-time
  * serving loop cannot afford).  Same arguments, semantics and results as
- * fd_block_attention; the work area for the block's rotated keys is instead a
- * static device array of FD_STATIC_WORK_BYTES inside this library, which
- * every GPU that loads the library holds until the process exits.
+ * fd_block_attention; the work area for the block's rotated keys (used by
+ * the tensor-core kernels) is instead a static device array of
+ * FD_STATIC_WORK_BYTES inside this library, which every GPU that loads the
+ * library holds until the process exits.
  *   - FD_ERR_CAPACITY (before any launch) when n_rollouts*F*Tf*Hkv*d*element
  *     size (the block's rotated keys, Hkv key/value heads) exceeds
  *     FD_STATIC_WORK_BYTES;

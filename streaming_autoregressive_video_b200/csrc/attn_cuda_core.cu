@@ -11,10 +11,14 @@
 // kernel does not take (d = 32, 96): bf16 values are widened to fp32 as
 // they are staged and the output is rounded to bf16 once, at the end.
 //
-// One CTA = (query tile of 32 rows, head, rollout); 8 warps x 4 rows.  Keys
-// are staged 64 at a time in shared memory, rotated in fp32; within a warp
-// lane j scores key j, then the warp forms the online softmax and each lane
-// accumulates d/32 output dimensions.
+// One CTA = (query tile of 8 x kRowsPerWarp rows, head, rollout); 8 warps,
+// each kRowsPerWarp rows (4 for calls with many rows; 1 when 4 would leave
+// most multiprocessors idle, as in launch-sized calls, where the warps' serial
+// row loops are the latency).  Keys are staged 64 at a time in smem (the
+// cache's keys arrive rotated, the block's keys are rotated in fp32 as they
+// are staged); within a warp lane j scores key j (four independent partial
+// sums over the head dimension), then the warp forms the online softmax and
+// each lane accumulates d/32 output dimensions.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -26,8 +30,6 @@ namespace fd {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kRowsPerWarp = 4;
-constexpr int kRows = kWarps * kRowsPerWarp;  // 32 query rows per CTA
 constexpr int kKeys = 64;                     // keys per staged tile
 
 struct KeyCoord {
@@ -58,9 +60,10 @@ __device__ __forceinline__ void store_elem(uint16_t* x, float v) {
 }
 
 // Elem: float (fp32 cache) or uint16_t (bf16 bit patterns)
-template <typename Elem, int D>
+template <typename Elem, int D, int kRowsPerWarp>
 __global__ void __launch_bounds__(kWarps * 32)
     attn_cuda_core_kernel(AttnParams p) {
+  constexpr int kRows = kWarps * kRowsPerWarp;  // query rows per CTA
   constexpr int kPerLane = D / 32;
   extern __shared__ float sm[];
   float* Qs = sm;                          // [kRows][D]
@@ -121,12 +124,21 @@ __global__ void __launch_bounds__(kWarps * 32)
         const size_t off = seg1
             ? (((size_t)r * p.slots * p.Tf + key) * p.Hkv + hk) * D + 2 * pair
             : (((size_t)r * p.F * p.Tf + key) * p.Hkv + hk) * D + 2 * pair;
-        // keys arrive rotated: cached frames were rotated when committed, the
-        // block's keys once per call before this kernel
+        // cached frames' keys arrive rotated (at commit); the block's keys
+        // are rotated here, frame f of the block at t-row slots + f
         const float2 kx = load_pair((seg1 ? kcg : kg) + off);
         const float2 vx = load_pair((seg1 ? vcg : vg) + off);
         a = kx.x;
         b = kx.y;
+        if (!seg1) {
+          const int f = key / p.Tf, tok = key - f * p.Tf;
+          const int tv = tok % p.Tv;  // inside its view; action tokens at (0, 0)
+          const KeyCoord kc{p.slots + f, tok < p.T ? tv / p.gw : 0,
+                            tok < p.T ? tv % p.gw : 0};
+          const float2 cs = rope_cs(p, tt, pair, kc);
+          a = kx.x * cs.x - kx.y * cs.y;
+          b = kx.x * cs.y + kx.y * cs.x;
+        }
         va = vx.x;
         vb = vx.y;
       }
@@ -143,9 +155,15 @@ __global__ void __launch_bounds__(kWarps * 32)
       for (int sub = 0; sub < kKeys / 32; ++sub) {
         const int kr = sub * 32 + lane;
         const bool valid = key0 + kr < nseg;
-        float s = 0.f;
+        // four independent partial sums shorten the dependent FMA chain
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
-        for (int e = 0; e < D; ++e) s = fmaf(qrow[e], Ks[kr * (D + 1) + e], s);
+        for (int e = 0; e < D; e += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            s4[u] = fmaf(qrow[e + u], Ks[kr * (D + 1) + e + u], s4[u]);
+        }
+        float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         s = valid ? s * p.scale : -INFINITY;
         float mt = s;
 #pragma unroll
@@ -190,19 +208,29 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-template <typename Elem, int D>
-cudaError_t launch_d(const AttnParams& p, cudaStream_t s) {
+template <typename Elem, int D, int kRowsPerWarp>
+cudaError_t launch_rows(const AttnParams& p, cudaStream_t s) {
+  constexpr int kRows = kWarps * kRowsPerWarp;
   const size_t smem = sizeof(float) * (kRows * D + kKeys * (D + 1) + kKeys * D);
   static PerDeviceOnce attr;
   cudaError_t e = once_per_device(attr, [smem] {
-    return cudaFuncSetAttribute(attn_cuda_core_kernel<Elem, D>,
+    return cudaFuncSetAttribute(attn_cuda_core_kernel<Elem, D, kRowsPerWarp>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   });
   if (e != cudaSuccess) return e;
   dim3 grid((p.Mq + kRows - 1) / kRows, p.H, p.n_rollouts);
-  attn_cuda_core_kernel<Elem, D><<<grid, kWarps * 32, smem, s>>>(p);
+  attn_cuda_core_kernel<Elem, D, kRowsPerWarp><<<grid, kWarps * 32, smem, s>>>(p);
   count_launch(1);
   return cudaGetLastError();
+}
+
+// Four rows per warp unless that leaves fewer CTAs than multiprocessors
+// (148 on B200): then one row per warp, four times the CTAs.
+template <typename Elem, int D>
+cudaError_t launch_d(const AttnParams& p, cudaStream_t s) {
+  const int64_t ctas4 = (int64_t)((p.Mq + 4 * kWarps - 1) / (4 * kWarps)) * p.H * p.n_rollouts;
+  if (ctas4 < kAttnMaxCtas) return launch_rows<Elem, D, 1>(p, s);
+  return launch_rows<Elem, D, 4>(p, s);
 }
 
 }  // namespace

@@ -516,12 +516,16 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
     if (it_max * g >= ((int64_t)1 << 31)) return FD_ERR_UNSUPPORTED;
     p.G = (int)g;
   }
+  // the CUDA-core kernel rotates the block's keys as it stages them
+  if (!tensor_cores) {
+    p.k = k;
+    return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
+  }
   // the block's keys belong to shard 0; other shards never read them
   if (c.shard == 0) {
     st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
     if (st != FD_OK) return st;
   }
-  if (!tensor_cores) return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
   if (c.shard != 0) {
     // rollouts with no key on this shard get zero rows and lse = -inf here;
     // the tensor-core kernel skips them

@@ -140,8 +140,9 @@ struct ResetParams {
 
 // Parameters of the attention kernels (the tensor maps travel separately).
 struct AttnParams {
-  const void* q;         // block tensors (CUDA-core path reads them directly)
-  const void* k;
+  const void* q;         // block tensors, as given (pre-RoPE)
+  const void* k;         // block keys: rotated (work area) for the tensor-core
+                         // kernel, as given for the CUDA-core kernel
   const void* v;
   const int32_t* pos;    // [R][slots] of the layer
   const int32_t* count;  // [R] of the layer
