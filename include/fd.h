@@ -39,9 +39,9 @@
  *   - the cache stores K/V as committed (pre-RoPE) plus an int32 frame
  *     position per slot; a cached key's rotation depends only on that
  *     position, so the commit also stores it rotated (krot).  Each attention
- *     call on the tensor cores rotates the block's keys once into a work area
- *     (kblk) that all query tiles read, and rotates each query tile as it is
- *     loaded (the CUDA-core kernel rotates both as it stages them).
+ *     call on the tensor cores first rotates the block's keys and queries
+ *     once, into work areas (kblk, qblk) that the attention kernel copies
+ *     tiles from (the CUDA-core kernel rotates both as it stages them).
  *
  * Conventions for every call:
  *   - all pointers to tensors are DEVICE pointers on the device that owns the
@@ -135,6 +135,8 @@ typedef struct {
  *   kblk : [Wk][R][F*Tf][Hkv][d] work area of fd_block_attention: the
  *          current block's keys rotated once per call, read by every query
  *          tile (one set per work set, see num_work_sets)
+ *   qblk : [Wk][R][F*T][H][d] work area of the same calls: the block's
+ *          queries rotated once per call (bf16 caches; empty for fp32)
  *   part : [Wk][148][2][256*128 + 512] float work area of the bf16 attention
  *          kernel: a CTA whose share of the work ends or begins inside a
  *          query tile pair leaves its partial result there (unnormalised
@@ -149,7 +151,7 @@ typedef struct {
  *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
  *   err  : int32 device error word (0 = none)                            */
 typedef struct {
-  size_t k, v, krot, kblk, part, cnt, pos, count, ttab, htab, wtab, err;
+  size_t k, v, krot, kblk, qblk, part, cnt, pos, count, ttab, htab, wtab, err;
   size_t total;           /* == fd_cache_bytes(desc)                       */
   size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
   int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
@@ -234,13 +236,13 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * CUDA cores in fp32 arithmetic (no TF32; bf16 output rounded once).  Other head sizes
  * return FD_ERR_UNSUPPORTED before any launch.  Tensor bases must be 16-byte
  * aligned.
- * The bf16 kernel is persistent (one CTA per multiprocessor, at most 148)
- * and splits the call's KV iterations evenly over its CTAs; it returns
- * FD_ERR_UNSUPPORTED when n_rollouts x H x ceil(F*T/256) x (ceil((S+W)*Tf
- * /128) + ceil(F*Tf/128)) x CTAs reaches 2^31, or when F*T x T reaches 2^40
- * (its query-coordinate arithmetic), or when the RoPE tables of the call
- * (S+W+F t-rows, the h and w tables) do not fit in shared memory.  A query-tile pair split
- * between CTAs is combined through the layer's `part` / `cnt` regions.
+ * On the tensor cores a pass first rotates the block's queries and keys into
+ * the call's work set (qblk, kblk); the attention kernel is persistent (one
+ * CTA per multiprocessor, at most 148) and splits the call's KV iterations
+ * evenly over its CTAs; it returns FD_ERR_UNSUPPORTED when n_rollouts x H x
+ * ceil(F*T/256) x (ceil((S+W)*Tf/128) + ceil(F*Tf/128)) x CTAs reaches 2^31.
+ * A query-tile pair split between CTAs is combined through the work set's
+ * `part` / `cnt` regions.
  * Device-side waits are bounded: a wait that gives up sets the error word
  * (fd_get_device_error) instead of hanging. */
 fd_status fd_block_attention(fd_cache* cache, int32_t layer,
@@ -254,12 +256,13 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
  * carved from a pool or arena someone else sizes, or a process that may not
  * call cudaMalloc at all (it can synchronise the device, which a real-time
  * serving loop cannot afford).  Same arguments, semantics and results as
- * fd_block_attention; the work area for the block's rotated keys (used by
- * the tensor-core kernels) is instead a static device array of
- * FD_STATIC_WORK_BYTES inside this library, which every GPU that loads the
- * library holds until the process exits.
- *   - FD_ERR_CAPACITY (before any launch) when n_rollouts*F*Tf*Hkv*d*element
- *     size (the block's rotated keys, Hkv key/value heads) exceeds
+ * fd_block_attention; the work area for the block's rotated keys and queries
+ * (used by the tensor-core kernels; CUDA-core calls need none) is instead a
+ * static device array of FD_STATIC_WORK_BYTES inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *   - FD_ERR_CAPACITY (before any launch) when a tensor-core call's
+ *     n_rollouts*F*(Tf*Hkv + T*H)*d*2 bytes (the block's rotated keys with
+ *     Hkv key/value heads and its rotated queries with H heads) exceed
  *     FD_STATIC_WORK_BYTES;
  *   - the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress), so make that first call before any stream

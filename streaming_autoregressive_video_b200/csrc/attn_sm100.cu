@@ -7,11 +7,11 @@
 // Memory for Infinite Rollouts) and all tokens of the block itself, which
 // attend to each other bidirectionally ("Cosmos3-H-Dreams" model card, Model
 // Architecture: block-causal student with a KV cache; AlpaDreams GTC 2026
-// write-up, section VII).  q' and k' carry 3D (t,h,w) RoPE: each query tile
-// is rotated as it lands in shared memory; keys arrive rotated (cache keys
-// were rotated once when their frame was committed, the block's keys once per
-// call by a pass over the block before this kernel), because every query
-// tile of a head reads the same keys.
+// write-up, section VII).  q' and k' carry 3D (t,h,w) RoPE and arrive rotated:
+// cache keys were rotated once when their frame was committed, the block's
+// queries and keys once per call by a pass over the block before this kernel
+// (every query tile of a head reads the same keys, and a rotated query tile
+// can be copied straight into the tensor core's operand layout).
 //
 // Schedule (persistent): a work unit is one 256-row query-tile pair of one
 // (rollout, head) against all of the rollout's KV tiles.  The units' KV
@@ -37,9 +37,7 @@
 //                 two query tiles ping-pong so one tile's softmax overlaps the
 //                 other tile's matrix products.
 //   warp 2        TMEM allocator (512 columns: S0, S1, O0, O1).
-//   warps 4-7     RoPE: rotate each piece's Q tiles in place in the swizzled
-//                 shared-memory layout, cos/sin from the cache's tables
-//                 (fp64-accurate angles rounded once to fp32).
+//   warps 4-7     no role (their registers go to the softmax warpgroups).
 //   warps 8-15    softmax: warpgroup x owns query tile x, one thread per
 //                 query row (TMEM lane), all 128 columns: row max, exp2, row
 //                 sum, P rounded to bf16 and written back into the S columns
@@ -79,10 +77,6 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 // polynomial's extra instructions cost more than they save (measured: 505 us
 // per 480p call all on MUFU, 521 us with every second pair on the FMA pipe).
 constexpr int kPolyEvery = 0;
-// Exponentials as packed pairs on MUFU (ex2.approx.ftz.bf16x2): the argument
-// pair is rounded to bf16 and one instruction returns both weights as bf16,
-// already in the layout the PV product reads.
-constexpr bool kExpPairs = false;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
 
@@ -92,12 +86,11 @@ constexpr uint32_t kColS0 = 0, kColO0 = 256;
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN, false);
 
 struct Shared {
-  uint64_t q_full, q_ready, q_empty;
+  uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_empty, drain;
-  uint64_t tab_bar;   // RoPE warpgroup: tables of the next rollout staged
   uint64_t part_bar;  // softmax: a piece's partial rows written
   uint64_t last_bar;  // softmax: the piece's arrival counted
   uint32_t tmem_base;
@@ -111,26 +104,23 @@ constexpr uint32_t kSmemMax = 232448;  // per-block opt-in limit on sm_100
 // Shared-memory layout and per-head-size constants of the kernel for head
 // size D (64 or 128): Q (two tiles), K and V stages of 128 rows x D bf16, each
 // tile stored as D/64 column halves of 128 rows x 128 bytes (one 128-byte
-// swizzle atom per row), then the barriers, the piece ring and the RoPE
-// tables (the dynamic size adds the tables per launch).
+// swizzle atom per row), then the barriers and the piece ring.
 template <int D>
 struct Geo {
   static_assert(D == 64 || D == 128, "head size of the tensor-core kernel");
   static constexpr uint32_t kTile = kBM * D * 2;  // 32 KB (D = 128) or 16 KB
   static constexpr int kHalves = D / 64;
-  static constexpr int kChunks = D / 8;           // 16-byte chunks per row
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = 2 * kTile;
   static constexpr uint32_t kOffV = kOffK + kKStages * kTile;
   static constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
   static constexpr uint32_t kOffMeta = kOffShared + 256;  // struct Meta
-  static constexpr uint32_t kOffTab = kOffMeta + 256;
-  static constexpr uint32_t kSmemFixed = kOffTab + 1024;  // + base alignment slack
+  static constexpr uint32_t kSmemFixed = kOffMeta + 256 + 1024;  // + base alignment slack
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
 };
 
 // Site codes for the device error word.
-enum : int { kSiteProducer = 1, kSiteRope = 2, kSiteMma = 3, kSiteSoftmax = 4,
+enum : int { kSiteProducer = 1, kSiteMma = 3, kSiteSoftmax = 4,
              kSiteSelftest = 5 };
 
 // Bounded wait.  kSpin (MMA issuer, softmax: the critical path) polls, so
@@ -316,91 +306,6 @@ struct Meta {
 };
 static_assert(sizeof(Meta) <= 256, "meta block");
 
-// ---------------------------------------------------------------- RoPE
-// Thread `tid` (0..127) of the RoPE warpgroup owns 16-byte chunk cc = tid%16
-// of every row (8 bf16 = 4 rotation pairs: pairs 4cc..4cc+3) and rows
-// tid/16 + 8m.  A 128-byte-swizzled row keeps each 16-byte chunk intact, so
-// the pairs of a chunk stay together; only the chunk's position moves.
-// cos/sin come from one table in shared memory: [t rows of this rollout |
-// h rows | w rows].  A lane's pair p reads entry off[p] + coord * stride[p],
-// where coord is the key's t-row, h or w; the choice is a select, not a
-// branch, so the lanes of a warp never diverge on the lookup.
-struct RopeLane {
-  int sec[4];     // 0 = t, 1 = h, 2 = w
-  int off[4];     // section base + pair index within the section
-  int stride[4];  // pairs of the section
-  int half, chunk, row0;
-};
-
-template <int D>
-__device__ __forceinline__ RopeLane rope_lane(const AttnParams& p, int tid) {
-  RopeLane rl;
-  const int cc = tid % Geo<D>::kChunks;
-  rl.half = cc >> 3;
-  rl.chunk = cc & 7;
-  rl.row0 = tid / Geo<D>::kChunks;
-  const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int pair = cc * 4 + e;
-    if (pair < p.pt) {
-      rl.sec[e] = 0; rl.off[e] = pair; rl.stride[e] = p.pt;
-    } else if (pair < p.pt + p.ph) {
-      rl.sec[e] = 1; rl.off[e] = n_t + pair - p.pt; rl.stride[e] = p.ph;
-    } else {
-      rl.sec[e] = 2; rl.off[e] = n_t + n_h + pair - p.pt - p.ph; rl.stride[e] = p.pw;
-    }
-  }
-  return rl;
-}
-
-__device__ __forceinline__ void rotate_chunk(uint8_t* tile, int row,
-                                             const RopeLane& rl,
-                                             const float2* tab, int tidx,
-                                             int hh, int ww) {
-  float2 cs[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int coord = rl.sec[e] == 0 ? tidx : (rl.sec[e] == 1 ? hh : ww);
-    cs[e] = tab[rl.off[e] + coord * rl.stride[e]];
-  }
-  uint4* ptr = reinterpret_cast<uint4*>(tile + rl.half * kHalf + row * 128 +
-                                        ((rl.chunk ^ (row & 7)) << 4));
-  uint4 u = *ptr;
-  uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float a = __uint_as_float(w4[e] << 16);
-    const float b = __uint_as_float(w4[e] & 0xFFFF0000u);
-    const __nv_bfloat162 r2 = __floats2bfloat162_rn(
-        a * cs[e].x - b * cs[e].y, a * cs[e].y + b * cs[e].x);
-    w4[e] = *reinterpret_cast<const uint32_t*>(&r2);
-  }
-  *ptr = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-}
-
-// Rotate the 128 query rows of a Q tile (rows past Mq are zero: skipped).
-// The 128 threads cover 128 / kChunks rows per pass.
-template <int D>
-__device__ __forceinline__ void rope_q_tile(uint8_t* tile, int qrow0,
-                                            const RopeLane& rl,
-                                            const float2* tab,
-                                            const AttnParams& p) {
-  constexpr int kRowsPerPass = 128 / Geo<D>::kChunks;
-#pragma unroll 4
-  for (int m = 0; m < Geo<D>::kChunks; ++m) {
-    const int row = rl.row0 + kRowsPerPass * m;
-    const int q = qrow0 + row;
-    if (q >= p.Mq) continue;
-    const int f = (int)fast_div((uint32_t)q, p.div_T);
-    const int tq = q - f * p.T;
-    const int tok = tq - (int)fast_div((uint32_t)tq, p.div_Tv) * p.Tv;  // inside its view
-    const int hh = (int)fast_div((uint32_t)tok, p.div_gw);
-    rotate_chunk(tile, row, rl, tab, p.slots + f, hh, tok - hh * p.gw);
-  }
-}
-
-
 // End of every role branch: all 512 threads meet on named barrier 1 (each
 // warp arrives from its own branch), then warp 2 releases the TMEM columns.
 __device__ __forceinline__ void teardown(int warp, uint32_t tmem) {
@@ -492,7 +397,6 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
 
   if (threadIdx.x == 0) {
     mbar_init(&sh->q_full, 1);
-    mbar_init(&sh->q_ready, 128);
     mbar_init(&sh->q_empty, 1);
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&sh->k_full[s], 1);
@@ -509,7 +413,6 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
     mbar_init(&sh->o_full, 1);
     mbar_init(&sh->o_empty, 256);
     mbar_init(&sh->drain, 1);
-    mbar_init(&sh->tab_bar, 128);
     mbar_init(&sh->part_bar, 256);
     mbar_init(&sh->last_bar, 1);
     sh->abort = 0;
@@ -537,7 +440,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
   const int n_pieces = meta->n_pieces;
 
   // Register split (launch: 512 threads x 128): the producer/MMA warpgroup and
-  // the RoPE warpgroup give registers to the two softmax warpgroups, which
+  // the idle warpgroup 1 give registers to the two softmax warpgroups, which
   // keep a whole 128-column S row in registers.  88 + 72 + 176 + 176 = 4 x 128.
   // Each warpgroup changes its count exactly once, at the top of its branch,
   // and never takes registers back: a later increase could claim registers a
@@ -682,7 +585,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
       for (int k = 0; k < n_pieces && ok; ++k) {
         int n = 0;
         bool two = true;
-        ok = wait_bar<true>(&sh->q_ready, k & 1, sh, p.err, kSiteMma) &&
+        ok = wait_bar<true>(&sh->q_full, k & 1, sh, p.err, kSiteMma) &&
              read_piece_len(meta, k, n, two, p, sh, p.err, kSiteMma) && wait_k(g);
         if (!ok) break;
         tc_fence_after();
@@ -748,46 +651,9 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
     teardown(warp, tmem);
     return;
   } else if (warp < 8) {
+    // warpgroup 1 has no role: the queries arrive rotated (a pass before
+    // this kernel rotates the block's queries and keys)
     regs_dec<72>();
-    // ------------------------------------------------------------ RoPE
-    const int tid = threadIdx.x - 128;
-    const RopeLane rl = rope_lane<D>(p, tid);
-    // this rollout's t table and the static h / w tables, in shared memory
-    float2* st = reinterpret_cast<float2*>(smem + G::kOffTab);
-    const int n_t = (p.slots + p.F) * p.pt, n_h = p.gh * p.ph, n_w = p.gw * p.pw;
-    int staged = -1;
-    uint32_t n_stage = 0;
-    bool ok = true;
-    for (int k = 0; k < n_pieces && ok; ++k) {
-      PieceInfo pi;
-      ok = __all_sync(0xffffffffu, wait_bar(&sh->q_full, k & 1, sh, p.err, kSiteRope) &&
-                                       read_piece(meta, k, pi, sh, p.err, kSiteRope));
-      if (!ok) break;
-      if (pi.r != staged) {
-        // every RoPE thread has finished the previous Q tiles (arrived on
-        // q_ready) before the tables are overwritten
-        if (k > 0) {
-          ok = __all_sync(0xffffffffu,
-                          wait_bar(&sh->q_ready, (k - 1) & 1, sh, p.err, kSiteRope));
-          if (!ok) break;
-        }
-        const float2* tt = p.ttab + (size_t)pi.r * n_t;
-        for (int i = tid; i < n_t; i += 128) st[i] = tt[i];
-        for (int i = tid; i < n_h; i += 128) st[n_t + i] = p.htab[i];
-        for (int i = tid; i < n_w; i += 128) st[n_t + n_h + i] = p.wtab[i];
-        mbar_arrive(&sh->tab_bar);
-        ok = __all_sync(0xffffffffu,
-                        wait_bar(&sh->tab_bar, n_stage & 1, sh, p.err, kSiteRope));
-        ++n_stage;
-        if (!ok) break;
-        staged = pi.r;
-      }
-      const int qrow0 = pi.b * 2 * kBM;
-      rope_q_tile<D>(smem + kOffQ, qrow0, rl, st, p);
-      rope_q_tile<D>(smem + kOffQ + kTile, qrow0 + kBM, rl, st, p);
-      fence_proxy_async_smem();
-      mbar_arrive(&sh->q_ready);
-    }
     teardown(warp, tmem);
     return;
   } else {
@@ -888,15 +754,6 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
           for (int i = 0; i < 32; ++i) {
             const uint64_t x2 = f2_fma(
                 f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
-            if constexpr (kExpPairs) {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              const uint32_t pb = ex2_bf16x2(pack_bf16(x0, x1));
-              pk[i] = pb;
-              ls2 = f2_add(ls2, f2_pack(__uint_as_float(pb << 16),
-                                        __uint_as_float(pb & 0xFFFF0000u)));
-              continue;
-            }
             uint64_t e2;
             constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
             if (kPolyEvery > 0 && full && (i % kEvery) == kEvery - 1) {
@@ -1109,10 +966,7 @@ cudaError_t prepare_kernel(AttnKernel k) {
 
 size_t attn_bf16_smem_bytes(const AttnParams& p) {
   if (p.d != 64 && p.d != 128) return 0;
-  const size_t tab = sizeof(float2) * ((size_t)(p.slots + p.F) * p.pt +
-                                        (size_t)p.gh * p.ph + (size_t)p.gw * p.pw);
-  const size_t fixed = p.d == 128 ? Geo<128>::kSmemFixed : Geo<64>::kSmemFixed;
-  const size_t smem = fixed + tab;
+  const size_t smem = p.d == 128 ? Geo<128>::kSmemFixed : Geo<64>::kSmemFixed;
   return smem > kSmemMax ? 0 : smem;
 }
 

@@ -1,7 +1,7 @@
 // fd_block_attention_static: the attention call with its per-call work area
-// (the block's keys rotated once for all query tiles) in a static device
-// array of this library instead of the layer's work area in the caller's
-// cache storage.  For callers that cannot set device memory aside for that
+// (the block's keys and queries rotated once per call, which the tensor-core
+// kernels read) in a static device array of this library instead of the
+// call's work set in the caller's cache storage.  For callers that cannot set device memory aside for that
 // area -- their storage comes from a pool or arena sized by someone else, or
 // they may not call cudaMalloc at all (it can synchronise the device, which a
 // real-time serving loop cannot afford).  The method on the pages has no

@@ -273,21 +273,34 @@ __global__ void reset_meta_kernel(CacheView c, ResetParams p) {
   fill_ttab(c, l, r, 0, pos);
 }
 
-// 3D RoPE of a block tensor [R][F][Tx][heads][d]: token row i of rollout r and
-// frame f sits at t = n_r + f (t-row slots + f of the rollout's table).  One
-// warp per token row; out may equal in (in place).
+// 3D RoPE of up to two block tensors [R][F][Tx][heads][d] (e.g. the block's
+// queries and keys of one call, in one launch): token row i of rollout r and
+// frame f sits at t = n_r + f (t-row slots + f of the rollout's table).  The
+// rows of tensor 0 come first, then those of tensor 1; one warp per token
+// row; out may equal in (in place).
+template <typename Elem>
+struct RopeJob {
+  const Elem* in;
+  Elem* out;
+  int Tx, heads;
+  uint32_t rows;  // n_rollouts * F * Tx
+};
+
 template <typename Elem>
 __global__ void __launch_bounds__(256)
-    rope3d_kernel(CacheView c, int layer, int n_rollouts, const Elem* in,
-                  Elem* out, int Tx, int heads) {
+    rope3d_kernel(CacheView c, int layer, RopeJob<Elem> j0, RopeJob<Elem> j1) {
   constexpr int kPer = 16 / sizeof(Elem);  // elements per 16-byte chunk
   const uint32_t cpr = c.d / kPer;         // chunks per head row
-  const uint32_t row_chunks = cpr * heads;  // chunks per token row
-  const uint32_t rows = (uint32_t)n_rollouts * c.F * Tx;
+  const uint32_t rows_all = j0.rows + j1.rows;
   const uint32_t warps = gridDim.x * (blockDim.x >> 5);
   const int lane = threadIdx.x & 31;
-  for (uint32_t row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       row < rows; row += warps) {
+  for (uint32_t row_all = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       row_all < rows_all; row_all += warps) {
+    const bool second = row_all >= j0.rows;
+    const RopeJob<Elem>& jb = second ? j1 : j0;
+    const uint32_t row = second ? row_all - j0.rows : row_all;
+    const int Tx = jb.Tx;
+    const uint32_t row_chunks = cpr * jb.heads;  // chunks per token row
     const uint32_t r = row / (c.F * Tx);
     const uint32_t rem = row - r * (c.F * Tx);
     const int f = (int)(rem / Tx);
@@ -297,8 +310,8 @@ __global__ void __launch_bounds__(256)
     const int tv = tok % c.Tv;  // position inside the token's view
     const int hh = tok < c.T ? tv / c.gw : 0;
     const int ww = tok < c.T ? tv - hh * c.gw : 0;
-    const uint4* src = reinterpret_cast<const uint4*>(in) + (size_t)row * row_chunks;
-    uint4* dst = reinterpret_cast<uint4*>(out) + (size_t)row * row_chunks;
+    const uint4* src = reinterpret_cast<const uint4*>(jb.in) + (size_t)row * row_chunks;
+    uint4* dst = reinterpret_cast<uint4*>(jb.out) + (size_t)row * row_chunks;
     if (32 % cpr == 0) {
       // every chunk a lane touches holds the same pairs (lane % cpr of each
       // head row): their cos/sin are looked up once per token row, and up to
@@ -326,14 +339,17 @@ __global__ void __launch_bounds__(256)
 
 template <typename Elem>
 cudaError_t launch_rope_rows(const CacheView& c, int layer, int n_rollouts,
-                             const void* in, void* out, int Tx, int heads,
+                             const void* in0, void* out0, int Tx0, int heads0,
+                             const void* in1, void* out1, int Tx1, int heads1,
                              cudaStream_t s) {
-  const uint64_t rows = (uint64_t)n_rollouts * c.F * Tx;
+  RopeJob<Elem> j0{static_cast<const Elem*>(in0), static_cast<Elem*>(out0), Tx0, heads0,
+                   (uint32_t)((uint64_t)n_rollouts * c.F * Tx0)};
+  RopeJob<Elem> j1{static_cast<const Elem*>(in1), static_cast<Elem*>(out1), Tx1, heads1,
+                   in1 != nullptr ? (uint32_t)((uint64_t)n_rollouts * c.F * Tx1) : 0u};
+  const uint64_t rows = (uint64_t)j0.rows + j1.rows;
   const uint64_t blocks_needed = (rows + 7) / 8;  // 8 warps per block
   const unsigned blocks = (unsigned)(blocks_needed < 148ull * 8 ? blocks_needed : 148ull * 8);
-  rope3d_kernel<Elem><<<blocks, 256, 0, s>>>(c, layer, n_rollouts,
-                                             static_cast<const Elem*>(in),
-                                             static_cast<Elem*>(out), Tx, heads);
+  rope3d_kernel<Elem><<<blocks, 256, 0, s>>>(c, layer, j0, j1);
   count_launch(1);
   return cudaGetLastError();
 }
@@ -383,16 +399,18 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
                           void* x, int Tx, int heads, cudaStream_t s) {
   if (c.esz == 2)
-    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, x, x, Tx, heads, s);
-  return launch_rope_rows<float>(c, layer, n_rollouts, x, x, Tx, heads, s);
+    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, x, x, Tx, heads, nullptr,
+                                      nullptr, 0, 0, s);
+  return launch_rope_rows<float>(c, layer, n_rollouts, x, x, Tx, heads, nullptr, nullptr, 0,
+                                 0, s);
 }
 
-cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
-                                   int n_rollouts, const void* k, void* out,
-                                   cudaStream_t s) {
-  if (c.esz == 2)
-    return launch_rope_rows<uint16_t>(c, layer, n_rollouts, k, out, c.Tf, c.Hkv, s);
-  return launch_rope_rows<float>(c, layer, n_rollouts, k, out, c.Tf, c.Hkv, s);
+cudaError_t launch_rope_block(const CacheView& c, int layer, int n_rollouts,
+                              const void* q, void* q_out, const void* k, void* k_out,
+                              cudaStream_t s) {
+  if (c.esz != 2) return cudaErrorInvalidValue;  // the tensor-core path is bf16
+  return launch_rope_rows<uint16_t>(c, layer, n_rollouts, q, q_out, c.T, c.H, k, k_out,
+                                    c.Tf, c.Hkv, s);
 }
 
 }  // namespace fd

@@ -107,8 +107,16 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   size_t blk;
   if (!mul_ok(frame * d->block_frames, ws_r, &blk) || blk > kRegionMax) return FD_ERR_CAPACITY;
   off = align_up(off + blk);
-  // partial results and arrival counters of the persistent bf16 kernel
+  // the block's rotated queries, the partial results and arrival counters of
+  // the persistent bf16 kernel
   const bool tensor_path = d->dtype == FD_BF16;
+  lay->qblk = off;
+  if (tensor_path) {
+    if (!mul_ok(T * d->block_frames * d->num_heads, (size_t)d->head_dim * esz * ws_r, &x) ||
+        x > kRegionMax)
+      return FD_ERR_CAPACITY;
+    off = align_up(off + x);
+  }
   const size_t pairs = (T * d->block_frames + 255) / 256;
   lay->part = off;
   if (tensor_path)
@@ -249,6 +257,7 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.v = base + lay.v;
   v.krot = base + lay.krot;
   v.kblk = base + lay.kblk;
+  v.qblk = base + lay.qblk;
   v.part = reinterpret_cast<float*>(base + lay.part);
   v.cnt = reinterpret_cast<int32_t*>(base + lay.cnt);
   v.pos = reinterpret_cast<int32_t*>(base + lay.pos);
@@ -401,8 +410,21 @@ fd_status fd_block_attention(fd_cache* cache, int32_t layer,
 
 }  // extern "C"
 
+// Work-area bytes of a call: the block's rotated keys, then its rotated
+// queries (tensor-core calls; the CUDA-core kernel rotates as it stages).
+bool fd::tensor_core_call(const fd_cache* cache) {
+  return cache->desc.dtype == FD_BF16 && (cache->view.d == 128 || cache->view.d == 64);
+}
+
+static size_t block_key_bytes(const fd::CacheView& c, int32_t n_rollouts) {
+  return (size_t)n_rollouts * c.F * c.frame_bytes;
+}
+
 size_t fd::block_work_bytes(const fd_cache* cache, int32_t n_rollouts) {
-  return (size_t)n_rollouts * cache->view.F * cache->view.frame_bytes;
+  const fd::CacheView& c = cache->view;
+  if (!tensor_core_call(cache)) return 0;
+  return block_key_bytes(c, n_rollouts) +
+         (size_t)n_rollouts * c.F * c.T * c.H * c.d * c.esz;
 }
 
 fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
@@ -423,15 +445,22 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
 
   fd::AttnParams p;
   memset(&p, 0, sizeof(p));
-  p.q = q;
-  // the call's work set: the block's keys, rotated once for all query tiles
-  // (see fd.h, kblk), the split-pair partials and their counters; the keys
-  // go to the caller's `work` instead when one is given
+  // bf16 with d = 128 or 64 runs on the tensor cores; fp32, and bf16 of the
+  // other head sizes, on CUDA cores
+  const bool tensor_cores = fd::tensor_core_call(cache);
+  // the call's work set: the block's keys and queries, rotated once for all
+  // query tiles (see fd.h, kblk and qblk), the split-pair partials and their
+  // counters; the rotated keys and queries go to the caller's `work` instead
+  // when one is given
   const int ws = layer % c.work_sets;
-  void* kblk = work != nullptr
-      ? work
-      : static_cast<void*>(c.kblk + (size_t)ws * c.R * c.F * c.frame_bytes);
-  p.k = kblk;
+  uint8_t* kblk = work != nullptr ? static_cast<uint8_t*>(work)
+                                  : c.kblk + (size_t)ws * c.R * c.F * c.frame_bytes;
+  uint8_t* qblk = work != nullptr
+      ? static_cast<uint8_t*>(work) + block_key_bytes(c, n_rollouts)
+      : c.qblk + (size_t)ws * c.R * c.F * c.T * c.H * c.d * c.esz;
+  // the CUDA-core kernel reads the block as given and rotates as it stages
+  p.q = tensor_cores ? static_cast<const void*>(qblk) : q;
+  p.k = tensor_cores ? static_cast<const void*>(kblk) : k;
   p.v = v_;
   p.pos = c.pos + (size_t)layer * c.R * c.slots;
   p.count = c.count + (size_t)layer * c.R;
@@ -476,30 +505,20 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  // bf16 with d = 128 or 64 runs on the tensor cores; fp32, and bf16 of the
-  // other head sizes, on CUDA cores
-  const bool tensor_cores = cache->desc.dtype == FD_BF16 && (c.d == 128 || c.d == 64);
   if (tensor_cores ? !cache->have_maps : (c.d % 32 != 0 || c.d > 128))
     return FD_ERR_UNSUPPORTED;
-  // The tensor-core kernel splits a query index q < Mq into (frame, token,
-  // h, w) with multiply-shift divisions (FastDiv), exact while n * divisor <
-  // 2^40: q / T, a token < T over Tv, a token < Tv over gw.
-  if (tensor_cores && ((uint64_t)p.Mq * c.T >= (1ull << 40) ||
-                       (uint64_t)c.T * c.Tv >= (1ull << 40) ||
-                       (uint64_t)c.Tv * c.gw >= (1ull << 40)))
-    return FD_ERR_UNSUPPORTED;
-  // and stages the call's RoPE tables in shared memory next to its tiles
   if (tensor_cores && fd::attn_bf16_smem_bytes(p) == 0) return FD_ERR_UNSUPPORTED;
   // a shard's result is only usable with its log-sum-exp (to be combined)
   if (c.N > 1 && lse == nullptr) return FD_ERR_INVALID_ARG;
-  // the RoPE pass walks the block's key rows with a 32-bit row counter
-  if (!fd::rope_rows_ok(n_rollouts, c.F, c.Tf)) return FD_ERR_UNSUPPORTED;
+  // the RoPE pass walks the block's query and key rows with a 32-bit row
+  // counter
+  if (!fd::rope_rows_ok(n_rollouts, c.F, c.T + c.Tf)) return FD_ERR_UNSUPPORTED;
   // Everything the tensor-core launch needs is prepared before the first
   // launch of the call, so a refusal leaves nothing half done.
   CUtensorMap tm_q, tm_vb, tm_kb_work;
   if (tensor_cores) {
     const uint64_t kb_rows = (uint64_t)c.F * c.Tf;
-    if (!fd::encode_bf16_map(&tm_q, q, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
+    if (!fd::encode_bf16_map(&tm_q, qblk, c.d, c.H, (uint64_t)p.Mq, n_rollouts) ||
         !fd::encode_bf16_map(&tm_vb, v_, c.d, c.Hkv, kb_rows, n_rollouts))
       return FD_ERR_CUDA;
     if (work != nullptr &&
@@ -516,16 +535,12 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
     if (it_max * g >= ((int64_t)1 << 31)) return FD_ERR_UNSUPPORTED;
     p.G = (int)g;
   }
-  // the CUDA-core kernel rotates the block's keys as it stages them
-  if (!tensor_cores) {
-    p.k = k;
-    return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
-  }
-  // the block's keys belong to shard 0; other shards never read them
-  if (c.shard == 0) {
-    st = fd::cuda_status(fd::launch_rope_block_keys(c, layer, n_rollouts, k, kblk, s));
-    if (st != FD_OK) return st;
-  }
+  if (!tensor_cores) return fd::cuda_status(fd::launch_attn_cuda_core(p, c.esz, s));
+  // one pass rotates the block's queries and (the block's keys belong to
+  // shard 0; other shards never read them) its keys
+  st = fd::cuda_status(fd::launch_rope_block(c, layer, n_rollouts, q, qblk,
+                                             c.shard == 0 ? k : nullptr, kblk, s));
+  if (st != FD_OK) return st;
   if (c.shard != 0) {
     // rollouts with no key on this shard get zero rows and lse = -inf here;
     // the tensor-core kernel skips them

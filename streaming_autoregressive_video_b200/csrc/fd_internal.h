@@ -92,6 +92,7 @@ struct CacheView {
   uint8_t* v;
   uint8_t* krot;  // committed keys rotated to their frame's position
   uint8_t* kblk;  // work areas: the block's keys rotated per call
+  uint8_t* qblk;  // work areas: the block's queries rotated per call (bf16)
   int32_t* pos;
   int32_t* count;
   float2* ttab;
@@ -140,9 +141,8 @@ struct ResetParams {
 
 // Parameters of the attention kernels (the tensor maps travel separately).
 struct AttnParams {
-  const void* q;         // block tensors, as given (pre-RoPE)
-  const void* k;         // block keys: rotated (work area) for the tensor-core
-                         // kernel, as given for the CUDA-core kernel
+  const void* q;         // block queries and keys: rotated (work area) for the
+  const void* k;         // tensor-core kernel, as given for the CUDA-core kernel
   const void* v;
   const int32_t* pos;    // [R][slots] of the layer
   const int32_t* count;  // [R] of the layer
@@ -180,11 +180,12 @@ cudaError_t launch_reset(const CacheView& c, const ResetParams& p,
 cudaError_t launch_rope3d(const CacheView& c, int layer, int n_rollouts,
                           void* x, int tokens_per_frame, int heads,
                           cudaStream_t s);
-// block keys k [n_rollouts][F*Tf][Hkv][d] rotated (positions from `layer`'s
-// counters) into out, same layout
-cudaError_t launch_rope_block_keys(const CacheView& c, int layer,
-                                   int n_rollouts, const void* k, void* out,
-                                   cudaStream_t s);
+// the block's queries q [n_rollouts][F*T][H][d] into q_out and (k not null)
+// keys k [n_rollouts][F*Tf][Hkv][d] into k_out, rotated (positions from
+// `layer`'s counters), same layouts, one launch (bf16)
+cudaError_t launch_rope_block(const CacheView& c, int layer, int n_rollouts,
+                              const void* q, void* q_out, const void* k, void* k_out,
+                              cudaStream_t s);
 // attention on CUDA cores in fp32 arithmetic: fp32 caches of any head size
 // d in {32, 64, 96, 128}; bf16 caches (esz = 2) whose d is 32 or 96
 cudaError_t launch_attn_cuda_core(const AttnParams& p, int esz, cudaStream_t s);
@@ -216,13 +217,16 @@ cudaError_t launch_bounded_wait_selftest(int32_t* err, uint64_t limit_ns,
                                          cudaStream_t s);
 
 // Shared body of the attention entry points.  `work` is a device area for the
-// block's rotated keys ([n_rollouts][F*Tf][Hkv][d], block_work_bytes bytes,
-// 16-byte aligned) or nullptr for the layer's work area in the cache storage.
+// block's rotated keys ([n_rollouts][F*Tf][Hkv][d]) followed by its rotated
+// queries ([n_rollouts][F*T][H][d]; block_work_bytes bytes in all,
+// 16-byte aligned) or nullptr for the call's work set in the cache storage.
 fd_status block_attention_impl(fd_cache* cache, int32_t layer,
                                int32_t n_rollouts, const void* q,
                                const void* k, const void* v, void* out,
                                float* lse, void* stream, void* work);
 size_t block_work_bytes(const fd_cache* cache, int32_t n_rollouts);
+// whether attention calls on this cache run on the tensor-core kernels
+bool tensor_core_call(const fd_cache* cache);
 
 }  // namespace fd
 

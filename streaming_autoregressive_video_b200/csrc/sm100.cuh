@@ -289,14 +289,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// Hardware base-2 exponential of a bf16 pair (MUFU, flush-to-zero): both
-// halves of the 32-bit word in one instruction, results as a bf16 pair.
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes).
 // max of three floats in one instruction (three-input max.f32, sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

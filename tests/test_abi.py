@@ -36,7 +36,8 @@ def test_cache_bytes_and_layout():
         esz = 2 if w.dtype == "bf16" else 4
         kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.hkv * w.head_dim * esz
         assert lay.layer_kv_bytes * w.layers == kv
-        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.part, lay.cnt, lay.pos, lay.count,
+        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.qblk, lay.part, lay.cnt, lay.pos,
+                   lay.count,
                    lay.ttab, lay.htab, lay.wtab, lay.err]
         assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
         assert lay.v - lay.k >= kv and lay.krot - lay.v >= kv and lay.kblk - lay.krot >= kv
@@ -45,7 +46,10 @@ def test_cache_bytes_and_layout():
         # and their counters, for one call at a time; none of the latter two
         # for fp32 caches
         blk = w.rollouts * w.block_frames * w.frame_tokens * w.hkv * w.head_dim * esz
-        assert blk <= lay.part - lay.kblk < blk + 1024
+        assert blk <= lay.qblk - lay.kblk < blk + 1024
+        # the block's rotated queries (bf16 caches: the tensor-core calls)
+        qb = w.rollouts * w.queries * w.heads * w.head_dim * esz if w.dtype == "bf16" else 0
+        assert qb <= lay.part - lay.qblk < qb + 1024
         part = 148 * 2 * (256 * 128 + 512) * 4 if w.dtype == "bf16" else 0
         assert part <= lay.cnt - lay.part < part + 1024
         pairs = -(-w.block_frames * w.tokens // 256)
@@ -53,10 +57,11 @@ def test_cache_bytes_and_layout():
         assert cnt <= lay.pos - lay.cnt < cnt + 1024
         # one work set per layer multiplies the three by L and nothing else
         lay_l = fd.fd_cache_get_layout(fd.make_desc(w, work_sets=w.layers))
-        assert lay_l.part - lay_l.kblk >= w.layers * blk
+        assert lay_l.qblk - lay_l.kblk >= w.layers * blk
+        assert lay_l.part - lay_l.qblk >= w.layers * qb
         assert lay_l.cnt - lay_l.part >= w.layers * part
         assert lay_l.pos - lay_l.cnt >= w.layers * cnt
-        assert (lay_l.total - lay.total) - (w.layers - 1) * (blk + part + cnt) < 3 * 1024
+        assert (lay_l.total - lay.total) - (w.layers - 1) * (blk + qb + part + cnt) < 4 * 1024
         assert (lay.rope_pairs_t, lay.rope_pairs_h, lay.rope_pairs_w) == \
             (w.head_dim // 2 - 2 * (w.head_dim // 6), w.head_dim // 6, w.head_dim // 6)
 
@@ -64,10 +69,10 @@ def test_cache_bytes_and_layout():
 def test_single_480p_cache_is_about_3_gb():
     n = fd.fd_cache_bytes(fd.make_desc(SINGLE_480P))
     # 30 layers x 7 slots x 1560 tokens x 12 heads x 128 x 2 B x (K, V, rotated K)
-    # + one work area for the block's rotated keys (3 frames)
+    # + one work area for the block's rotated keys and queries (3 frames each)
     # + one set of partial-result slots of the attention kernel
     part = 148 * 2 * (256 * 128 + 512) * 4
-    assert abs(n - (30 * 7 * 3 + 3) * 1560 * 12 * 128 * 2 - part) < 1 << 20
+    assert abs(n - (30 * 7 * 3 + 3 + 3) * 1560 * 12 * 128 * 2 - part) < 1 << 20
     assert n <= 3.1e9
     # K and V as the method keeps them: 2.01 GB
     assert 30 * 7 * 2 * 1560 * 12 * 128 * 2 == 2012774400

@@ -7,8 +7,9 @@ array of the library, so it allocates nothing.
 Checked here: two calls in a row through the C ABI give exactly the results of
 the regular entry point (the same kernels on the same inputs; only the work
 area's address differs, so outputs and log-sum-exps must be bit-identical), on
-the tensor-core path (multi-head and grouped-query) and on the CUDA-core path
-(fp32); and a request larger than the static area is refused before any
+the tensor-core path (multi-head and grouped-query; the area holds the
+block's rotated keys and queries) and on the CUDA-core path (fp32, which needs
+no area); and a request larger than the static area is refused before any
 launch.  This file is collected last; it passes alone in a fresh process (the
 first call looks up the array's device address) and after the other tests."""
 import pytest
@@ -28,7 +29,7 @@ CASES = {
     "bf16-mha": BF16,
     # grouped-query: the rotated-block-key map of the static area has Hkv rows
     "bf16-gqa": BF16.scaled(name="static-work-bf16-gqa", kv_heads=2),
-    # fp32: the CUDA-core kernel reads the rotated block keys straight from it
+    # fp32: the CUDA-core kernel rotates as it stages and uses no work area
     "f32-tiny": TINY_F32.scaled(layers=2),
 }
 
@@ -64,27 +65,30 @@ def test_static_work_area_matches_regular_entry_point_twice(case):
 
 
 def test_static_work_area_refuses_oversized_calls():
-    # 40 query heads over 20 key/value heads: the rotated block keys take
-    # 3 frames x 1564 tokens x 20 heads x 128 x 2 bytes = 24 MB per rollout,
-    # so two rollouts (48 MB) do not fit in the 32 MiB area
-    big = Workload("static-work-too-big", layers=1, rollouts=2, heads=40, head_dim=128,
+    # a tensor-core call's area holds the block's rotated keys (Hkv heads) and
+    # rotated queries (H heads): 3 frames x (1564 x 4 + 1560 x 8) tokens x
+    # heads x 128 x 2 bytes = 14.4 MB per rollout, so two rollouts fit in the
+    # 32 MiB area and three do not
+    big = Workload("static-work-too-big", layers=1, rollouts=3, heads=8, head_dim=128,
                    grid_h=30, grid_w=52, action_tokens=4, block_frames=3, sink_frames=0,
-                   window_frames=3, steps=1, blocks=1, dtype="bf16", kv_heads=20)
-    need = fd._Geom(fd.make_desc(big)).kv            # bytes of one rollout's block keys
-    assert need == big.block_frames * big.frame_tokens * big.hkv * big.head_dim * 2
-    assert need <= fd.STATIC_WORK_BYTES < big.rollouts * need
+                   window_frames=3, steps=1, blocks=1, dtype="bf16", kv_heads=4)
+    g = fd._Geom(fd.make_desc(big))
+    need = g.kv + g.q                                # bytes of one rollout
+    assert g.kv == big.block_frames * big.frame_tokens * big.hkv * big.head_dim * 2
+    assert g.q == big.queries * big.heads * big.head_dim * 2
+    assert 2 * need <= fd.STATIC_WORK_BYTES < 3 * need
     cache = new_cache(big)
-    q = torch.zeros((2, big.queries, big.heads, big.head_dim), dtype=torch.int16,
+    q = torch.zeros((3, big.queries, big.heads, big.head_dim), dtype=torch.int16,
                     device="cuda")
-    kv = torch.zeros((2, big.block_frames * big.frame_tokens, big.hkv, big.head_dim),
+    kv = torch.zeros((3, big.block_frames * big.frame_tokens, big.hkv, big.head_dim),
                      dtype=torch.int16, device="cuda")
     out = torch.empty_like(q)
-    # one rollout fits and runs
-    fd.fd_block_attention_static(cache, 0, 1, q, kv, kv, out)
+    # two rollouts fit and run
+    fd.fd_block_attention_static(cache, 0, 2, q, kv, kv, out)
     torch.cuda.synchronize()
     launches = fd.fd_launch_count()
     with pytest.raises(fd.FdError) as e:
-        fd.fd_block_attention_static(cache, 0, 2, q, kv, kv, out)
+        fd.fd_block_attention_static(cache, 0, 3, q, kv, kv, out)
     assert e.value.status == 4   # FD_ERR_CAPACITY
     assert fd.fd_launch_count() == launches
     assert fd.fd_get_device_error(cache) == 0
