@@ -140,10 +140,8 @@ typedef struct {
  *   part : [Wk][148][2][256*128 + 512] float work area of the bf16 attention
  *          kernel: a CTA whose share of the work ends or begins inside a
  *          query tile pair leaves its partial result there (unnormalised
- *          output rows, running max, row sum); empty (size 0) for fp32
- *   cnt  : [Wk][R][H][ceil(F*T/256)] int32 arrival counters of those split
- *          tile pairs; zero between calls (the last arriving CTA combines
- *          the partial results and clears its counter)
+ *          output rows, running max, row sum), which a fold kernel launched
+ *          right after combines; empty (size 0) for fp32
  *   pos  : [L][R][S+W] int32, frame index held by a slot, -1 = empty
  *   count: [L][R] int32, frames committed since the last reset (n)
  *   ttab : [L][R][S+W+F][p_t] float2 (cos, sin) of the t-section angles for
@@ -151,7 +149,7 @@ typedef struct {
  *   htab : [grid_h][p_h] float2, wtab : [grid_w][p_w] float2 (static)
  *   err  : int32 device error word (0 = none)                            */
 typedef struct {
-  size_t k, v, krot, kblk, qblk, part, cnt, pos, count, ttab, htab, wtab, err;
+  size_t k, v, krot, kblk, qblk, part, pos, count, ttab, htab, wtab, err;
   size_t total;           /* == fd_cache_bytes(desc)                       */
   size_t layer_kv_bytes;  /* bytes of one layer's K (or V) region          */
   int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
@@ -241,8 +239,9 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * CTA per multiprocessor, at most 148) and splits the call's KV iterations
  * evenly over its CTAs; it returns FD_ERR_UNSUPPORTED when n_rollouts x H x
  * ceil(F*T/256) x (ceil((S+W)*Tf/128) + ceil(F*Tf/128)) x CTAs reaches 2^31.
- * A query-tile pair split between CTAs is combined through the work set's
- * `part` / `cnt` regions.
+ * A query-tile pair split between CTAs leaves its pieces in the work set's
+ * `part` region; a fold kernel launched right after the attention kernel
+ * combines them (a fixed order: results do not depend on timing).
  * Device-side waits are bounded: a wait that gives up sets the error word
  * (fd_get_device_error) instead of hanging. */
 fd_status fd_block_attention(fd_cache* cache, int32_t layer,

@@ -54,7 +54,7 @@ class CacheLayout(ctypes.Structure):
     _fields_ = [("k", ctypes.c_size_t), ("v", ctypes.c_size_t), ("krot", ctypes.c_size_t),
                 ("kblk", ctypes.c_size_t), ("qblk", ctypes.c_size_t),
                 ("part", ctypes.c_size_t),
-                ("cnt", ctypes.c_size_t), ("pos", ctypes.c_size_t),
+                ("pos", ctypes.c_size_t),
                 ("count", ctypes.c_size_t), ("ttab", ctypes.c_size_t),
                 ("htab", ctypes.c_size_t), ("wtab", ctypes.c_size_t),
                 ("err", ctypes.c_size_t), ("total", ctypes.c_size_t),

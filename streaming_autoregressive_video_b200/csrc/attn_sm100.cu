@@ -19,11 +19,10 @@
 // equal ranges, one per CTA and G = one CTA per multiprocessor, so every CTA
 // does the same number of KV tiles (+-1) whatever the number of units: no
 // partly idle last wave.  A unit cut by a range boundary is computed in
-// pieces; every piece but the last to finish leaves its unnormalised rows,
-// row maxima and row sums (fp32) in the layer's partial-result area and
-// counts itself in the unit's arrival counter; the piece that arrives last
-// folds the others into its own rows, writes them and clears the counter.
-// No CTA ever waits for another.
+// pieces; every piece leaves its unnormalised rows, row maxima and row sums
+// (fp32) in the work set's partial-result area, and a fold kernel launched
+// right after this one combines the pieces of each split unit in a fixed
+// order and writes its rows.  No CTA ever waits for another.
 //
 // Roles (all warps walk the same sequence of pieces):
 //   warp 0        TMA producer: each piece's two Q tiles (once the previous
@@ -91,11 +90,8 @@ struct Shared {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_empty, drain;
-  uint64_t part_bar;  // softmax: a piece's partial rows written
-  uint64_t last_bar;  // softmax: the piece's arrival counted
   uint32_t tmem_base;
   int32_t abort;
-  int32_t last;       // this piece arrived last: it writes the unit's rows
 };
 
 static_assert(sizeof(Shared) <= 256, "barrier block");
@@ -413,10 +409,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
     mbar_init(&sh->o_full, 1);
     mbar_init(&sh->o_empty, 256);
     mbar_init(&sh->drain, 1);
-    mbar_init(&sh->part_bar, 256);
-    mbar_init(&sh->last_bar, 1);
     sh->abort = 0;
-    sh->last = 0;
     fence_mbarrier_init();
     // the CTA's schedule: how many pieces, where its split range starts
     const Sched sd = make_sched(p);
@@ -672,7 +665,6 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
     const uint32_t tO = tmem + lane_off + kColO0 + x * D;
     const float sl2 = p.scale_log2;
     int g = 0;  // KV iterations this warpgroup's tile has run (its barriers' phases)
-    uint32_t n_part = 0;
     bool ok = true;
     uint32_t sa[64], sb[64];
     for (int k = 0; k < n_pieces && ok; ++k) {
@@ -794,15 +786,12 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
       PieceInfo pi;
       ok = __all_sync(0xffffffffu, read_piece(meta, k, pi, sh, p.err, kSiteSoftmax));
       if (!ok) break;
-      const Sched sd = meta->sd;
       const int row = x * kBM + row_t;  // row within the pair
       const bool whole = pi.kv0 == 0 && pi.kv1 == pi.nt;
-      bool write_rows = whole;
-      // CTAs whose pieces make up the unit, folded in this fixed order (so
-      // the rounding does not depend on which piece arrived last)
-      int c_lo = blockIdx.x, c_hi = blockIdx.x;
+      const int qrow = pi.b * 2 * kBM + row;
       if (!whole) {
-        // hand this piece over: unnormalised row, running max, row sum
+        // a piece of a unit split between CTAs: hand it over (unnormalised
+        // row, running max, row sum) to the fold that runs after this kernel
         float* part = p.part + ((size_t)blockIdx.x * 2 +
                                 (pi.U0 + pi.kv0 == meta->my_begin ? 0 : 1)) * kPartSlotFloats;
         uint32_t rr[32];
@@ -817,95 +806,21 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
         }
         part[2 * kBM * D + row] = m;
         part[2 * kBM * D + 2 * kBM + row] = l;
-        __threadfence();
-        mbar_arrive(&sh->part_bar);
-        if (threadIdx.x == 256) {
-          // all 256 threads' rows are out: count this piece's arrival
-          bool got = wait_bar<true>(&sh->part_bar, n_part & 1, sh, p.err, kSiteSoftmax);
-          int last = 0;
-          if (got) {
-            __threadfence();
-            const int lo = cta_of(pi.U0, sd, p.G), hi = cta_of(pi.U0 + pi.nt - 1, sd, p.G);
-            int pieces = 0;
-            for (int c = lo; c <= hi; ++c)
-              pieces += cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G) ? 1 : 0;
-            const int before = atomicAdd(&p.cnt[pi.unit], 1);
-            last = before == pieces - 1;
-            if (last) {
-              atomicExch(&p.cnt[pi.unit], 0);  // ready for the next call
-              __threadfence();
-            }
-          }
-          *reinterpret_cast<volatile int32_t*>(&sh->last) = last;
-          mbar_arrive(&sh->last_bar);
-        }
-        ok = __all_sync(0xffffffffu,
-                        wait_bar<true>(&sh->last_bar, n_part & 1, sh, p.err, kSiteSoftmax));
-        ++n_part;
-        if (!ok) break;
-        write_rows = *reinterpret_cast<volatile int32_t*>(&sh->last) != 0;
-        if (write_rows) {
-          __threadfence();
-          c_lo = cta_of(pi.U0, sd, p.G);
-          c_hi = cta_of(pi.U0 + pi.nt - 1, sd, p.G);
-        }
-      }
-      if (write_rows) {
-        // row = sum over pieces i of O_i 2^(m_i - M) / sum of l_i 2^(m_i - M),
-        // M the largest max; this CTA's own piece comes from TMEM
-        constexpr size_t kOffM = 2 * kBM * D, kOffL = kOffM + 2 * kBM;
-        const int qrow = pi.b * 2 * kBM + row;
-        auto skip = [&](int c) {
-          return c != (int)blockIdx.x && cta_begin(c, sd, p.G) == cta_begin(c + 1, sd, p.G);
-        };
-        auto max_of = [&](int c) {
-          return c == (int)blockIdx.x ? m : __ldcg(part_slot(p, c, pi.U0, sd) + kOffM + row);
-        };
-        float M = -INFINITY;
-        for (int c = c_lo; c <= c_hi; ++c)
-          if (!skip(c)) M = fmaxf(M, max_of(c));
-        auto weight = [&](float mc) { return mc == M ? 1.f : ex2_approx(mc - M); };
-        float L = 0.f;
-        for (int c = c_lo; c <= c_hi; ++c) {
-          if (skip(c)) continue;
-          const float lc = c == (int)blockIdx.x ? l
-                                                : __ldcg(part_slot(p, c, pi.U0, sd) + kOffL + row);
-          L += lc * weight(max_of(c));
-        }
-        const float inv_l = 1.f / L;
+      } else {
+        // a whole unit: O / l in bf16 (and the log-sum-exp)
+        const float inv_l = 1.f / l;
         uint16_t* out = static_cast<uint16_t*>(p.out) +
                         (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * D;
         uint32_t rr[32];
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, rr);
-          float acc[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-          for (int c2 = c_lo; c2 <= c_hi; ++c2) {
-            if (skip(c2)) continue;
-            const float w = weight(max_of(c2));
-            if (c2 == (int)blockIdx.x) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) acc[i] += w * __uint_as_float(rr[i]);
-            } else {
-              const float4* src = reinterpret_cast<const float4*>(
-                  part_slot(p, c2, pi.U0, sd) + (size_t)row * D + c * 32);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 f = __ldcg(src + i);
-                acc[4 * i] += w * f.x;
-                acc[4 * i + 1] += w * f.y;
-                acc[4 * i + 2] += w * f.z;
-                acc[4 * i + 3] += w * f.w;
-              }
-            }
-          }
           if (qrow < p.Mq) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16(acc[2 * i] * inv_l, acc[2 * i + 1] * inv_l);
+              pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l,
+                                __uint_as_float(rr[2 * i + 1]) * inv_l);
             uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -914,7 +829,7 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
         }
         if (p.lse != nullptr && qrow < p.Mq)
           p.lse[((size_t)pi.r * p.H + pi.h) * p.Mq + qrow] =
-              (M + log2f(L)) * 0.69314718055994530942f;
+              (m + log2f(l)) * 0.69314718055994530942f;
       }
       // O may now be overwritten by the next piece
       tc_fence_before();
@@ -962,6 +877,108 @@ cudaError_t prepare_kernel(AttnKernel k) {
                               (int)kSmemMax);
 }
 
+// Folds the pieces of the query-tile pairs that the persistent kernel split
+// between CTAs: row = sum_i O_i 2^(m_i - M) / sum_i l_i 2^(m_i - M) over the
+// unit's pieces i in CTA order (a fixed order, so the rounding does not depend
+// on which CTA finished first), M the largest max, written in bf16 with the
+// log-sum-exp.  It runs after the attention kernel on the same stream, so
+// every piece's slot is complete; no CTA of the attention kernel waits or
+// folds.  A block takes 32 of a split unit's 256 rows: 8 warps x 4 rows, a
+// warp reads a row of a piece with one load per lane (D / 32 columns a
+// lane), the 4 rows' loads in flight together.
+constexpr int kFoldRows = 32;      // rows per block
+constexpr int kFoldRowsPerWarp = 4;
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    fold_split_units(const __grid_constant__ AttnParams p) {
+  constexpr int kPerLane = D / 32;
+  constexpr size_t kOffM = 2 * kBM * D, kOffL = kOffM + 2 * kBM;
+  __shared__ Sched s_sd;
+  __shared__ int s_unit[6];  // r, h, b, U0, c_lo, c_hi (c_lo == c_hi: nothing to fold)
+  if (threadIdx.x == 0) {
+    const Sched sd = make_sched(p);
+    const int per_r = p.H * p.nb;
+    const int unit = sd.W * p.G + (int)blockIdx.x / (2 * kBM / kFoldRows);
+    const int r = unit / per_r;
+    int U0 = 0;  // the unit's first iteration: the iterations of the units before it
+    for (int rr = 0; rr < r; ++rr) U0 += per_r * tile_counts(p, rr).nt;
+    const int nt = tile_counts(p, r).nt;
+    U0 += (unit - r * per_r) * nt;
+    const int u = unit - r * per_r;
+    s_sd = sd;
+    s_unit[0] = r;
+    s_unit[1] = u / p.nb;
+    s_unit[2] = u - (u / p.nb) * p.nb;
+    s_unit[3] = U0;
+    s_unit[4] = nt > 0 ? cta_of(U0, sd, p.G) : 0;
+    s_unit[5] = nt > 0 ? cta_of(U0 + nt - 1, sd, p.G) : 0;
+  }
+  __syncthreads();
+  const int c_lo = s_unit[4], c_hi = s_unit[5];
+  if (c_lo == c_hi) return;  // whole: the attention kernel wrote its rows
+  const Sched sd = s_sd;
+  const int r = s_unit[0], h = s_unit[1], b = s_unit[2], U0 = s_unit[3];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = ((int)blockIdx.x % (2 * kBM / kFoldRows)) * kFoldRows + warp * kFoldRowsPerWarp;
+  auto piece = [&](int c) { return cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G); };
+  float M[kFoldRowsPerWarp], L[kFoldRowsPerWarp], acc[kFoldRowsPerWarp][kPerLane];
+#pragma unroll
+  for (int i = 0; i < kFoldRowsPerWarp; ++i) {
+    M[i] = -INFINITY;
+    L[i] = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) acc[i][e] = 0.f;
+  }
+  for (int c = c_lo; c <= c_hi; ++c) {
+    if (!piece(c)) continue;
+    const float* sl = part_slot(p, c, U0, sd);
+#pragma unroll
+    for (int i = 0; i < kFoldRowsPerWarp; ++i) M[i] = fmaxf(M[i], __ldcg(sl + kOffM + row0 + i));
+  }
+  for (int c = c_lo; c <= c_hi; ++c) {
+    if (!piece(c)) continue;
+    const float* sl = part_slot(p, c, U0, sd);
+    float mv[kFoldRowsPerWarp], lv[kFoldRowsPerWarp], ov[kFoldRowsPerWarp][kPerLane];
+#pragma unroll
+    for (int i = 0; i < kFoldRowsPerWarp; ++i) {
+      mv[i] = __ldcg(sl + kOffM + row0 + i);
+      lv[i] = __ldcg(sl + kOffL + row0 + i);
+      const float* o = sl + (size_t)(row0 + i) * D + lane * kPerLane;
+      if constexpr (kPerLane == 4) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(o));
+        ov[i][0] = f.x; ov[i][1] = f.y; ov[i][2] = f.z; ov[i][3] = f.w;
+      } else {
+        const float2 f = __ldcg(reinterpret_cast<const float2*>(o));
+        ov[i][0] = f.x; ov[i][1] = f.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kFoldRowsPerWarp; ++i) {
+      const float w = mv[i] == M[i] ? 1.f : ex2_approx(mv[i] - M[i]);
+      L[i] += lv[i] * w;
+#pragma unroll
+      for (int e = 0; e < kPerLane; ++e) acc[i][e] += w * ov[i][e];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kFoldRowsPerWarp; ++i) {
+    const int qrow = b * 2 * kBM + row0 + i;
+    if (qrow >= p.Mq) continue;
+    const float inv_l = 1.f / L[i];
+    uint16_t* out = static_cast<uint16_t*>(p.out) + (((size_t)r * p.Mq + qrow) * p.H + h) * D +
+                    lane * kPerLane;
+    if constexpr (kPerLane == 4) {
+      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(acc[i][0] * inv_l, acc[i][1] * inv_l),
+                                                  pack_bf16(acc[i][2] * inv_l, acc[i][3] * inv_l));
+    } else {
+      *reinterpret_cast<uint32_t*>(out) = pack_bf16(acc[i][0] * inv_l, acc[i][1] * inv_l);
+    }
+    if (p.lse != nullptr && lane == 0)
+      p.lse[((size_t)r * p.H + h) * p.Mq + qrow] = (M[i] + log2f(L[i])) * 0.69314718055994530942f;
+  }
+}
+
 }  // namespace
 
 size_t attn_bf16_smem_bytes(const AttnParams& p) {
@@ -989,6 +1006,18 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
     attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
   else
     attn_bf16_d64_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
+  count_launch(1);
+  cudaError_t e2 = cudaGetLastError();
+  if (e2 != cudaSuccess) return e2;
+  // the units past the whole-unit waves may be split between CTAs: fold them
+  const int64_t units = (int64_t)p.n_rollouts * p.H * p.nb;
+  const int64_t split = units - units / p.G * p.G;
+  if (split == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)(split * (2 * kBM / kFoldRows));
+  if (p.d == 128)
+    fold_split_units<128><<<blocks, 256, 0, s>>>(p);
+  else
+    fold_split_units<64><<<blocks, 256, 0, s>>>(p);
   count_launch(1);
   return cudaGetLastError();
 }

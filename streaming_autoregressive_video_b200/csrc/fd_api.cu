@@ -74,7 +74,7 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
       d->shard_index >= shards)
     return FD_ERR_SHAPE;
   const size_t slots = (gslots + shards - 1) / shards;  // local slots
-  // per-call work areas (rotated block keys, split-pair partials, counters)
+  // per-call work areas (rotated block keys and queries, split-pair partials)
   const int32_t sets = d->num_work_sets == 0 ? 1 : d->num_work_sets;
   if (sets < 1 || sets > d->num_layers) return FD_ERR_SHAPE;
   const size_t ws_r = (size_t)sets * d->max_rollouts;
@@ -107,8 +107,8 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
   size_t blk;
   if (!mul_ok(frame * d->block_frames, ws_r, &blk) || blk > kRegionMax) return FD_ERR_CAPACITY;
   off = align_up(off + blk);
-  // the block's rotated queries, the partial results and arrival counters of
-  // the persistent bf16 kernel
+  // the block's rotated queries and the partial results of the persistent
+  // bf16 kernel
   const bool tensor_path = d->dtype == FD_BF16;
   lay->qblk = off;
   if (tensor_path) {
@@ -117,16 +117,9 @@ fd_status compute_layout(const fd_cache_desc* d, fd_cache_layout* lay) {
       return FD_ERR_CAPACITY;
     off = align_up(off + x);
   }
-  const size_t pairs = (T * d->block_frames + 255) / 256;
   lay->part = off;
   if (tensor_path)
     off = align_up(off + (size_t)sets * kAttnMaxCtas * 2 * kPartSlotFloats * sizeof(float));
-  lay->cnt = off;
-  if (tensor_path) {
-    if (!mul_ok(ws_r * d->num_heads, pairs * sizeof(int32_t), &x) || x > kRegionMax)
-      return FD_ERR_CAPACITY;
-    off = align_up(off + x);
-  }
   lay->pos = off;
   off = align_up(off + lr * slots * sizeof(int32_t));
   lay->count = off;
@@ -259,7 +252,6 @@ fd_status fd_cache_create(const fd_cache_desc* desc, void* dev_storage,
   v.kblk = base + lay.kblk;
   v.qblk = base + lay.qblk;
   v.part = reinterpret_cast<float*>(base + lay.part);
-  v.cnt = reinterpret_cast<int32_t*>(base + lay.cnt);
   v.pos = reinterpret_cast<int32_t*>(base + lay.pos);
   v.count = reinterpret_cast<int32_t*>(base + lay.count);
   v.ttab = reinterpret_cast<float2*>(base + lay.ttab);
@@ -449,9 +441,9 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   // other head sizes, on CUDA cores
   const bool tensor_cores = fd::tensor_core_call(cache);
   // the call's work set: the block's keys and queries, rotated once for all
-  // query tiles (see fd.h, kblk and qblk), the split-pair partials and their
-  // counters; the rotated keys and queries go to the caller's `work` instead
-  // when one is given
+  // query tiles (see fd.h, kblk and qblk), and the split-pair partials; the
+  // rotated keys and queries go to the caller's `work` instead when one is
+  // given
   const int ws = layer % c.work_sets;
   uint8_t* kblk = work != nullptr ? static_cast<uint8_t*>(work)
                                   : c.kblk + (size_t)ws * c.R * c.F * c.frame_bytes;
@@ -475,7 +467,6 @@ fd_status fd::block_attention_impl(fd_cache* cache, int32_t layer,
   p.kc = c.krot + (size_t)layer * cache->layout.layer_kv_bytes;
   p.vc = c.v + (size_t)layer * cache->layout.layer_kv_bytes;
   p.part = c.part + (size_t)ws * fd::kAttnMaxCtas * 2 * fd::kPartSlotFloats;
-  p.cnt = c.cnt + (size_t)ws * c.R * c.H * c.nb;
   p.nb = c.nb;
   p.H = c.H;
   p.Hkv = c.Hkv;
@@ -616,10 +607,6 @@ fd_status fd_get_device_error(fd_cache* cache, int32_t* code) {
   *code = v;
   if (v != 0) {
     if (cudaMemset(cache->view.err, 0, sizeof(int32_t)) != cudaSuccess) return FD_ERR_CUDA;
-    // a kernel that gave up may have left split-unit arrival counters set
-    const size_t cnt_bytes = cache->layout.pos - cache->layout.cnt;
-    if (cnt_bytes > 0 && cudaMemset(cache->view.cnt, 0, cnt_bytes) != cudaSuccess)
-      return FD_ERR_CUDA;
     return FD_ERR_DEVICE_TIMEOUT;
   }
   return FD_OK;

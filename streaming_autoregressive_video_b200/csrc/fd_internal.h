@@ -99,7 +99,6 @@ struct CacheView {
   float2* htab;
   float2* wtab;
   float* part;    // [work_sets][kAttnMaxCtas][2][kPartSlotFloats] (bf16 caches)
-  int32_t* cnt;   // [work_sets][R][H][nb] (bf16 caches)
   int32_t* err;
   int L, R, H, d, gh, gw, T, Tf, F, S, W, slots, pt, ph, pw, esz, nb;
   int Hkv;               // key/value heads (divides H)
@@ -155,7 +154,6 @@ struct AttnParams {
   const uint8_t* kc;     // rotated cache K of the layer, rollout 0 (CUDA cores)
   const uint8_t* vc;
   float* part;           // per-CTA partial results of split units (tensor path)
-  int32_t* cnt;          // per-unit arrival counters of split units
   int H, d, T, Tf, gh, gw, F, S, W, slots, Mq, pt, ph, pw, n_rollouts;
   int nb;                // query-tile pairs per (rollout, head)
   int Hkv;               // key/value heads

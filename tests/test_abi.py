@@ -36,7 +36,7 @@ def test_cache_bytes_and_layout():
         esz = 2 if w.dtype == "bf16" else 4
         kv = w.layers * w.rollouts * w.slots * w.frame_tokens * w.hkv * w.head_dim * esz
         assert lay.layer_kv_bytes * w.layers == kv
-        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.qblk, lay.part, lay.cnt, lay.pos,
+        regions = [lay.k, lay.v, lay.krot, lay.kblk, lay.qblk, lay.part, lay.pos,
                    lay.count,
                    lay.ttab, lay.htab, lay.wtab, lay.err]
         assert regions == sorted(regions) and all(r % 1024 == 0 for r in regions)
@@ -51,17 +51,13 @@ def test_cache_bytes_and_layout():
         qb = w.rollouts * w.queries * w.heads * w.head_dim * esz if w.dtype == "bf16" else 0
         assert qb <= lay.part - lay.qblk < qb + 1024
         part = 148 * 2 * (256 * 128 + 512) * 4 if w.dtype == "bf16" else 0
-        assert part <= lay.cnt - lay.part < part + 1024
-        pairs = -(-w.block_frames * w.tokens // 256)
-        cnt = w.rollouts * w.heads * pairs * 4 if w.dtype == "bf16" else 0
-        assert cnt <= lay.pos - lay.cnt < cnt + 1024
+        assert part <= lay.pos - lay.part < part + 1024
         # one work set per layer multiplies the three by L and nothing else
         lay_l = fd.fd_cache_get_layout(fd.make_desc(w, work_sets=w.layers))
         assert lay_l.qblk - lay_l.kblk >= w.layers * blk
         assert lay_l.part - lay_l.qblk >= w.layers * qb
-        assert lay_l.cnt - lay_l.part >= w.layers * part
-        assert lay_l.pos - lay_l.cnt >= w.layers * cnt
-        assert (lay_l.total - lay.total) - (w.layers - 1) * (blk + qb + part + cnt) < 4 * 1024
+        assert lay_l.pos - lay_l.part >= w.layers * part
+        assert (lay_l.total - lay.total) - (w.layers - 1) * (blk + qb + part) < 4 * 1024
         assert (lay.rope_pairs_t, lay.rope_pairs_h, lay.rope_pairs_w) == \
             (w.head_dim // 2 - 2 * (w.head_dim // 6), w.head_dim // 6, w.head_dim // 6)
 
