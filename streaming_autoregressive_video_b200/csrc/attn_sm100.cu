@@ -111,9 +111,13 @@ struct Geo {
   static constexpr uint32_t kOffV = kOffK + kKStages * kTile;
   static constexpr uint32_t kOffShared = kOffV + kVStages * kTile;
   static constexpr uint32_t kOffMeta = kOffShared + 256;  // struct Meta
-  static constexpr uint32_t kSmemFixed = kOffMeta + 256 + 1024;  // + base alignment slack
+  // epilogue staging: 4 KB per softmax warp (32 rows x 64 bf16 columns)
+  static constexpr uint32_t kOffStage = kOffMeta + 256;
+  static constexpr uint32_t kStageWarp = 32 * 64 * 2;
+  static constexpr uint32_t kSmemFixed = kOffStage + 8 * kStageWarp + 1024;  // + alignment slack
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, D, true);
 };
+static_assert(Geo<128>::kSmemFixed <= kSmemMax, "shared memory of the d = 128 kernel");
 
 // Site codes for the device error word.
 enum : int { kSiteProducer = 1, kSiteMma = 3, kSiteSoftmax = 4,
@@ -431,6 +435,11 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   const int n_pieces = meta->n_pieces;
+  // launched as a programmatic dependent of the pass that rotates the
+  // block's queries and keys: wait for it before any copy, then let the fold
+  // kernel that follows start on multiprocessors this grid leaves
+  griddep_wait();
+  griddep_launch_dependents();
 
   // Register split (launch: 512 threads x 128): the producer/MMA warpgroup and
   // the idle warpgroup 1 give registers to the two softmax warpgroups, which
@@ -794,38 +803,59 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
         // row, running max, row sum) to the fold that runs after this kernel
         float* part = p.part + ((size_t)blockIdx.x * 2 +
                                 (pi.U0 + pi.kv0 == meta->my_begin ? 0 : 1)) * kPartSlotFloats;
+        // O in column-chunk-major order ([D/4][256 rows][4 columns]): the
+        // 32 lanes of a warp hold consecutive rows, so each store of a warp
+        // covers 512 contiguous bytes
         uint32_t rr[32];
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           tmem_ld32(tO + c * 32, rr);
-          float4* dst = reinterpret_cast<float4*>(part + (size_t)row * D + c * 32);
+          float4* dst = reinterpret_cast<float4*>(part) + (size_t)c * 8 * 2 * kBM + row;
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
-                                 __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3]));
+            dst[i * 2 * kBM] =
+                make_float4(__uint_as_float(rr[4 * i]), __uint_as_float(rr[4 * i + 1]),
+                            __uint_as_float(rr[4 * i + 2]), __uint_as_float(rr[4 * i + 3]));
         }
         part[2 * kBM * D + row] = m;
         part[2 * kBM * D + 2 * kBM + row] = l;
       } else {
-        // a whole unit: O / l in bf16 (and the log-sum-exp)
+        // a whole unit: O / l in bf16 (and the log-sum-exp).  Each warp
+        // stages its 32 rows 64 columns at a time in shared memory (16-byte
+        // chunks XOR-swizzled by row) and writes them back four rows per
+        // store, 128 contiguous bytes a row, instead of one row per lane.
         const float inv_l = 1.f / l;
-        uint16_t* out = static_cast<uint16_t*>(p.out) +
-                        (((size_t)pi.r * p.Mq + qrow) * p.H + pi.h) * D;
+        uint8_t* stage = smem + G::kOffStage + (warp - 8) * G::kStageWarp;
+        const int qrow_w = pi.b * 2 * kBM + x * kBM + wq * 32;  // the warp's first row
         uint32_t rr[32];
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tO + c * 32, rr);
-          if (qrow < p.Mq) {
-            uint32_t pk[16];
+        for (int hf = 0; hf < D / 64; ++hf) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l,
-                                __uint_as_float(rr[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+          for (int c2 = 0; c2 < 2; ++c2) {
+            tmem_ld32(tO + hf * 64 + c2 * 32, rr);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) {
+              const uint4 v = make_uint4(
+                  pack_bf16(__uint_as_float(rr[8 * i]) * inv_l, __uint_as_float(rr[8 * i + 1]) * inv_l),
+                  pack_bf16(__uint_as_float(rr[8 * i + 2]) * inv_l, __uint_as_float(rr[8 * i + 3]) * inv_l),
+                  pack_bf16(__uint_as_float(rr[8 * i + 4]) * inv_l, __uint_as_float(rr[8 * i + 5]) * inv_l),
+                  pack_bf16(__uint_as_float(rr[8 * i + 6]) * inv_l, __uint_as_float(rr[8 * i + 7]) * inv_l));
+              const int chunk = c2 * 4 + i;
+              *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = v;
+            }
           }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rw = i * 4 + (lane >> 3), cc = lane & 7;
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + rw * 128 + ((cc ^ (rw & 7)) << 4));
+            const int qr = qrow_w + rw;
+            if (qr < p.Mq)
+              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                                        (((size_t)pi.r * p.Mq + qr) * p.H + pi.h) * D + hf * 64 +
+                                        cc * 8) = v;
+          }
+          __syncwarp();
         }
         if (p.lse != nullptr && qrow < p.Mq)
           p.lse[((size_t)pi.r * p.H + pi.h) * p.Mq + qrow] =
@@ -883,19 +913,20 @@ cudaError_t prepare_kernel(AttnKernel k) {
 // on which CTA finished first), M the largest max, written in bf16 with the
 // log-sum-exp.  It runs after the attention kernel on the same stream, so
 // every piece's slot is complete; no CTA of the attention kernel waits or
-// folds.  A block takes 32 of a split unit's 256 rows: 8 warps x 4 rows, a
-// warp reads a row of a piece with one load per lane (D / 32 columns a
-// lane), the 4 rows' loads in flight together.
-constexpr int kFoldRows = 32;      // rows per block
-constexpr int kFoldRowsPerWarp = 4;
+// folds.  A block takes 32 of a split unit's 256 rows: lane = row, warp w =
+// the w-th eighth of the columns (D/32 four-column chunks), so every load of
+// a warp reads 512 contiguous bytes of a slot; the bf16 rows are staged in
+// shared memory and written row by row.
+constexpr int kFoldRows = 32;  // rows per block
 
 template <int D>
 __global__ void __launch_bounds__(256)
     fold_split_units(const __grid_constant__ AttnParams p) {
-  constexpr int kPerLane = D / 32;
+  constexpr int kChunks = D / 32;  // four-column chunks per thread
   constexpr size_t kOffM = 2 * kBM * D, kOffL = kOffM + 2 * kBM;
   __shared__ Sched s_sd;
   __shared__ int s_unit[6];  // r, h, b, U0, c_lo, c_hi (c_lo == c_hi: nothing to fold)
+  __shared__ __align__(16) uint16_t s_out[kFoldRows][D];
   if (threadIdx.x == 0) {
     const Sched sd = make_sched(p);
     const int per_r = p.H * p.nb;
@@ -915,67 +946,62 @@ __global__ void __launch_bounds__(256)
     s_unit[5] = nt > 0 ? cta_of(U0 + nt - 1, sd, p.G) : 0;
   }
   __syncthreads();
+  // every block waits for the attention kernel (also those with nothing to
+  // fold), so this grid completes after it and work later on the stream sees
+  // both kernels' rows
+  griddep_wait();
   const int c_lo = s_unit[4], c_hi = s_unit[5];
   if (c_lo == c_hi) return;  // whole: the attention kernel wrote its rows
   const Sched sd = s_sd;
   const int r = s_unit[0], h = s_unit[1], b = s_unit[2], U0 = s_unit[3];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row0 = ((int)blockIdx.x % (2 * kBM / kFoldRows)) * kFoldRows + warp * kFoldRowsPerWarp;
+  const int row_b = ((int)blockIdx.x % (2 * kBM / kFoldRows)) * kFoldRows;  // block's first row
+  const int row = row_b + lane;
+  const int ch0 = warp * kChunks;  // first chunk of this thread
   auto piece = [&](int c) { return cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G); };
-  float M[kFoldRowsPerWarp], L[kFoldRowsPerWarp], acc[kFoldRowsPerWarp][kPerLane];
+  float M = -INFINITY, L = 0.f;
+  float4 acc[kChunks];
 #pragma unroll
-  for (int i = 0; i < kFoldRowsPerWarp; ++i) {
-    M[i] = -INFINITY;
-    L[i] = 0.f;
-#pragma unroll
-    for (int e = 0; e < kPerLane; ++e) acc[i][e] = 0.f;
-  }
+  for (int e = 0; e < kChunks; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c = c_lo; c <= c_hi; ++c)
+    if (piece(c)) M = fmaxf(M, __ldcg(part_slot(p, c, U0, sd) + kOffM + row));
   for (int c = c_lo; c <= c_hi; ++c) {
     if (!piece(c)) continue;
     const float* sl = part_slot(p, c, U0, sd);
+    const float mv = __ldcg(sl + kOffM + row), lv = __ldcg(sl + kOffL + row);
+    float4 ov[kChunks];
 #pragma unroll
-    for (int i = 0; i < kFoldRowsPerWarp; ++i) M[i] = fmaxf(M[i], __ldcg(sl + kOffM + row0 + i));
-  }
-  for (int c = c_lo; c <= c_hi; ++c) {
-    if (!piece(c)) continue;
-    const float* sl = part_slot(p, c, U0, sd);
-    float mv[kFoldRowsPerWarp], lv[kFoldRowsPerWarp], ov[kFoldRowsPerWarp][kPerLane];
+    for (int e = 0; e < kChunks; ++e)
+      ov[e] = __ldcg(reinterpret_cast<const float4*>(sl) + (size_t)(ch0 + e) * 2 * kBM + row);
+    const float w = mv == M ? 1.f : ex2_approx(mv - M);
+    L += lv * w;
 #pragma unroll
-    for (int i = 0; i < kFoldRowsPerWarp; ++i) {
-      mv[i] = __ldcg(sl + kOffM + row0 + i);
-      lv[i] = __ldcg(sl + kOffL + row0 + i);
-      const float* o = sl + (size_t)(row0 + i) * D + lane * kPerLane;
-      if constexpr (kPerLane == 4) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(o));
-        ov[i][0] = f.x; ov[i][1] = f.y; ov[i][2] = f.z; ov[i][3] = f.w;
-      } else {
-        const float2 f = __ldcg(reinterpret_cast<const float2*>(o));
-        ov[i][0] = f.x; ov[i][1] = f.y;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kFoldRowsPerWarp; ++i) {
-      const float w = mv[i] == M[i] ? 1.f : ex2_approx(mv[i] - M[i]);
-      L[i] += lv[i] * w;
-#pragma unroll
-      for (int e = 0; e < kPerLane; ++e) acc[i][e] += w * ov[i][e];
+    for (int e = 0; e < kChunks; ++e) {
+      acc[e].x += w * ov[e].x;
+      acc[e].y += w * ov[e].y;
+      acc[e].z += w * ov[e].z;
+      acc[e].w += w * ov[e].w;
     }
   }
+  const float inv_l = 1.f / L;
 #pragma unroll
-  for (int i = 0; i < kFoldRowsPerWarp; ++i) {
-    const int qrow = b * 2 * kBM + row0 + i;
-    if (qrow >= p.Mq) continue;
-    const float inv_l = 1.f / L[i];
-    uint16_t* out = static_cast<uint16_t*>(p.out) + (((size_t)r * p.Mq + qrow) * p.H + h) * D +
-                    lane * kPerLane;
-    if constexpr (kPerLane == 4) {
-      *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16(acc[i][0] * inv_l, acc[i][1] * inv_l),
-                                                  pack_bf16(acc[i][2] * inv_l, acc[i][3] * inv_l));
-    } else {
-      *reinterpret_cast<uint32_t*>(out) = pack_bf16(acc[i][0] * inv_l, acc[i][1] * inv_l);
-    }
-    if (p.lse != nullptr && lane == 0)
-      p.lse[((size_t)r * p.H + h) * p.Mq + qrow] = (M[i] + log2f(L[i])) * 0.69314718055994530942f;
+  for (int e = 0; e < kChunks; ++e)
+    *reinterpret_cast<uint2*>(&s_out[lane][(ch0 + e) * 4]) =
+        make_uint2(pack_bf16(acc[e].x * inv_l, acc[e].y * inv_l),
+                   pack_bf16(acc[e].z * inv_l, acc[e].w * inv_l));
+  const int qrow = b * 2 * kBM + row;
+  if (warp == 0 && p.lse != nullptr && qrow < p.Mq)
+    p.lse[((size_t)r * p.H + h) * p.Mq + qrow] = (M + log2f(L)) * 0.69314718055994530942f;
+  __syncthreads();
+  // rows of D bf16 = D / 8 sixteen-byte vectors; the block's 256 threads
+  // write 256 vectors per round
+  constexpr int kVecRow = D / 8;
+  for (int t = threadIdx.x; t < kFoldRows * kVecRow; t += 256) {
+    const int i = t / kVecRow, v = t % kVecRow;
+    const int q = b * 2 * kBM + row_b + i;
+    if (q >= p.Mq) continue;
+    uint16_t* out = static_cast<uint16_t*>(p.out) + (((size_t)r * p.Mq + q) * p.H + h) * D;
+    reinterpret_cast<uint4*>(out)[v] = *reinterpret_cast<const uint4*>(&s_out[i][v * 8]);
   }
 }
 
@@ -1002,24 +1028,32 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
   const size_t smem = attn_bf16_smem_bytes(p);
   if (smem == 0) return cudaErrorNotSupported;
   if (p.G < 1 || p.G > kAttnMaxCtas) return cudaErrorInvalidValue;
-  if (p.d == 128)
-    attn_bf16_d128_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
-  else
-    attn_bf16_d64_sm100<<<p.G, kThreads, smem, s>>>(tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
+  // both kernels start as programmatic dependents of the kernel before them
+  // on the stream (each waits for it on the device before reading its data)
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.G);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e2 = cudaLaunchKernelEx(&cfg, p.d == 128 ? attn_bf16_d128_sm100 : attn_bf16_d64_sm100,
+                                      tm_q, tm_kc, tm_vc, tm_kb, tm_vb, p);
   count_launch(1);
-  cudaError_t e2 = cudaGetLastError();
   if (e2 != cudaSuccess) return e2;
   // the units past the whole-unit waves may be split between CTAs: fold them
   const int64_t units = (int64_t)p.n_rollouts * p.H * p.nb;
   const int64_t split = units - units / p.G * p.G;
   if (split == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)(split * (2 * kBM / kFoldRows));
-  if (p.d == 128)
-    fold_split_units<128><<<blocks, 256, 0, s>>>(p);
-  else
-    fold_split_units<64><<<blocks, 256, 0, s>>>(p);
+  cfg.gridDim = dim3((unsigned)(split * (2 * kBM / kFoldRows)));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  e2 = cudaLaunchKernelEx(&cfg, p.d == 128 ? fold_split_units<128> : fold_split_units<64>, p);
   count_launch(1);
-  return cudaGetLastError();
+  return e2;
 }
 
 }  // namespace fd

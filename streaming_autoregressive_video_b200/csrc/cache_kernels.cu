@@ -290,6 +290,9 @@ template <typename Elem>
 __global__ void __launch_bounds__(256)
     rope3d_kernel(CacheView c, int layer, RopeJob<Elem> j0, RopeJob<Elem> j1) {
   constexpr int kPer = 16 / sizeof(Elem);  // elements per 16-byte chunk
+  // the attention kernel that follows may take multiprocessors this grid has
+  // left (it waits for this grid's completion before reading its rows)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint32_t cpr = c.d / kPer;         // chunks per head row
   const uint32_t rows_all = j0.rows + j1.rows;
   const uint32_t warps = gridDim.x * (blockDim.x >> 5);
