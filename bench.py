@@ -588,8 +588,9 @@ def run_fd(args, w, rank, world, local_rank):
                 "peak_source": f"{src} bf16_tflops (burst)",
                 "algorithmic_bytes_per_launch": ro.bytes_call,
                 "flops_per_launch": ro.flops_call, "launch_ms": attn_ms,
-                "launch_covers": "fd_block_attention call: block-key RoPE pass + attention "
-                                 "kernel"}
+                "launch_covers": "fd_block_attention call: RoPE pass over the block's "
+                                 "queries and keys + attention kernel + fold of the "
+                                 "split query-tile pairs"}
     else:
         achieved = ro.bytes_call / (attn_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
