@@ -72,10 +72,14 @@ constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 2^8
 // Every kPolyEvery-th pair of exponentials on the FMA pipe (0: all on MUFU).
-// With one warpgroup per query tile the MUFU unit is not the limit and the
-// polynomial's extra instructions cost more than they save (measured: 505 us
-// per 480p call all on MUFU, 521 us with every second pair on the FMA pipe).
-constexpr int kPolyEvery = 0;
+// At D = 128 the polynomial's extra instructions cost more than the MUFU time
+// they free (measured: 505 us per 480p call all on MUFU, 521 us with every
+// second pair on the FMA pipe).  At D = 64 the tensor work per tile halves
+// while the exponentials stay, so MUFU is the limit and every third pair on
+// the FMA pipe pays (0.805 -> 0.763 ms per 24-head 480p call; every second
+// pair 0.859, every fourth 0.773).
+template <int D>
+constexpr int kPolyEvery = D == 64 ? 3 : 0;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s
 
@@ -756,8 +760,8 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
             const uint64_t x2 = f2_fma(
                 f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nm2);
             uint64_t e2;
-            constexpr int kEvery = kPolyEvery > 0 ? kPolyEvery : 1;
-            if (kPolyEvery > 0 && full && (i % kEvery) == kEvery - 1) {
+            constexpr int kEvery = kPolyEvery<D> > 0 ? kPolyEvery<D> : 1;
+            if (kPolyEvery<D> > 0 && full && (i % kEvery) == kEvery - 1) {
               e2 = exp2_poly2(x2);
             } else {
               float x0, x1;
@@ -959,28 +963,59 @@ __global__ void __launch_bounds__(256)
   const int row = row_b + lane;
   const int ch0 = warp * kChunks;  // first chunk of this thread
   auto piece = [&](int c) { return cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G); };
+  // pieces in groups of four, every load of a group in flight together; M
+  // is the running max over the groups so far (one group in practice: a
+  // unit is split between at most a few CTAs)
+  constexpr int kGroup = 4;
   float M = -INFINITY, L = 0.f;
   float4 acc[kChunks];
 #pragma unroll
   for (int e = 0; e < kChunks; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c = c_lo; c <= c_hi; ++c)
-    if (piece(c)) M = fmaxf(M, __ldcg(part_slot(p, c, U0, sd) + kOffM + row));
-  for (int c = c_lo; c <= c_hi; ++c) {
-    if (!piece(c)) continue;
-    const float* sl = part_slot(p, c, U0, sd);
-    const float mv = __ldcg(sl + kOffM + row), lv = __ldcg(sl + kOffL + row);
-    float4 ov[kChunks];
+  for (int c0 = c_lo; c0 <= c_hi; c0 += kGroup) {
+    bool has[kGroup];
+    float mv[kGroup], lv[kGroup];
+    float4 ov[kGroup][kChunks];
 #pragma unroll
-    for (int e = 0; e < kChunks; ++e)
-      ov[e] = __ldcg(reinterpret_cast<const float4*>(sl) + (size_t)(ch0 + e) * 2 * kBM + row);
-    const float w = mv == M ? 1.f : ex2_approx(mv - M);
-    L += lv * w;
+    for (int i = 0; i < kGroup; ++i) {
+      has[i] = c0 + i <= c_hi && piece(c0 + i);
+      mv[i] = -INFINITY;
+      lv[i] = 0.f;
+      if (has[i]) {
+        const float* sl = part_slot(p, c0 + i, U0, sd);
+        mv[i] = __ldcg(sl + kOffM + row);
+        lv[i] = __ldcg(sl + kOffL + row);
 #pragma unroll
-    for (int e = 0; e < kChunks; ++e) {
-      acc[e].x += w * ov[e].x;
-      acc[e].y += w * ov[e].y;
-      acc[e].z += w * ov[e].z;
-      acc[e].w += w * ov[e].w;
+        for (int e = 0; e < kChunks; ++e)
+          ov[i][e] = __ldcg(reinterpret_cast<const float4*>(sl) + (size_t)(ch0 + e) * 2 * kBM + row);
+      }
+    }
+    float Mg = M;
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) Mg = fmaxf(Mg, mv[i]);
+    if (Mg > M) {  // rescale what earlier groups left (nothing in the first group)
+      const float sc = ex2_approx(M - Mg);
+      L *= sc;
+#pragma unroll
+      for (int e = 0; e < kChunks; ++e) {
+        acc[e].x *= sc;
+        acc[e].y *= sc;
+        acc[e].z *= sc;
+        acc[e].w *= sc;
+      }
+      M = Mg;
+    }
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) {
+      if (!has[i]) continue;
+      const float w = mv[i] == M ? 1.f : ex2_approx(mv[i] - M);
+      L += lv[i] * w;
+#pragma unroll
+      for (int e = 0; e < kChunks; ++e) {
+        acc[e].x += w * ov[i][e].x;
+        acc[e].y += w * ov[i][e].y;
+        acc[e].z += w * ov[i][e].z;
+        acc[e].w += w * ov[i][e].w;
+      }
     }
   }
   const float inv_l = 1.f / L;
