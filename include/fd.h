@@ -241,7 +241,12 @@ fd_status fd_rope3d(const fd_cache* cache, int32_t layer, int32_t n_rollouts,
  * ceil(F*T/256) x (ceil((S+W)*Tf/128) + ceil(F*Tf/128)) x CTAs reaches 2^31.
  * A query-tile pair split between CTAs leaves its pieces in the work set's
  * `part` region; a fold kernel launched right after the attention kernel
- * combines them (a fixed order: results do not depend on timing).
+ * combines them (a fixed order: results do not depend on timing).  The
+ * attention and fold kernels are launched as programmatic dependents of the
+ * kernel before them on the stream: each starts its prologue early and waits
+ * on the device for its predecessor before reading that kernel's output, and
+ * every block of the fold waits for the attention kernel, so work enqueued
+ * after the call sees all of its results as with plain stream order.
  * Device-side waits are bounded: a wait that gives up sets the error word
  * (fd_get_device_error) instead of hanging. */
 fd_status fd_block_attention(fd_cache* cache, int32_t layer,
