@@ -55,6 +55,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "attn_sched.cuh"
 #include "fd_internal.h"
 #include "sm100.cuh"
 
@@ -62,10 +63,9 @@ namespace fd {
 namespace {
 
 using namespace sm100;
+using namespace attn;
 
 constexpr int kThreads = 512;
-constexpr int kBM = 128;  // query rows per tile
-constexpr int kBN = 128;  // keys per tile
 // one 64-column, 128-byte-swizzled half of a tile: 128 rows x 128 bytes
 constexpr uint32_t kHalf = kBM * 64 * 2;
 constexpr int kKStages = 2;
@@ -161,136 +161,6 @@ __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
   }
 }
 
-struct TileCounts {
-  int n1, n2, nt1, nt;
-};
-
-__device__ __forceinline__ TileCounts tile_counts(const AttnParams& p, int r) {
-  TileCounts t;
-  const int nv = valid_slots_local(valid_slots_global(p.count[r], p.S, p.W), p.N, p.shard);
-  t.n1 = nv * p.Tf;
-  t.n2 = p.shard == 0 ? p.F * p.Tf : 0;  // the block's keys belong to shard 0
-  t.nt1 = (t.n1 + kBN - 1) / kBN;
-  t.nt = t.nt1 + (t.n2 + kBN - 1) / kBN;
-  return t;
-}
-
-// ---------------------------------------------------------------- schedule
-// Work unit u = (rollout, head, pair) in that order; unit u has nt(rollout)
-// KV iterations.  With U units and G CTAs, the first W = floor(U / G) waves
-// run whole units (CTA c takes units c, c + G, ...: the CTAs of one head
-// stream the same K/V tiles at the same time, so most of them come from L2);
-// the iterations of the remaining U - W*G units, laid end to end, are cut
-// into G equal ranges, one per CTA (its range starts at the SK iteration
-// sk0 + c * I2 / G of the call's iteration space).  The host bounds the
-// call's iterations so that iterations x G < 2^31: all of this is 32-bit.
-struct Sched {
-  int W;    // whole-unit waves
-  int sk0;  // first iteration of the split part
-  int I2;   // iterations of the split part
-};
-
-__device__ __forceinline__ Sched make_sched(const AttnParams& p) {
-  const int per_r = p.H * p.nb;
-  Sched s;
-  s.W = p.n_rollouts * per_r / p.G;
-  const int D = s.W * p.G;  // units run whole
-  int total = 0, below = 0;
-  for (int r = 0; r < p.n_rollouts; ++r) {
-    const int nt = tile_counts(p, r).nt;
-    total += per_r * nt;
-    below += min(max(D - r * per_r, 0), per_r) * nt;
-  }
-  s.sk0 = below;
-  s.I2 = total - below;
-  return s;
-}
-
-// First iteration of CTA c's split range.
-__device__ __forceinline__ int cta_begin(int c, const Sched& s, int G) {
-  return s.sk0 + c * s.I2 / G;
-}
-
-// The (non-empty) CTA whose split range holds iteration x.
-__device__ __forceinline__ int cta_of(int x, const Sched& s, int G) {
-  return ((x - s.sk0 + 1) * G - 1) / s.I2;
-}
-
-// One unit's share of a CTA's work: KV tiles [kv0, kv1) of query-tile pair
-// b of (rollout r, head h); the unit's iterations start at U0.
-struct Piece {
-  int r, h, b, kv0, kv1, unit, U0;
-  TileCounts tc;
-};
-
-struct Cursor {
-  int w;        // next whole-unit wave
-  int it, end;  // next iteration, end of this CTA's split range
-  int base;     // first iteration of rollout r
-  int r;
-  TileCounts tc;
-};
-
-__device__ __forceinline__ Cursor cursor_init(const AttnParams& p, const Sched& s) {
-  Cursor c;
-  c.w = 0;
-  c.it = cta_begin(blockIdx.x, s, p.G);
-  c.end = cta_begin(blockIdx.x + 1, s, p.G);
-  c.base = 0;
-  c.r = 0;
-  c.tc = tile_counts(p, 0);
-  return c;
-}
-
-// Next piece of this CTA's work, or false at its end.
-__device__ __forceinline__ bool next_piece(const AttnParams& p, const Sched& s,
-                                           Cursor& c, Piece& pc) {
-  const int per_r = p.H * p.nb;
-  while (c.w < s.W) {  // a whole unit
-    const int unit = c.w * p.G + blockIdx.x;
-    ++c.w;
-    pc.r = unit / per_r;
-    const int u = unit - pc.r * per_r;
-    pc.tc = tile_counts(p, pc.r);
-    if (pc.tc.nt == 0) continue;  // a shard with no key of this rollout
-    pc.h = u / p.nb;
-    pc.b = u - pc.h * p.nb;
-    pc.kv0 = 0;
-    pc.kv1 = pc.tc.nt;
-    pc.unit = unit;
-    pc.U0 = -1;  // not used by whole units
-    return true;
-  }
-  if (c.it >= c.end) return false;
-  int span = per_r * c.tc.nt;
-  while (c.it >= c.base + span && c.r + 1 < p.n_rollouts) {
-    c.base += span;
-    ++c.r;
-    c.tc = tile_counts(p, c.r);
-    span = per_r * c.tc.nt;
-  }
-  const int rel = c.it - c.base;
-  const int u = rel / c.tc.nt;
-  pc.r = c.r;
-  pc.tc = c.tc;
-  pc.h = u / p.nb;
-  pc.b = u - pc.h * p.nb;
-  pc.U0 = c.base + u * c.tc.nt;
-  pc.kv0 = c.it - pc.U0;
-  pc.kv1 = min(c.tc.nt, c.end - pc.U0);
-  pc.unit = c.r * per_r + u;
-  c.it = pc.U0 + pc.kv1;
-  return true;
-}
-
-// Partial-result slot of CTA c's piece of the split unit starting at U0:
-// slot 0 when the piece opens the CTA's split range, slot 1 when it closes it.
-__device__ __forceinline__ const float* part_slot(const AttnParams& p, int c,
-                                                  int U0, const Sched& s) {
-  const int slot = cta_begin(c, s, p.G) >= U0 ? 0 : 1;
-  return p.part + ((size_t)c * 2 + slot) * kPartSlotFloats;
-}
-
 // What every role needs to know about a piece.  The producer walks the
 // schedule and publishes each piece in a 4-entry ring in shared memory
 // (entry k & 3, `seq` = k written last); the other roles read the entry
@@ -319,10 +189,6 @@ __device__ __forceinline__ void teardown(int warp, uint32_t tmem) {
   if (warp == 2) tmem_dealloc(tmem, 512);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
 
 // Reads ring entry k once the producer has published it (bounded wait).
 __device__ __forceinline__ bool read_piece(const Meta* meta, int k, PieceInfo& pi,
@@ -911,135 +777,6 @@ cudaError_t prepare_kernel(AttnKernel k) {
                               (int)kSmemMax);
 }
 
-// Folds the pieces of the query-tile pairs that the persistent kernel split
-// between CTAs: row = sum_i O_i 2^(m_i - M) / sum_i l_i 2^(m_i - M) over the
-// unit's pieces i in CTA order (a fixed order, so the rounding does not depend
-// on which CTA finished first), M the largest max, written in bf16 with the
-// log-sum-exp.  It runs after the attention kernel on the same stream, so
-// every piece's slot is complete; no CTA of the attention kernel waits or
-// folds.  A block takes 32 of a split unit's 256 rows: lane = row, warp w =
-// the w-th eighth of the columns (D/32 four-column chunks), so every load of
-// a warp reads 512 contiguous bytes of a slot; the bf16 rows are staged in
-// shared memory and written row by row.
-constexpr int kFoldRows = 32;  // rows per block
-
-template <int D>
-__global__ void __launch_bounds__(256)
-    fold_split_units(const __grid_constant__ AttnParams p) {
-  constexpr int kChunks = D / 32;  // four-column chunks per thread
-  constexpr size_t kOffM = 2 * kBM * D, kOffL = kOffM + 2 * kBM;
-  __shared__ Sched s_sd;
-  __shared__ int s_unit[6];  // r, h, b, U0, c_lo, c_hi (c_lo == c_hi: nothing to fold)
-  __shared__ __align__(16) uint16_t s_out[kFoldRows][D];
-  if (threadIdx.x == 0) {
-    const Sched sd = make_sched(p);
-    const int per_r = p.H * p.nb;
-    const int unit = sd.W * p.G + (int)blockIdx.x / (2 * kBM / kFoldRows);
-    const int r = unit / per_r;
-    int U0 = 0;  // the unit's first iteration: the iterations of the units before it
-    for (int rr = 0; rr < r; ++rr) U0 += per_r * tile_counts(p, rr).nt;
-    const int nt = tile_counts(p, r).nt;
-    U0 += (unit - r * per_r) * nt;
-    const int u = unit - r * per_r;
-    s_sd = sd;
-    s_unit[0] = r;
-    s_unit[1] = u / p.nb;
-    s_unit[2] = u - (u / p.nb) * p.nb;
-    s_unit[3] = U0;
-    s_unit[4] = nt > 0 ? cta_of(U0, sd, p.G) : 0;
-    s_unit[5] = nt > 0 ? cta_of(U0 + nt - 1, sd, p.G) : 0;
-  }
-  __syncthreads();
-  // every block waits for the attention kernel (also those with nothing to
-  // fold), so this grid completes after it and work later on the stream sees
-  // both kernels' rows
-  griddep_wait();
-  const int c_lo = s_unit[4], c_hi = s_unit[5];
-  if (c_lo == c_hi) return;  // whole: the attention kernel wrote its rows
-  const Sched sd = s_sd;
-  const int r = s_unit[0], h = s_unit[1], b = s_unit[2], U0 = s_unit[3];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row_b = ((int)blockIdx.x % (2 * kBM / kFoldRows)) * kFoldRows;  // block's first row
-  const int row = row_b + lane;
-  const int ch0 = warp * kChunks;  // first chunk of this thread
-  auto piece = [&](int c) { return cta_begin(c, sd, p.G) < cta_begin(c + 1, sd, p.G); };
-  // pieces in groups of four, every load of a group in flight together; M
-  // is the running max over the groups so far (one group in practice: a
-  // unit is split between at most a few CTAs)
-  constexpr int kGroup = 4;
-  float M = -INFINITY, L = 0.f;
-  float4 acc[kChunks];
-#pragma unroll
-  for (int e = 0; e < kChunks; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = c_lo; c0 <= c_hi; c0 += kGroup) {
-    bool has[kGroup];
-    float mv[kGroup], lv[kGroup];
-    float4 ov[kGroup][kChunks];
-#pragma unroll
-    for (int i = 0; i < kGroup; ++i) {
-      has[i] = c0 + i <= c_hi && piece(c0 + i);
-      mv[i] = -INFINITY;
-      lv[i] = 0.f;
-      if (has[i]) {
-        const float* sl = part_slot(p, c0 + i, U0, sd);
-        mv[i] = __ldcg(sl + kOffM + row);
-        lv[i] = __ldcg(sl + kOffL + row);
-#pragma unroll
-        for (int e = 0; e < kChunks; ++e)
-          ov[i][e] = __ldcg(reinterpret_cast<const float4*>(sl) + (size_t)(ch0 + e) * 2 * kBM + row);
-      }
-    }
-    float Mg = M;
-#pragma unroll
-    for (int i = 0; i < kGroup; ++i) Mg = fmaxf(Mg, mv[i]);
-    if (Mg > M) {  // rescale what earlier groups left (nothing in the first group)
-      const float sc = ex2_approx(M - Mg);
-      L *= sc;
-#pragma unroll
-      for (int e = 0; e < kChunks; ++e) {
-        acc[e].x *= sc;
-        acc[e].y *= sc;
-        acc[e].z *= sc;
-        acc[e].w *= sc;
-      }
-      M = Mg;
-    }
-#pragma unroll
-    for (int i = 0; i < kGroup; ++i) {
-      if (!has[i]) continue;
-      const float w = mv[i] == M ? 1.f : ex2_approx(mv[i] - M);
-      L += lv[i] * w;
-#pragma unroll
-      for (int e = 0; e < kChunks; ++e) {
-        acc[e].x += w * ov[i][e].x;
-        acc[e].y += w * ov[i][e].y;
-        acc[e].z += w * ov[i][e].z;
-        acc[e].w += w * ov[i][e].w;
-      }
-    }
-  }
-  const float inv_l = 1.f / L;
-#pragma unroll
-  for (int e = 0; e < kChunks; ++e)
-    *reinterpret_cast<uint2*>(&s_out[lane][(ch0 + e) * 4]) =
-        make_uint2(pack_bf16(acc[e].x * inv_l, acc[e].y * inv_l),
-                   pack_bf16(acc[e].z * inv_l, acc[e].w * inv_l));
-  const int qrow = b * 2 * kBM + row;
-  if (warp == 0 && p.lse != nullptr && qrow < p.Mq)
-    p.lse[((size_t)r * p.H + h) * p.Mq + qrow] = (M + log2f(L)) * 0.69314718055994530942f;
-  __syncthreads();
-  // rows of D bf16 = D / 8 sixteen-byte vectors; the block's 256 threads
-  // write 256 vectors per round
-  constexpr int kVecRow = D / 8;
-  for (int t = threadIdx.x; t < kFoldRows * kVecRow; t += 256) {
-    const int i = t / kVecRow, v = t % kVecRow;
-    const int q = b * 2 * kBM + row_b + i;
-    if (q >= p.Mq) continue;
-    uint16_t* out = static_cast<uint16_t*>(p.out) + (((size_t)r * p.Mq + q) * p.H + h) * D;
-    reinterpret_cast<uint4*>(out)[v] = *reinterpret_cast<const uint4*>(&s_out[i][v * 8]);
-  }
-}
-
 }  // namespace
 
 size_t attn_bf16_smem_bytes(const AttnParams& p) {
@@ -1063,8 +800,9 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
   const size_t smem = attn_bf16_smem_bytes(p);
   if (smem == 0) return cudaErrorNotSupported;
   if (p.G < 1 || p.G > kAttnMaxCtas) return cudaErrorInvalidValue;
-  // both kernels start as programmatic dependents of the kernel before them
-  // on the stream (each waits for it on the device before reading its data)
+  // launched as a programmatic dependent of the kernel before it on the
+  // stream (the RoPE pass): it waits for that kernel on the device before
+  // reading its rows; the fold that follows is launched the same way
   cudaLaunchAttribute attr_pdl[1];
   attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
@@ -1083,10 +821,7 @@ cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
   const int64_t units = (int64_t)p.n_rollouts * p.H * p.nb;
   const int64_t split = units - units / p.G * p.G;
   if (split == 0) return cudaSuccess;
-  cfg.gridDim = dim3((unsigned)(split * (2 * kBM / kFoldRows)));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  e2 = cudaLaunchKernelEx(&cfg, p.d == 128 ? fold_split_units<128> : fold_split_units<64>, p);
+  e2 = launch_fold_split_units(p, (uint64_t)split, s);
   count_launch(1);
   return e2;
 }

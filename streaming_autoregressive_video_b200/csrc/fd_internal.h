@@ -201,14 +201,20 @@ struct CombineParams {
 };
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 // Dynamic shared memory the tensor-core kernel needs for this call (its
-// fixed stages plus the call's RoPE tables), 0 if that exceeds the limit.
+// operand stages, barriers and epilogue staging), 0 if that exceeds the limit.
 size_t attn_bf16_smem_bytes(const AttnParams& p);
+// Launches the persistent tensor-core attention kernel and, when it splits
+// query-tile pairs between CTAs, the fold of those pairs.
 cudaError_t launch_attn_bf16_sm100(const CUtensorMap& tm_q,
                                    const CUtensorMap& tm_kc,
                                    const CUtensorMap& tm_vc,
                                    const CUtensorMap& tm_kb,
                                    const CUtensorMap& tm_vb,
                                    const AttnParams& p, cudaStream_t s);
+// Folds the split_units query-tile pairs past the whole-unit waves of the
+// attention kernel just launched on `s` (fold.cu).
+cudaError_t launch_fold_split_units(const AttnParams& p, uint64_t split_units,
+                                    cudaStream_t s);
 
 void count_launch(int n);
 cudaError_t launch_bounded_wait_selftest(int32_t* err, uint64_t limit_ns,
