@@ -345,18 +345,19 @@ class Rollout:
         self.qshape = (R, w.queries, H, d)
         self.kshape = (R, F * Tf, w.hkv, d)
         base = replica_seed_base(rank)
-        pk = [gen(synth.seed_of(base, 1, l), self.kshape) for l in range(L)]
-        pv = [gen(synth.seed_of(base, 2, l), self.kshape) for l in range(L)]
+        self._pk = [gen(synth.seed_of(base, 1, l), self.kshape) for l in range(L)]
+        self._pv = [gen(synth.seed_of(base, 2, l), self.kshape) for l in range(L)]
         self.fill = prefill_frames(w, rank)
-        left = list(self.fill)
-        while max(left) > 0:
-            fr = [min(F, x) for x in left]
-            fd.fd_cache_commit(self.cache, 0, L, R, pk, pv, frames=fr)
-            left = [a - b for a, b in zip(left, fr)]
+        self.stream = torch.cuda.current_stream(dev)
+        self._prefill()
         torch.cuda.synchronize()
         # the library's own frame counters agree with the described prefill
         assert [fd.fd_cache_frames(self.cache, 0, r) for r in range(R)] == self.fill
-        del pk, pv
+        # a ragged workload keeps its prefill keys to restore its fill before
+        # every timed block (each block's commit advances every rollout's fill)
+        self.ragged = bool(w.ragged_window)
+        if not self.ragged:
+            del self._pk, self._pv
         self.q = [[gen(synth.seed_of(base, 10, s, l), self.qshape) for l in range(L)]
                   for s in range(S)]
         self.k = [[gen(synth.seed_of(base, 11, s, l), self.kshape) for l in range(L)]
@@ -364,13 +365,33 @@ class Rollout:
         self.v = [[gen(synth.seed_of(base, 12, s, l), self.kshape) for l in range(L)]
                   for s in range(S)]
         self.outs = [torch.empty(self.qshape, dtype=tdt, device=dev) for _ in range(L)]
-        self.stream = torch.cuda.current_stream(dev)
         self.nk = keys_per_rollout(w, self.fill)
         self.flops_call = attn_flops(w, self.nk)
         self.bytes_call = attn_bytes(w, self.nk, self.esz)
         self.kv_bytes = 2 * w.layers * w.rollouts * w.slots * Tf * w.hkv * d * self.esz
         # one block's commit: read k, v; write K, V and the rotated K
         self.commit_bytes = 5.0 * L * R * F * Tf * w.hkv * d * self.esz
+
+    def _prefill(self):
+        from streaming_autoregressive_video_b200 import binding as fd
+        w = self.w
+        left = list(self.fill)
+        while max(left) > 0:
+            fr = [min(w.block_frames, x) for x in left]
+            fd.fd_cache_commit(self.cache, 0, w.layers, w.rollouts, self._pk, self._pv,
+                               frames=fr, stream=self.stream)
+            left = [a - b for a, b in zip(left, fr)]
+
+    def restore_fill(self):
+        """Back to the described ragged fill (reset every rollout, commit the
+        prefill again), so the next block's calls see the same key counts
+        as the first; a no-op for steady-state workloads, whose window stays
+        full as blocks are committed."""
+        from streaming_autoregressive_video_b200 import binding as fd
+        if not self.ragged:
+            return
+        fd.fd_cache_reset(self.cache, list(range(self.w.rollouts)), stream=self.stream)
+        self._prefill()
 
     def _timed(self, fn, evs):
         import torch
@@ -425,24 +446,33 @@ class Rollout:
 
 def time_steps(ro, steps, warmup, world=1, barrier=None):
     """Device time of `steps` blocks after `warmup` untimed ones: (ms per
-    step, mean ms per attention call, mean ms per commit)."""
+    step, mean ms per attention call, mean ms per commit).  A ragged
+    workload's fill is restored before every block, and its step time is
+    the sum of the blocks' own intervals (the restores are not timed)."""
     import torch
     for _ in range(warmup):
+        ro.restore_fill()
         ro.step()
     torch.cuda.synchronize()
     if barrier:
         barrier()
     torch.cuda.synchronize()
-    evs, cevs = [], []
+    evs, cevs, sevs = [], [], []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(ro.stream)
     for _ in range(steps):
+        ro.restore_fill()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(ro.stream)
         ro.step(evs, cevs)
+        b.record(ro.stream)
+        sevs.append((a, b))
     e1.record(ro.stream)
     torch.cuda.synchronize()
     if barrier:
         barrier()
-    ms_step = e0.elapsed_time(e1) / steps
+    ms_step = (sum(a.elapsed_time(b) for a, b in sevs) if ro.ragged
+               else e0.elapsed_time(e1)) / steps
     attn_ms = sum(a.elapsed_time(b) for a, b in evs) / len(evs)
     commit_ms = sum(a.elapsed_time(b) for a, b in cevs) / len(cevs)
     return ms_step, attn_ms, commit_ms
@@ -544,6 +574,7 @@ def run_fd(args, w, rank, world, local_rank):
             dist.barrier()
 
     for _ in range(max(3, args.warmup)):
+        ro.restore_fill()
         ro.step()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank)
@@ -563,9 +594,9 @@ def run_fd(args, w, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, ro.cache, dev, ro.stream, ro.q, ro.k, ro.v, ro.outs,
-                      flops_step, world)
+                      flops_step, world, restore=ro.restore_fill)
     overlap = None
-    if not args.no_extra and world == 1:
+    if not args.no_extra and world == 1 and not ro.ragged:
         overlap = finalize_overlap(ro, 5)
 
     if rank != 0:
@@ -637,7 +668,7 @@ def run_fd(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
+def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world, restore=None):
     """Same steps through the C ABI with the q/k/v of every call copied from
     pinned host memory and every output copied back, inside the timed region.
     Copies run on their own streams so they overlap the kernels.  The host
@@ -671,6 +702,10 @@ def run_e2e(args, w, cache, dev, stream, q, k, v, outs, flops_step, world):
 
     def step():
         nonlocal h2d_bytes, d2h_bytes
+        if restore is not None:
+            # a ragged workload's fill before every block (timed with it: the
+            # end-to-end figure of that workload is slightly pessimistic)
+            restore()
         i = 0
         for s in range(S):
             last = s == S - 1

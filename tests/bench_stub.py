@@ -86,8 +86,16 @@ def _attention(cache, l, R, q, k, v, out, lse=None, stream=None):
     _state["launches"] += 2
 
 
+def _reset(cache, rollout_ids, stream=None):
+    for row in _state["n"]:
+        for r in rollout_ids:
+            row[r] = 0
+    _state["launches"] += 1
+
+
 fd.fd_cache_create = _Cache
 fd.fd_cache_commit = _commit
+fd.fd_cache_reset = _reset
 fd.fd_cache_frames = lambda cache, l, r: _state["n"][l][r]
 fd.fd_block_attention = _attention
 fd.fd_launch_count = lambda: _state["launches"]

@@ -64,8 +64,13 @@ def test_gpu_arm_line_keeps_the_contract(workload):
     assert line["config"]["cache_bytes"] == fd_cache_bytes(w)
     assert line["config"]["kv_bytes"] == 2 * w.layers * w.rollouts * w.slots * \
         w.frame_tokens * w.hkv * w.head_dim * esz
-    fo = line["finalize_overlap"]
-    assert fo["layers"] == w.layers and fo["ms_per_step_side_stream_commits"] > 0
+    if w0.ragged_window:
+        # a ragged fill is restored before every timed block; the background
+        # commit comparison is made on steady-state workloads only
+        assert "finalize_overlap" not in line
+    else:
+        fo = line["finalize_overlap"]
+        assert fo["layers"] == w.layers and fo["ms_per_step_side_stream_commits"] > 0
     if workload == "480p":
         oc = line["other_configs"]
         assert sorted(oc) == ["d64", "large", "long", "ragged", "tiny"]
