@@ -13,16 +13,18 @@
 // (every query tile of a head reads the same keys, and a rotated query tile
 // can be copied straight into the tensor core's operand layout).
 //
-// Schedule (persistent): a work unit is one 256-row query-tile pair of one
-// (rollout, head) against all of the rollout's KV tiles.  The units' KV
-// iterations, laid end to end (rollout, head, pair, KV tile), are cut into G
-// equal ranges, one per CTA and G = one CTA per multiprocessor, so every CTA
-// does the same number of KV tiles (+-1) whatever the number of units: no
-// partly idle last wave.  A unit cut by a range boundary is computed in
-// pieces; every piece leaves its unnormalised rows, row maxima and row sums
-// (fp32) in the work set's partial-result area, and a fold kernel launched
-// right after this one combines the pieces of each split unit in a fixed
-// order and writes its rows.  No CTA ever waits for another.
+// Schedule (persistent, G = one CTA per multiprocessor): a work unit is one
+// 256-row query-tile pair of one (rollout, head) against all of the
+// rollout's KV tiles.  The first floor(U / G) waves run whole units (CTA c
+// takes units c, c + G, ...: the CTAs of one head stream the same K/V tiles
+// together); the KV iterations of the remaining units, laid end to end
+// (rollout, head, pair, KV tile), are cut into G equal ranges, one per CTA,
+// so no SM idles through a partly filled last wave (attn_sched.cuh).  A unit
+// cut by a range boundary is computed in pieces; every piece leaves its
+// unnormalised rows (column-chunk-major), row maxima and row sums (fp32) in
+// the work set's partial-result area, and a fold kernel launched right after
+// this one (fold.cu) combines the pieces of each split unit in a fixed order
+// and writes its rows.  No CTA ever waits for another.
 //
 // Roles (all warps walk the same sequence of pieces):
 //   warp 0        TMA producer: each piece's two Q tiles (once the previous
@@ -44,8 +46,9 @@
 //                 O rescale is skipped unless the running max grows by more
 //                 than 2^8, which keeps P <= 256 and the result exact up to
 //                 rounding.  The epilogue divides by the row sum and writes
-//                 bf16 rows (and the optional log-sum-exp), or hands a split
-//                 unit's piece over as described above.
+//                 bf16 rows staged through shared memory (and the optional
+//                 log-sum-exp), or hands a split unit's piece over as
+//                 described above.
 // Every mbarrier wait is bounded: a wait that gives up raises a CTA-wide
 // abort flag and the device error word, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is released and the CTA exits.
