@@ -34,11 +34,13 @@ sys.path.insert(0, ROOT)
 METRIC = ("chunk-attention TFLOP/s & latent-frames/s per layer; "
           "% of bf16 tensor/HBM roofline")
 PROFILE = os.path.join(ROOT, "profiles", "attn_bf16_d128_sm100.480p.md")
-KERNEL_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
-                          "attn_sm100.cu")
+_CSRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc")
+# a kernel's source files: the .cu and the package headers it includes (the
+# summaries record the sha256 of their bytes concatenated in this order)
+KERNEL_SRCS = [os.path.join(_CSRC, f)
+               for f in ("attn_sm100.cu", "attn_sched.cuh", "sm100.cuh", "fd_internal.h")]
 COMMIT_PROFILE = os.path.join(ROOT, "profiles", "commit_copy_kernel.480p_l30.md")
-COMMIT_SRC = os.path.join(ROOT, "streaming_autoregressive_video_b200", "csrc",
-                          "cache_kernels.cu")
+COMMIT_SRCS = [os.path.join(_CSRC, f) for f in ("cache_kernels.cu", "fd_internal.h")]
 
 
 def workloads():
@@ -93,12 +95,20 @@ def measured_peaks():
             "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _traffic_from(profile, source):
+def sources_sha256(sources):
+    h = hashlib.sha256()
+    for path in sources:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _traffic_from(profile, sources):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (sha256 recorded in the summary)."""
+    the current kernel sources (sha256 recorded in the summary)."""
     try:
         text = open(profile).read()
-        src = hashlib.sha256(open(source, "rb").read()).hexdigest()
+        src = sources_sha256(sources)
     except OSError:
         return None
     m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
@@ -109,11 +119,11 @@ def _traffic_from(profile, source):
 
 
 def profile_traffic():
-    return _traffic_from(PROFILE, KERNEL_SRC)
+    return _traffic_from(PROFILE, KERNEL_SRCS)
 
 
 def commit_traffic():
-    return _traffic_from(COMMIT_PROFILE, COMMIT_SRC)
+    return _traffic_from(COMMIT_PROFILE, COMMIT_SRCS)
 
 
 class ClockSampler:
