@@ -7,6 +7,7 @@ the bench contract.  Used by tests/test_bench_contract.py in a subprocess
     python tests/bench_stub.py <workload> [layers]
 """
 import contextlib
+import json
 import os
 import sys
 import types
@@ -58,7 +59,7 @@ torch.Tensor.pin_memory = lambda self: self
 synth.normal_device = lambda seed, shape, dtype, dev, scale=1.0: torch.zeros(
     shape, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
 
-_state = {"n": None, "launches": 0}
+_state = {"n": None, "launches": 0, "fills": []}
 
 
 class _Cache:
@@ -79,6 +80,7 @@ def _commit(cache, l0, l1, R, ks, vs, frames=None, stream=None):
 
 
 def _attention(cache, l, R, q, k, v, out, lse=None, stream=None):
+    _state["fills"].append(list(_state["n"][l][:R]))  # frames each rollout's call sees
     g = fd._Geom(cache.desc)
     assert q.numel() * q.element_size() == R * g.q
     assert k.numel() * k.element_size() == R * g.kv == v.numel() * v.element_size()
@@ -122,3 +124,5 @@ if __name__ == "__main__":
     args = types.SimpleNamespace(steps=2, warmup=3, no_e2e=False, no_cpu_baseline=True,
                                  gpus=1, no_extra=False, workload=sys.argv[1])
     bench.run_fd(args, w, 0, 1, 0)
+    # the frame counts every attention call saw, for the tests to check
+    print("FILLS " + json.dumps(_state["fills"]), file=sys.stderr)

@@ -17,11 +17,29 @@ import bench  # noqa: E402
 from streaming_autoregressive_video_b200.workloads import Workload  # noqa: E402
 
 
-def _stub_line(workload):
+def _stub_run(workload):
     res = subprocess.run([sys.executable, os.path.join(ROOT, "tests", "bench_stub.py"),
                           workload], capture_output=True, text=True, timeout=600)
     assert res.returncode == 0, res.stderr[-2000:]
-    return json.loads(res.stdout.strip().splitlines()[-1])
+    fills = [json.loads(x[len("FILLS "):]) for x in res.stderr.splitlines()
+             if x.startswith("FILLS ")]
+    return json.loads(res.stdout.strip().splitlines()[-1]), fills[-1]
+
+
+def _stub_line(workload):
+    return _stub_run(workload)[0]
+
+
+def test_ragged_calls_all_see_the_ragged_fill():
+    """Every block's commit adds frames to every rollout; the bench restores
+    a ragged workload's fill before each block, so every attention call (warm
+    up, timed, end to end) sees the fill whose work the line counts."""
+    line, fills = _stub_run("ragged")
+    w = bench.workloads()["ragged"]
+    want = bench.prefill_frames(w, 0)
+    assert len(set(want)) > 1          # the fill really is ragged
+    assert fills and all(f == want for f in fills), fills[:3]
+    assert line["config"]["keys_per_rollout"] == bench.keys_per_rollout(w, want)
 
 
 @pytest.mark.parametrize("workload", ["480p", "gqa", "ragged", "multiview", "tiny"])
