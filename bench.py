@@ -525,7 +525,8 @@ def finalize_overlap(ro, steps):
 # from HBM rather than from L2 (each call has the workload's shape)
 OTHER_CONFIGS = {"tiny": ("tiny", 1, 40), "large": ("large", 4, 4),
                  "long": ("long", 8, 10), "ragged": ("ragged", 1, 10),
-                 "d64": ("d64", 4, 4)}
+                 "d64": ("d64", 4, 4), "gqa": ("gqa", 8, 4),
+                 "multiview": ("multiview", 2, 2)}
 
 
 def other_configs(dev, rank):

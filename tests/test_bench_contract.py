@@ -91,7 +91,7 @@ def test_gpu_arm_line_keeps_the_contract(workload):
         assert fo["layers"] == w.layers and fo["ms_per_step_side_stream_commits"] > 0
     if workload == "480p":
         oc = line["other_configs"]
-        assert sorted(oc) == ["d64", "large", "long", "ragged", "tiny"]
+        assert sorted(oc) == ["d64", "gqa", "large", "long", "multiview", "ragged", "tiny"]
         for name, e in oc.items():
             for key in ("ms_per_call", "tflops_per_call", "frac_of_burst_bf16", "clocks",
                         "commit_frac_of_hbm", "workload"):
