@@ -566,7 +566,39 @@ def other_configs(dev, rank):
         del ro
         gc.collect()
         torch.cuda.empty_cache()
+    res["long"]["rollout"] = whole_rollout(workloads()["long"], dev, rank)
     return res
+
+
+def whole_rollout(w, dev, rank):
+    """The one-frame-per-block workload's whole rollout as the workload states
+    it (its layers, its blocks: 10,000 blocks through the ring), timed on the
+    device from the first block to the last: every block runs its denoising
+    steps and commits, so the ring wraps about 1,250 times.  The device
+    memory the process holds is compared before and after (the cache and the
+    inputs are allocated once)."""
+    import torch
+    ro = Rollout(w, dev, rank)
+    ro.step()
+    torch.cuda.synchronize()
+    mem0 = torch.cuda.memory_allocated(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(ro.stream)
+    for _ in range(w.blocks):
+        ro.step()
+    e1.record(ro.stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    ro.check()
+    out = {"blocks": w.blocks, "layers": w.layers, "steps": w.steps, "ms_total": ms,
+           "ms_per_block": ms / w.blocks,
+           "tflops": ro.flops_call * w.steps * w.layers * w.blocks / (ms * 1e-3) / 1e12,
+           "device_bytes_constant": torch.cuda.memory_allocated(dev) == mem0,
+           "note": "one layer: consecutive blocks read the same layer's cache, "
+                   "partly from L2"}
+    del ro
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_fd(args, w, rank, world, local_rank):

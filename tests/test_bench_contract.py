@@ -97,6 +97,9 @@ def test_gpu_arm_line_keeps_the_contract(workload):
                         "commit_frac_of_hbm", "workload"):
                 assert key in e, (name, key)
         assert oc["tiny"]["dtype"] == "f32" and "us_per_call" in oc["tiny"]
+        ro = oc["long"]["rollout"]   # the 10,000-block rollout, timed whole
+        assert ro["blocks"] == bench.workloads()["long"].blocks == 10000
+        assert ro["device_bytes_constant"] is True and ro["ms_per_block"] > 0
     else:
         assert "other_configs" not in line
 
