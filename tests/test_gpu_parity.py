@@ -209,6 +209,25 @@ def test_attention_bf16_ragged_rollouts():
     ls.attention(0, q[:2], k[:2], v[:2], n_rollouts=2, what="ragged n=2")
 
 
+def test_attention_bf16_many_rollouts():
+    """More rollouts than the fold kernel keeps iteration offsets for in
+    shared memory (64), with ragged fills so the rollouts' units differ in
+    length: 70 single-tile units on at most 148 CTAs, every one split between
+    CTAs and folded, the offsets of rollouts 64-69 recomputed."""
+    w = Workload("many-rollouts-bf16", layers=1, rollouts=70, heads=1, head_dim=128,
+                 grid_h=3, grid_w=4, action_tokens=0, block_frames=2, sink_frames=1,
+                 window_frames=4, steps=1, blocks=1, dtype="bf16")
+    ls = Lockstep(w)
+    rng = np.random.default_rng(5)
+    for blk in range(3):
+        frames = [int(x) for x in rng.integers(0, w.block_frames + 1, w.rollouts)]
+        _commit_block(ls, w, 500 + blk, frames=frames)
+    ls.check_cache_exact()
+    q, k, v = block_inputs(w, (5,), w.rollouts)
+    ls.attention(0, q, k, v, what="70 rollouts")
+    assert fd.fd_get_device_error(ls.cache) == 0
+
+
 def test_softmax_exp2_against_exp2f():
     """The FMA-pipe exponential used for part of the softmax weights agrees
     with CUDA's exp2f (and the exact 2^x) to the fitted polynomial's bound."""
