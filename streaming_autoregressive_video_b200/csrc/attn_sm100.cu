@@ -645,9 +645,20 @@ __device__ __forceinline__ void attn_body(const CUtensorMap& tm_q, const CUtenso
         };
         // bf16 P of columns 0-63 goes to TMEM columns 0-31, of columns
         // 64-127 to columns 32-63 (S columns 64-127 are already in registers)
-        if (valid == kBN) exps(sa, true); else exps(sa, false);
+        // with every exponential on MUFU, a partial tile's masked columns
+        // give exactly 0 and one copy of the loop serves all tiles; with
+        // the FMA-pipe share (d = 64) full and partial tiles get their own
+        if constexpr (kPolyEvery<D> > 0) {
+          if (valid == kBN) exps(sa, true); else exps(sa, false);
+        } else {
+          exps(sa, true);
+        }
         tmem_st32(tS, pk);
-        if (valid == kBN) exps(sb, true); else exps(sb, false);
+        if constexpr (kPolyEvery<D> > 0) {
+          if (valid == kBN) exps(sb, true); else exps(sb, false);
+        } else {
+          exps(sb, true);
+        }
         tmem_st32(tS + 32, pk);
         {
           float la, lb;
